@@ -1,0 +1,388 @@
+"""Benchmark: block-causal ReLU linear attention forward on B200.
+
+One step = one lcla_forward over the whole workload (pass A partial states,
+scan, pass C outputs) with the inputs resident in HBM.  Default workload: the
+480p-like forward (B=1, H=70, d=32, 21 frames x 30x52 tokens = 32760 tokens,
+blocks of 3 frames = 4680 tokens, bf16, 3D rotary tables).  Prints one JSON
+line with the whole-job throughput in attended token-heads per second, the
+end-to-end number through the same call with host buffers, the roofline of
+the dominant kernel, and the fp64 CPU oracle timed on the host as a baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-e2e] [--cpu-seconds S]
+
+N > 1 is launched by torchrun (one rank per GPU): every rank runs its own
+independent copy of the workload (different seed), no data-path collective;
+timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import NAMED, make_inputs  # noqa: E402
+
+METRIC = "attended tokens*heads/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+UNIT = "token*heads/s"
+L2_BYTES = 126 * 1024 * 1024
+STATE_BYTES = 33 * 32 * 4
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="fwd480p_bf16", choices=sorted(NAMED))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def workload_config(spec, world):
+    cfg = {"workload": f"{spec.name}: B={spec.B} H={spec.H} d={spec.d} N={spec.N} "
+                       f"block_len={spec.block_len} ({spec.nblocks} blocks)",
+           "B": spec.B, "H": spec.H, "d": spec.d, "N": spec.N, "block_len": spec.block_len,
+           "rope": spec.rope if spec.grid is None else f"3d t/h/w 8/12/12 on {spec.grid}",
+           "eps": spec.eps, "seed": spec.seed,
+           "parallelism": "single GPU" if world == 1 else f"{world} independent replicas (weak)"}
+    io = 4 * spec.B * spec.N * spec.H * spec.d * spec.elem_bytes
+    cfg["l2"] = (f"inputs larger than L2: {io / 1e6:.0f} MB read+written per step > 126 MB"
+                 if io > L2_BYTES else "inputs smaller than L2: L2 flushed between steps")
+    return cfg
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "block_causal_relu_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, when it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    ent = rec.get("kernels", {}).get(kernel)
+    if not ent or rec.get("source_digest") != source_digest() or ent.get("workload") != workload:
+        return None
+    return ent.get("traffic_bytes_per_launch")
+
+
+class ClockSampler:
+    """NVML (the library behind nvidia-smi) samples of SM clock, power and
+    clock-event reasons on this rank's GPU while running."""
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+             0x8: "hw_slowdown", 0x20: "sync_boost", 0x40: "sw_thermal_slowdown",
+             0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown",
+             0x200: "display_clock_setting"}
+
+    def __init__(self, torch_device, period=0.005):
+        self.period = period
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            idx = torch.cuda._get_nvml_device_index(torch_device)
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, do not guess
+            self.err = repr(e)
+
+    def _one(self):
+        nv = self.nv
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                             nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0, int(r)))
+
+    def _loop(self):
+        while not self.stop.is_set():
+            self._one()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.stop = threading.Event()
+            self._one()
+            self.th = threading.Thread(target=self._loop, daemon=True)
+            self.th.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop.set()
+            self.th.join()
+            self._one()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[2]
+        reasons = [n for b, n in sorted(self.NAMES.items()) if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples),
+                "power_w_max": max(s[1] for s in self.samples), "source": "NVML"}
+
+
+def cpu_baseline(inp, seconds):
+    """The fp64 oracle (block-recurrence route, every output) on the host cores,
+    on a bounded sample: whole passes over the workload until ``seconds``."""
+    import oracle
+    orc = oracle.default()
+    spec = inp.spec
+    threads = orc.max_threads()
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        orc.recurrence(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, spec.block_len, spec.eps)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or n >= 50:
+            break
+    return {"value": n * spec.token_heads / el, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} full pass(es) of the recurrence route over the whole {spec.name} "
+                      f"workload ({spec.token_heads} token-heads each, every output and the final "
+                      f"state), fp64, {threads} OpenMP threads, {el:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle, rank 0 only, each step a bounded
+    sample (a subset of heads) of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    spec = NAMED[args.workload]
+    inp = make_inputs(spec)
+    orc = oracle.default()
+    # calibrate: time of one head
+    t0 = time.perf_counter()
+    sub = lambda a, nh: np.ascontiguousarray(a[:, :, :nh])
+    orc.recurrence(sub(inp.q, 1), sub(inp.k, 1), sub(inp.v, 1), inp.rope_cos, inp.rope_sin,
+                   spec.block_len, spec.eps)
+    per_head = max(time.perf_counter() - t0, 1e-4)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    nh = int(max(1, min(spec.H, budget / per_head)))
+    q, k, v = sub(inp.q, nh), sub(inp.k, nh), sub(inp.v, nh)
+    for _ in range(args.warmup):
+        orc.recurrence(q, k, v, inp.rope_cos, inp.rope_sin, spec.block_len, spec.eps)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.recurrence(q, k, v, inp.rope_cos, inp.rope_sin, spec.block_len, spec.eps)
+    el = time.perf_counter() - t0
+    units = spec.B * spec.N * nh
+    val = units * args.steps / el
+    line = {"metric": METRIC, "value": val, "unit": UNIT, "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(spec, 1),
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": orc.max_threads(), "kind": "oracle",
+                             "sample": f"each step: recurrence route over {nh} of {spec.H} heads "
+                                       f"of {spec.name} ({units} token-heads)"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(device)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    import block_causal_relu_b200 as lcla
+
+    base = NAMED[args.workload]
+    from dataclasses import replace
+    spec = replace(base, seed=base.seed + 1000 * rank)       # independent problem per rank
+    inp = make_inputs(spec)
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(a).to(device)
+
+    q, k, v, c, s = (to_dev(a) for a in (inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin))
+    code = lcla.BF16 if spec.dtype == "bf16" else lcla.F32
+    out = torch.empty_like(q)
+    st = torch.empty((spec.B, spec.H, 33, 32), dtype=torch.float32, device=device)
+    ws = torch.empty(max(1, lcla.forward_workspace_bytes(spec.B, spec.H, spec.N, 32,
+                                                         spec.block_len, code)),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    K, W = args.steps, args.warmup
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for row in evs:                       # materialise the event handles
+        for e in row:
+            e.record(stream)
+
+    def step(events=None):
+        lcla.forward(q, k, v, c, s, spec.block_len, spec.eps, out=out, state_out=st,
+                     workspace=ws, stream=stream, events=events)
+
+    for _ in range(W):
+        step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device) as clk:
+        e0.record(stream)
+        for i in range(K):
+            step(evs[i])
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms = ms_total / K
+    units = spec.token_heads
+    value = world * units * K / (ms_total / 1e3)
+
+    # per-pass device times over the timed region
+    pa = [r[0].elapsed_time(r[1]) for r in evs]
+    sc = [r[1].elapsed_time(r[2]) for r in evs]
+    pc = [r[2].elapsed_time(r[3]) for r in evs]
+    esz = spec.elem_bytes
+    tok_bytes = spec.B * spec.N * spec.H * spec.d * esz             # one [B, N, H, d] tensor
+    tab_bytes = 2 * spec.N * (spec.d // 2) * 4
+    plan = lcla.plan_info(spec.B, spec.H, spec.N, 32, spec.block_len, code)
+    nseg, npref = plan["segments"], plan["prefixes"]
+    sl = spec.B * spec.H * STATE_BYTES
+    bytes_a = 2 * tok_bytes + tab_bytes + nseg * sl
+    bytes_c = 2 * tok_bytes + tab_bytes + npref * sl
+    bytes_s = nseg * sl + npref * sl + sl
+    passes = {"pass_a": (statistics.mean(pa), bytes_a, "pass_a_ffma"),
+              "scan": (statistics.mean(sc), bytes_s, "scan_states"),
+              "pass_c": (statistics.mean(pc), bytes_c,
+                         "pass_c_chunk_ffma" if plan["chunk_mode"] else "pass_c_ffma")}
+    dom = max(passes, key=lambda kk: passes[kk][0])
+    dms, dbytes, dname = passes[dom]
+    peak, peak_kind = measured_peak()
+    achieved = dbytes / (dms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dname, "achieved": achieved, "peak": peak,
+                "peak_source": f"{peak_kind} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
+                "traffic": ncu_traffic(dname, spec.name), "algorithmic_bytes": dbytes}
+    path_bytes = 4 * tok_bytes + 2 * tab_bytes + sl      # q,k,v in + out + tables + state
+    pass_ms = {kk: vv[0] for kk, vv in passes.items()}
+
+    # end to end through the same call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3))
+        hq.copy_(q); hk.copy_(k); hv.copy_(v)
+        hc = torch.empty(c.shape, dtype=c.dtype, pin_memory=True); hc.copy_(c)
+        hs = torch.empty(s.shape, dtype=s.dtype, pin_memory=True); hs.copy_(s)
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hst = torch.empty(st.shape, dtype=st.dtype, pin_memory=True)
+        KE = max(1, min(args.e2e_steps, K))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True); c.copy_(hc, non_blocking=True)
+            s.copy_(hs, non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+            hst.copy_(st, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(KE):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        ems = max_over_ranks(a0.elapsed_time(a1))
+        h2d = 3 * tok_bytes + tab_bytes
+        d2h = tok_bytes + sl
+        e2e = {"value": world * units * KE / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ems / KE, "steps": KE}
+
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_baseline(inp, args.cpu_seconds)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+                "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic (seeded)",
+                "config": workload_config(spec, world),
+                "achieved_hbm_gbs": world * path_bytes / (ms / 1e3) / 1e9 / world,
+                "hbm_frac_of_peak": path_bytes / (ms / 1e3) / 1e9 / peak,
+                "pass_ms": pass_ms, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": 3 * K, "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

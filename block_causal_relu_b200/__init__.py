@@ -1,0 +1,169 @@
+"""Block-causal ReLU linear attention with a carried fp32 state, on B200.
+
+Thin binding of the C-ABI library ``liblcla.so`` (declared in
+``include/lcla.h``): it checks and marshals torch tensors (device memory and
+the current CUDA stream) into the two entry points.  Every step of the
+computation runs in the library's sm_100a kernels; there is no other path.
+Importing this package fails if the library has not been built
+(``python block_causal_relu_b200/build.py``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["forward", "step", "forward_workspace_bytes", "step_workspace_bytes", "plan_info",
+           "LclaError", "LIB_PATH", "lib", "BF16", "F32", "D"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblcla.so")
+BF16, F32 = 0, 1
+D = 32
+DEFAULT_EPS = 1e-8
+
+
+class LclaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"lcla status {status}: {msg}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python block_causal_relu_b200/build.py`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.lcla_forward_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    L.lcla_forward_workspace_bytes.restype = Z
+    L.lcla_step_workspace_bytes.argtypes = [I, I, I, I, I]
+    L.lcla_step_workspace_bytes.restype = Z
+    L.lcla_forward.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P, P, I, P, Z, P]
+    L.lcla_forward.restype = I
+    L.lcla_forward_timed.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P, P, I, P, Z, P, P]
+    L.lcla_forward_timed.restype = I
+    L.lcla_step.argtypes = [P, P, P, P, P, I, I, I, I, F, P, I, P, I, P, Z, P]
+    L.lcla_step.restype = I
+    L.lcla_forward_plan_info.argtypes = [I, I, I, I, I, I, P]
+    L.lcla_forward_plan_info.restype = I
+    L.lcla_status_string.argtypes = [I]
+    L.lcla_status_string.restype = ctypes.c_char_p
+    L.lcla_version.restype = I
+    return L
+
+
+lib = _load()
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise LclaError(rc, lib.lcla_status_string(rc).decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"q, k, v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _inputs(q, k, v, cos, sin):
+    for name, t in (("q", q), ("k", k), ("v", v), ("cos", cos), ("sin", sin)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one [B, N, H, d] shape")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, d = q.shape
+    if cos.dtype != torch.float32 or sin.dtype != torch.float32:
+        raise TypeError("rope tables must be float32")
+    if tuple(cos.shape) != (N, d // 2) or tuple(sin.shape) != (N, d // 2):
+        raise ValueError("rope tables must be [N, d/2]")
+    return B, N, H, d, _dtype_code(q)
+
+
+def forward_workspace_bytes(B: int, H: int, N: int, d: int, block_len: int, dtype: int) -> int:
+    return int(lib.lcla_forward_workspace_bytes(B, H, N, d, block_len, dtype))
+
+
+def step_workspace_bytes(B: int, H: int, L: int, d: int, dtype: int) -> int:
+    return int(lib.lcla_step_workspace_bytes(B, H, L, d, dtype))
+
+
+def plan_info(B: int, H: int, N: int, d: int, block_len: int, dtype: int) -> dict:
+    """The library's cut of a forward problem (see ``lcla_forward_plan_info``)."""
+    info = (ctypes.c_int * 4)()
+    _check(lib.lcla_forward_plan_info(B, H, N, d, block_len, dtype, info))
+    return {"chunk_mode": bool(info[0]), "segments": info[1], "prefixes": info[2],
+            "tile_tokens": info[3]}
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rope_cos: torch.Tensor,
+            rope_sin: torch.Tensor, block_len: int, eps: float = DEFAULT_EPS, *,
+            out: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
+            want_state: bool = True, workspace: Optional[torch.Tensor] = None,
+            stream=None, events=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """``lcla_forward``: whole-sequence block-causal attention.
+
+    q, k, v [B, N, H, d] (bf16 or fp32), rope tables [N, d/2] fp32, all CUDA.
+    Returns (out [B, N, H, d], state_out [B, H, d+1, d] fp32 or None).
+    Buffers not passed in are allocated with torch on q's device.
+    ``events``: optional 4 already-recorded ``torch.cuda.Event(enable_timing=True)``
+    that the library re-records around its passes (``lcla_forward_timed``).
+    """
+    B, N, H, d, code = _inputs(q, k, v, rope_cos, rope_sin)
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, d + 1, d), dtype=torch.float32, device=q.device)
+    need = forward_workspace_bytes(B, H, N, d, block_len, code)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    evp = None
+    if events is not None:
+        if len(events) != 4:
+            raise ValueError("events must hold 4 torch.cuda.Event")
+        evp = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
+    _check(lib.lcla_forward_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin),
+                                  B, H, N, d, int(block_len), float(eps), _ptr(out),
+                                  _ptr(state_out), code, _ptr(workspace),
+                                  0 if workspace is None else workspace.numel(),
+                                  _stream(stream, q.device), evp))
+    return out, state_out
+
+
+def step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cos: torch.Tensor,
+         sin: torch.Tensor, state: torch.Tensor, save: bool, eps: float = DEFAULT_EPS, *,
+         out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+         stream=None) -> torch.Tensor:
+    """``lcla_step``: one block [B, L, H, d] against ``state`` [B, H, d+1, d]
+    fp32 (updated in place when ``save``).  Returns the block's outputs."""
+    B, L, H, d, code = _inputs(q, k, v, cos, sin)
+    if (not state.is_cuda or state.dtype != torch.float32 or not state.is_contiguous()
+            or tuple(state.shape) != (B, H, d + 1, d)):
+        raise ValueError("state must be a contiguous float32 CUDA tensor [B, H, d+1, d]")
+    if out is None:
+        out = torch.empty_like(q)
+    need = step_workspace_bytes(B, H, L, d, code)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(lib.lcla_step(_ptr(q), _ptr(k), _ptr(v), _ptr(cos), _ptr(sin), B, H, L, d, float(eps),
+                         _ptr(state), int(bool(save)), _ptr(out), code, _ptr(workspace),
+                         0 if workspace is None else workspace.numel(), _stream(stream, q.device)))
+    return out

@@ -1,0 +1,266 @@
+// lcla_api.cu -- the C ABI declared in include/lcla.h.
+//
+// Validates every argument on the host before anything is enqueued, builds
+// the work plan, and launches pass A (segment partial states), the scan
+// (prefix states, carried state in/out) and pass C (outputs) on the caller's
+// stream.  Allocates nothing.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "lcla.h"
+#include "lcla_ffma.cuh"
+#include "lcla_plan.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Shape checks shared by both entry points and the workspace queries.
+int check_shape(int B, int H, int N, int d, int L, int dtype)
+{
+    if (B < 1 || H < 1 || N < 0 || d < 1 || L < 1) return LCLA_ERR_INVALID_ARG;
+    if (dtype != LCLA_BF16 && dtype != LCLA_F32) return LCLA_ERR_INVALID_ARG;
+    if (d & 1) return LCLA_ERR_INVALID_ARG;
+    if (d != LCLA_D) return LCLA_ERR_UNSUPPORTED;
+    if (N > (1 << 30)) return LCLA_ERR_UNSUPPORTED;
+    if (B > 65535 || (H + LCLA_HG - 1) / LCLA_HG > 65535) return LCLA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0x7fffffffLL) return LCLA_ERR_UNSUPPORTED;
+    return LCLA_OK;
+}
+
+// Cut the problem into segments (see lcla_plan.h) and lay out the workspace:
+// [part: nseg x B x H x (d+1) x d fp32][pref: npref x B x H x (d+1) x d fp32].
+LclaPlan make_plan(int B, int H, int N, int L, int dtype)
+{
+    LclaPlan p;
+    memset(&p, 0, sizeof p);
+    p.B = B; p.H = H; p.N = N; p.L = L; p.dtype = dtype;
+    p.ngroups = (H + LCLA_HG - 1) / LCLA_HG;
+    if (N == 0) return p;
+    p.nb = (int)(((long long)N + L - 1) / L);
+    const long long units = (long long)p.ngroups * B;
+    if (L > LCLA_T) {
+        p.chunk = 0;
+        p.T = LCLA_T;
+        const long long tpb = ((long long)(L < N ? L : N) + LCLA_T - 1) / LCLA_T;   // tiles per full block
+        long long nsb = (LCLA_TARGET_CTAS + units * p.nb - 1) / (units * p.nb);
+        if (nsb > tpb) nsb = tpb;
+        if (nsb < 1) nsb = 1;
+        p.nsb = (int)nsb;
+        p.nseg = p.nb * p.nsb;
+        p.npref = p.nb;
+    } else {
+        p.chunk = 1;
+        p.T = (LCLA_T / L) * L;
+        const long long ntiles = ((long long)N + p.T - 1) / p.T;
+        long long tps = (ntiles * units + LCLA_TARGET_CTAS - 1) / LCLA_TARGET_CTAS;
+        if (tps < 1) tps = 1;
+        if (tps > ntiles) tps = ntiles;
+        p.tps = (int)tps;
+        p.nseg = (int)((ntiles + tps - 1) / tps);
+        p.npref = p.nseg;
+    }
+    const size_t slice = (size_t)B * H * LCLA_SZ * sizeof(float);
+    p.part_off = 0;
+    p.pref_off = round_up((size_t)p.nseg * slice);
+    p.ws_bytes = p.pref_off + round_up((size_t)p.npref * slice);
+    return p;
+}
+
+bool misaligned(const void *ptr) { return ((uintptr_t)ptr & 15u) != 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    if (!a || !b || !na || !nb) return false;
+    const uintptr_t a0 = (uintptr_t)a, a1 = a0 + na, b0 = (uintptr_t)b, b1 = b0 + nb;
+    return a0 < b1 && b0 < a1;
+}
+
+template <typename F>
+void set_smem(F *kernel, int bytes)
+{
+    // Idempotent; cheap compared with the launches it precedes.
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <typename Tin>
+int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const float *rs,
+               const LclaPlan &p, float eps, Tin *out, const float *state_in, float *state_out,
+               unsigned char *ws, cudaStream_t st, cudaEvent_t const *ev)
+{
+    using G = lcla::Geo<Tin>;
+    float *part = reinterpret_cast<float *>(ws + p.part_off);
+    float *pref = reinterpret_cast<float *>(ws + p.pref_off);
+    const dim3 grid(p.nseg, p.ngroups, p.B);
+
+    const int smem_a = 2 * (2 * G::TILE_IN + 2 * G::TILE_TAB) + G::TILE_F;
+    set_smem(lcla::pass_a_ffma<Tin>, smem_a);
+    if (ev) cudaEventRecord(ev[0], st);
+    lcla::pass_a_ffma<Tin><<<grid, 256, smem_a, st>>>(k, v, rc, rs, p, part);
+
+    if (ev) cudaEventRecord(ev[1], st);
+    lcla::scan_states<<<p.B * p.H, 264, 0, st>>>(p, part, pref, state_in, state_out);
+    if (ev) cudaEventRecord(ev[2], st);
+
+    if (!p.chunk) {
+        const int smem_c = 2 * (G::TILE_IN + 2 * G::TILE_TAB) + G::TILE_F +
+                           (LCLA_HG * LCLA_D * LCLA_D + LCLA_HG * LCLA_D + LCLA_T * LCLA_HG) * 4;
+        set_smem(lcla::pass_c_ffma<Tin>, smem_c);
+        lcla::pass_c_ffma<Tin><<<grid, 256, smem_c, st>>>(q, rc, rs, p, pref, eps, out);
+    } else {
+        const int smem_c = 3 * G::TILE_IN + 2 * G::TILE_TAB + 4 * G::TILE_F +
+                           (LCLA_HG * LCLA_T * LCLA_T + LCLA_HG * LCLA_D * LCLA_D + LCLA_HG * LCLA_D) * 4;
+        set_smem(lcla::pass_c_chunk_ffma<Tin>, smem_c);
+        lcla::pass_c_chunk_ffma<Tin><<<grid, 256, smem_c, st>>>(q, k, v, rc, rs, p, pref, eps, out);
+    }
+    if (ev) cudaEventRecord(ev[3], st);
+    return cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
+}
+
+// Shared body of lcla_forward and lcla_step once the arguments are checked.
+int run(const void *q, const void *k, const void *v, const float *rc, const float *rs,
+        const LclaPlan &p, float eps, void *out, const float *state_in, float *state_out,
+        void *ws, cudaStream_t st, cudaEvent_t const *ev = nullptr)
+{
+    if (p.dtype == LCLA_BF16)
+        return launch_all<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                         (const __nv_bfloat16 *)v, rc, rs, p, eps,
+                                         (__nv_bfloat16 *)out, state_in, state_out,
+                                         (unsigned char *)ws, st, ev);
+    return launch_all<float>((const float *)q, (const float *)k, (const float *)v, rc, rs, p, eps,
+                             (float *)out, state_in, state_out, (unsigned char *)ws, st, ev);
+}
+
+// Pointer, alignment, overlap and workspace checks for one call.
+int check_buffers(const void *q, const void *k, const void *v, const float *rc, const float *rs,
+                  const void *out, const float *state, bool state_required, int B, int H, int N,
+                  int dtype, float eps, const void *ws, size_t ws_bytes, size_t need)
+{
+    if (!(eps >= 0.f) || !isfinite(eps)) return LCLA_ERR_INVALID_ARG;
+    if (state_required && !state) return LCLA_ERR_INVALID_ARG;
+    if (N == 0) {
+        if (state && misaligned(state)) return LCLA_ERR_MISALIGNED;
+        return LCLA_OK;
+    }
+    if (!q || !k || !v || !rc || !rs || !out) return LCLA_ERR_INVALID_ARG;
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(rc) || misaligned(rs) ||
+        misaligned(out) || (state && misaligned(state)) || (ws && misaligned(ws)))
+        return LCLA_ERR_MISALIGNED;
+    const size_t esz = dtype == LCLA_BF16 ? 2 : 4;
+    const size_t nio = (size_t)B * N * H * LCLA_D * esz;
+    const size_t ntab = (size_t)N * (LCLA_D / 2) * sizeof(float);
+    const size_t nst = (size_t)B * H * LCLA_SZ * sizeof(float);
+    if (overlaps(out, nio, q, nio) || overlaps(out, nio, k, nio) || overlaps(out, nio, v, nio) ||
+        overlaps(out, nio, rc, ntab) || overlaps(out, nio, rs, ntab) ||
+        overlaps(out, nio, state, nst) || overlaps(out, nio, ws, ws_bytes))
+        return LCLA_ERR_INVALID_ARG;
+    if (need > 0) {
+        if (!ws || ws_bytes < need) return LCLA_ERR_WORKSPACE;
+        if (overlaps(ws, need, q, nio) || overlaps(ws, need, k, nio) || overlaps(ws, need, v, nio) ||
+            overlaps(ws, need, rc, ntab) || overlaps(ws, need, rs, ntab) || overlaps(ws, need, state, nst))
+            return LCLA_ERR_INVALID_ARG;
+    }
+    if (state && (overlaps(state, nst, q, nio) || overlaps(state, nst, k, nio) ||
+                  overlaps(state, nst, v, nio) || overlaps(state, nst, rc, ntab) ||
+                  overlaps(state, nst, rs, ntab)))
+        return LCLA_ERR_INVALID_ARG;
+    return LCLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lcla_forward_workspace_bytes(int B, int H, int N, int d, int block_len, int dtype)
+{
+    if (check_shape(B, H, N, d, block_len, dtype) != LCLA_OK) return 0;
+    return make_plan(B, H, N, block_len, dtype).ws_bytes;
+}
+
+size_t lcla_step_workspace_bytes(int B, int H, int L, int d, int dtype)
+{
+    if (check_shape(B, H, L, d, L < 1 ? 1 : L, dtype) != LCLA_OK) return 0;
+    return make_plan(B, H, L, L < 1 ? 1 : L, dtype).ws_bytes;
+}
+
+int lcla_forward_timed(const void *q, const void *k, const void *v, const float *rope_cos,
+                       const float *rope_sin, int B, int H, int N, int d, int block_len, float eps,
+                       void *out, float *state_out, int dtype, void *workspace,
+                       size_t workspace_bytes, void *stream, void *const *events)
+{
+    int rc = check_shape(B, H, N, d, block_len, dtype);
+    if (rc != LCLA_OK) return rc;
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, dtype, eps,
+                       workspace, workspace_bytes, p.ws_bytes);
+    if (rc != LCLA_OK) return rc;
+    if (events && (!events[0] || !events[1] || !events[2] || !events[3])) return LCLA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaEvent_t const *ev = reinterpret_cast<cudaEvent_t const *>(events);
+    if (N == 0) {
+        if (ev) cudaEventRecord(ev[0], st);
+        if (state_out && cudaMemsetAsync(state_out, 0, (size_t)B * H * LCLA_SZ * sizeof(float), st) != cudaSuccess)
+            return LCLA_ERR_CUDA;
+        if (ev) { cudaEventRecord(ev[1], st); cudaEventRecord(ev[2], st); cudaEventRecord(ev[3], st); }
+        return LCLA_OK;
+    }
+    return run(q, k, v, rope_cos, rope_sin, p, eps, out, nullptr, state_out, workspace, st, ev);
+}
+
+int lcla_forward(const void *q, const void *k, const void *v, const float *rope_cos,
+                 const float *rope_sin, int B, int H, int N, int d, int block_len, float eps,
+                 void *out, float *state_out, int dtype, void *workspace, size_t workspace_bytes,
+                 void *stream)
+{
+    return lcla_forward_timed(q, k, v, rope_cos, rope_sin, B, H, N, d, block_len, eps, out,
+                              state_out, dtype, workspace, workspace_bytes, stream, nullptr);
+}
+
+int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk, const float *cos_blk,
+              const float *sin_blk, int B, int H, int L, int d, float eps, float *state, int save,
+              void *out, int dtype, void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_shape(B, H, L, d, L < 1 ? 1 : L, dtype);
+    if (rc != LCLA_OK) return rc;
+    const LclaPlan p = make_plan(B, H, L, L < 1 ? 1 : L, dtype);
+    rc = check_buffers(q_blk, k_blk, v_blk, cos_blk, sin_blk, out, state, true, B, H, L, dtype, eps,
+                       workspace, workspace_bytes, p.ws_bytes);
+    if (rc != LCLA_OK) return rc;
+    if (L == 0) return LCLA_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    return run(q_blk, k_blk, v_blk, cos_blk, sin_blk, p, eps, out, state, save ? state : nullptr,
+               workspace, st);
+}
+
+int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype, int *info)
+{
+    const int rc = check_shape(B, H, N, d, block_len, dtype);
+    if (rc != LCLA_OK) return rc;
+    if (!info) return LCLA_ERR_INVALID_ARG;
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    info[0] = p.chunk;
+    info[1] = p.nseg;
+    info[2] = p.npref;
+    info[3] = p.T;
+    return LCLA_OK;
+}
+
+const char *lcla_status_string(int status)
+{
+    switch (status) {
+    case LCLA_OK: return "ok";
+    case LCLA_ERR_INVALID_ARG: return "invalid argument";
+    case LCLA_ERR_UNSUPPORTED: return "unsupported problem (this build serves d = 32, N <= 2^30)";
+    case LCLA_ERR_MISALIGNED: return "array pointer not 16-byte aligned";
+    case LCLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case LCLA_ERR_CUDA: return "CUDA launch failed";
+    default: return "unknown status";
+    }
+}
+
+int lcla_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,660 @@
+// lcla_ffma.cuh -- CUDA-core (FFMA) kernels for every dtype and block length.
+//
+// Pass A: per segment, the partial state
+//           S[c][e] = sum_j v_j[c] (R_j phi(k_j))[e],  z[e] = sum_j phi(k_j)[e]
+//         ("Implementing Block Causal Linear Attention for Long Video
+//          Generation with Sana", section "The Linear Attention Kernel":
+//          vk = v k_rotated^T and the key sum of the normaliser).
+// Pass C: out_i = (P S) R_i phi(q_i) / (P_z . phi(q_i) + eps) with P the
+//         prefix state the token sees (same section: out = vk q_rotated,
+//         output = out * z).  Chunk mode adds the masked in-tile term.
+// phi = ReLU applied to q and k only; the rotary embedding R acts on the
+// ReLU features, interleaved pairs (same page, "Rotary Position Embeddings").
+//
+// Both passes stream [tile][head group] slices of the [B, N, H, d] inputs
+// through shared memory with cp.async (16-byte chunks, zero fill for ragged
+// tiles and missing heads, so padding contributes exact zeros), keep all
+// arithmetic in fp32 and reduce in a fixed order (no atomics).
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "lcla_plan.h"
+
+namespace lcla {
+
+// ---------------------------------------------------------------------------
+// small device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    const int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+// ReLU written as a comparison so that NaN passes through.
+__device__ __forceinline__ float relu(float x) { return x < 0.f ? 0.f : x; }
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// 8 consecutive elements -> fp32
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float *x)
+{
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    x[0] = bf_lo(u.x); x[1] = bf_hi(u.x); x[2] = bf_lo(u.y); x[3] = bf_hi(u.y);
+    x[4] = bf_lo(u.z); x[5] = bf_hi(u.z); x[6] = bf_lo(u.w); x[7] = bf_hi(u.w);
+}
+__device__ __forceinline__ void load8(const float *p, float *x)
+{
+    const float4 a = reinterpret_cast<const float4 *>(p)[0];
+    const float4 b = reinterpret_cast<const float4 *>(p)[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+// 4 consecutive elements -> fp32
+__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float *x)
+{
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    x[0] = bf_lo(u.x); x[1] = bf_hi(u.x); x[2] = bf_lo(u.y); x[3] = bf_hi(u.y);
+}
+__device__ __forceinline__ void load4(const float *p, float *x)
+{
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+}
+// 4 fp32 -> 4 consecutive outputs (bf16 round-to-nearest-even)
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, const float *x)
+{
+    __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(x[2], x[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+__device__ __forceinline__ void store4(float *p, const float *x)
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+}
+
+// phi then the rotary embedding on 8 consecutive elements (4 pairs) of a head
+// row; x holds the raw values on entry, f the ReLU features and y the rotated
+// features on exit.  c4/s4 are the 4 table entries of these pairs.
+__device__ __forceinline__ void relu_rope8(const float *x, const float4 &c4, const float4 &s4,
+                                           float *f, float *y)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = relu(x[i]);
+    const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+    const float ss[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float a = f[2 * p], b = f[2 * p + 1];
+        y[2 * p] = a * cc[p] - b * ss[p];
+        y[2 * p + 1] = a * ss[p] + b * cc[p];
+    }
+}
+
+// Tile geometry for one input type.
+template <typename Tin>
+struct Geo {
+    static constexpr int EB = (int)sizeof(Tin);
+    static constexpr int ROWB = LCLA_D * EB;                  // bytes of one head row
+    static constexpr int CPR = ROWB / 16;                     // 16-byte chunks per head row
+    static constexpr int TILE_IN = LCLA_T * LCLA_HG * ROWB;   // one input tile [T][HG][D]
+    static constexpr int TILE_TAB = LCLA_T * (LCLA_D / 2) * 4; // one table tile [T][D/2] fp32
+    static constexpr int TILE_F = LCLA_T * LCLA_HG * LCLA_D * 4; // fp32 tile [T][HG][D]
+};
+
+// Queue cp.async copies of rows [t, t + nt) of an input tensor for heads
+// h0, h0+1 into buf ([T][HG][D] elements); rows and heads outside the valid
+// range are zero-filled without reading global memory.
+template <typename Tin>
+__device__ __forceinline__ void issue_rows(unsigned char *buf, const Tin *src, const LclaPlan &p,
+                                           int b, int t, int nt, int h0, int tid, int nthr)
+{
+    using G = Geo<Tin>;
+    for (int c = tid; c < LCLA_T * LCLA_HG * G::CPR; c += nthr) {
+        const int tok = c / (LCLA_HG * G::CPR);
+        const int rem = c - tok * (LCLA_HG * G::CPR);
+        const int hh = rem / G::CPR;
+        const int part = rem - hh * G::CPR;
+        const bool ok = tok < nt && h0 + hh < p.H;
+        const size_t off = ok ? ((((size_t)b * p.N + (size_t)(t + tok)) * p.H + (size_t)(h0 + hh)) *
+                                     LCLA_D) * G::EB + (size_t)part * 16
+                              : 0;
+        cp_async16(buf + (size_t)c * 16, reinterpret_cast<const unsigned char *>(src) + off, ok);
+    }
+}
+
+// Same for the [N, D/2] fp32 tables.
+__device__ __forceinline__ void issue_table(unsigned char *buf, const float *tab, int t, int nt,
+                                            int tid, int nthr)
+{
+    for (int c = tid; c < LCLA_T * 4; c += nthr) {
+        const int tok = c >> 2, part = c & 3;
+        const bool ok = tok < nt;
+        const size_t off = ok ? (size_t)(t + tok) * (LCLA_D / 2) * 4 + (size_t)part * 16 : 0;
+        cp_async16(buf + (size_t)c * 16, reinterpret_cast<const unsigned char *>(tab) + off, ok);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pass A: segment partial states.  grid (nseg, ngroups, B), 256 threads.
+// part layout: [nseg][B][H][D+1][D] fp32.
+// ---------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(256)
+pass_a_ffma(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *__restrict__ rcos,
+            const float *__restrict__ rsin, const LclaPlan p, float *__restrict__ part)
+{
+    using G = Geo<Tin>;
+    constexpr int STAGE = 2 * G::TILE_IN + 2 * G::TILE_TAB;
+    extern __shared__ __align__(128) unsigned char sm[];
+    float *kt = reinterpret_cast<float *>(sm + 2 * STAGE);   // [T][HG][D] rotated features
+
+    const int s = blockIdx.x, h0 = blockIdx.y * LCLA_HG, b = blockIdx.z;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const LclaSeg g = lcla_segment(p, s);
+    const int ntile = (g.t1 - g.t0 + LCLA_T - 1) / LCLA_T;
+
+    // outer-product micro tile: warp w -> head w>>2, 16 tokens of each tile;
+    // lane -> value dims c0..c0+3, key dims e0..e0+7
+    const int ohh = w >> 2, otq = (w & 3) * 16;
+    const int c0 = (lane >> 2) * 4, e0 = (lane & 3) * 8;
+    float acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    float zacc[8];   // key-sum partial of (head (tid>>2)&1, dims (tid&3)*8..+8)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) zacc[i] = 0.f;
+
+    auto issue = [&](int st, int i) {
+        unsigned char *buf = sm + st * STAGE;
+        const int t = g.t0 + i * LCLA_T, nt = min(LCLA_T, g.t1 - t);
+        issue_rows<Tin>(buf, k, p, b, t, nt, h0, tid, 256);
+        issue_rows<Tin>(buf + G::TILE_IN, v, p, b, t, nt, h0, tid, 256);
+        issue_table(buf + 2 * G::TILE_IN, rcos, t, nt, tid, 256);
+        issue_table(buf + 2 * G::TILE_IN + G::TILE_TAB, rsin, t, nt, tid, 256);
+        cp_async_commit();
+    };
+
+    if (ntile > 0) issue(0, 0);
+    for (int i = 0; i < ntile; ++i) {
+        if (i + 1 < ntile) {
+            issue((i + 1) & 1, i + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const unsigned char *buf = sm + (i & 1) * STAGE;
+        const Tin *kraw = reinterpret_cast<const Tin *>(buf);
+        const Tin *vraw = reinterpret_cast<const Tin *>(buf + G::TILE_IN);
+        const float *ct = reinterpret_cast<const float *>(buf + 2 * G::TILE_IN);
+        const float *st = reinterpret_cast<const float *>(buf + 2 * G::TILE_IN + G::TILE_TAB);
+
+        // prologue: phi, rotary, key sum
+        for (int it = tid; it < LCLA_T * LCLA_HG * 4; it += 256) {
+            const int tok = it >> 3, hh = (it >> 2) & 1, qtr = it & 3;
+            float x[8], f[8], y[8];
+            load8(kraw + (tok * LCLA_HG + hh) * LCLA_D + qtr * 8, x);
+            const float4 c4 = reinterpret_cast<const float4 *>(ct + tok * (LCLA_D / 2))[qtr];
+            const float4 s4 = reinterpret_cast<const float4 *>(st + tok * (LCLA_D / 2))[qtr];
+            relu_rope8(x, c4, s4, f, y);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) zacc[j] += f[j];
+            float4 *dst = reinterpret_cast<float4 *>(kt + (tok * LCLA_HG + hh) * LCLA_D + qtr * 8);
+            dst[0] = make_float4(y[0], y[1], y[2], y[3]);
+            dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+        }
+        __syncthreads();
+
+        // outer products over this warp's 16 tokens
+#pragma unroll 4
+        for (int t = 0; t < 16; ++t) {
+            const int tok = otq + t;
+            float vv[4];
+            load4(vraw + (tok * LCLA_HG + ohh) * LCLA_D + c0, vv);
+            const float4 ka = *reinterpret_cast<const float4 *>(kt + (tok * LCLA_HG + ohh) * LCLA_D + e0);
+            const float4 kb = *reinterpret_cast<const float4 *>(kt + (tok * LCLA_HG + ohh) * LCLA_D + e0 + 4);
+            const float kk[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[ii][j] = fmaf(vv[ii], kk[j], acc[ii][j]);
+        }
+        __syncthreads();
+    }
+
+    // fixed-order reduction of the 4 warps of each head and of the key sums
+    float *red = reinterpret_cast<float *>(sm);                 // [8][D][D]
+    float *zred = red + 8 * LCLA_D * LCLA_D;                     // [256][8]
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) red[w * LCLA_D * LCLA_D + (c0 + ii) * LCLA_D + e0 + j] = acc[ii][j];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) zred[tid * 8 + j] = zacc[j];
+    __syncthreads();
+    for (int x = tid; x < LCLA_HG * LCLA_SZ; x += 256) {
+        const int hh = x / LCLA_SZ, e = x - hh * LCLA_SZ;
+        float val;
+        if (e < LCLA_D * LCLA_D) {
+            const float *r = red + (hh * 4) * LCLA_D * LCLA_D + e;
+            val = ((r[0] + r[LCLA_D * LCLA_D]) + r[2 * LCLA_D * LCLA_D]) + r[3 * LCLA_D * LCLA_D];
+        } else {
+            const int ez = e - LCLA_D * LCLA_D, qtr = ez >> 3, jj = ez & 7;
+            const int t0 = hh * 4 + qtr;      // threads t0, t0+8, ... hold this key-sum slot
+            val = 0.f;
+            for (int m = 0; m < 32; ++m) val += zred[(t0 + 8 * m) * 8 + jj];
+        }
+        if (h0 + hh < p.H)
+            part[(((size_t)s * p.B + b) * p.H + (h0 + hh)) * LCLA_SZ + e] = val;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pass C, block mode: every token of the segment uses its block's inclusive
+// prefix.  grid (nseg, ngroups, B), 256 threads.
+// pref layout: [npref][B][H][D+1][D] fp32.
+// ---------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(256)
+pass_c_ffma(const Tin *__restrict__ q, const float *__restrict__ rcos, const float *__restrict__ rsin,
+            const LclaPlan p, const float *__restrict__ pref, const float eps, Tin *__restrict__ out)
+{
+    using G = Geo<Tin>;
+    constexpr int STAGE = G::TILE_IN + 2 * G::TILE_TAB;
+    extern __shared__ __align__(128) unsigned char sm[];
+    float *qt = reinterpret_cast<float *>(sm + 2 * STAGE);            // [T][HG][D]
+    float *PT = qt + LCLA_T * LCLA_HG * LCLA_D;                       // [HG][D e][D c]
+    float *zz = PT + LCLA_HG * LCLA_D * LCLA_D;                       // [HG][D]
+    float *inv = zz + LCLA_HG * LCLA_D;                               // [T][HG]
+
+    const int s = blockIdx.x, h0 = blockIdx.y * LCLA_HG, b = blockIdx.z;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const LclaSeg g = lcla_segment(p, s);
+    const int ntile = (g.t1 - g.t0 + LCLA_T - 1) / LCLA_T;
+    if (ntile <= 0) return;
+
+    // prefix state of this block, transposed to [e][c]
+    for (int x = tid; x < LCLA_HG * LCLA_SZ; x += 256) {
+        const int hh = x / LCLA_SZ, e = x - hh * LCLA_SZ;
+        float val = 0.f;
+        if (h0 + hh < p.H) val = pref[(((size_t)g.blk * p.B + b) * p.H + (h0 + hh)) * LCLA_SZ + e];
+        if (e < LCLA_D * LCLA_D) PT[hh * LCLA_D * LCLA_D + (e & 31) * LCLA_D + (e >> 5)] = val;
+        else zz[hh * LCLA_D + (e - LCLA_D * LCLA_D)] = val;
+    }
+
+    const int ohh = w >> 2, otq = (w & 3) * 16 + (lane >> 3) * 4;   // 4 tokens per lane
+    const int c0 = (lane & 7) * 4;
+
+    auto issue = [&](int st, int i) {
+        unsigned char *buf = sm + st * STAGE;
+        const int t = g.t0 + i * LCLA_T, nt = min(LCLA_T, g.t1 - t);
+        issue_rows<Tin>(buf, q, p, b, t, nt, h0, tid, 256);
+        issue_table(buf + G::TILE_IN, rcos, t, nt, tid, 256);
+        issue_table(buf + G::TILE_IN + G::TILE_TAB, rsin, t, nt, tid, 256);
+        cp_async_commit();
+    };
+
+    issue(0, 0);
+    for (int i = 0; i < ntile; ++i) {
+        if (i + 1 < ntile) {
+            issue((i + 1) & 1, i + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const unsigned char *buf = sm + (i & 1) * STAGE;
+        const Tin *qraw = reinterpret_cast<const Tin *>(buf);
+        const float *ct = reinterpret_cast<const float *>(buf + G::TILE_IN);
+        const float *st = reinterpret_cast<const float *>(buf + G::TILE_IN + G::TILE_TAB);
+        const int t = g.t0 + i * LCLA_T, nt = min(LCLA_T, g.t1 - t);
+
+        // prologue: phi, rotary, denominator (4 lanes per (token, head))
+        for (int it = tid; it < LCLA_T * LCLA_HG * 4; it += 256) {
+            const int tok = it >> 3, hh = (it >> 2) & 1, qtr = it & 3;
+            float x[8], f[8], y[8];
+            load8(qraw + (tok * LCLA_HG + hh) * LCLA_D + qtr * 8, x);
+            const float4 c4 = reinterpret_cast<const float4 *>(ct + tok * (LCLA_D / 2))[qtr];
+            const float4 s4 = reinterpret_cast<const float4 *>(st + tok * (LCLA_D / 2))[qtr];
+            relu_rope8(x, c4, s4, f, y);
+            float dp = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dp = fmaf(f[j], zz[hh * LCLA_D + qtr * 8 + j], dp);
+            dp += __shfl_xor_sync(0xffffffffu, dp, 1);
+            dp += __shfl_xor_sync(0xffffffffu, dp, 2);
+            if (qtr == 0) inv[tok * LCLA_HG + hh] = 1.0f / (dp + eps);
+            float4 *dst = reinterpret_cast<float4 *>(qt + (tok * LCLA_HG + hh) * LCLA_D + qtr * 8);
+            dst[0] = make_float4(y[0], y[1], y[2], y[3]);
+            dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+        }
+        __syncthreads();
+
+        // outputs: 4 tokens x 4 value dims per lane
+        float acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+#pragma unroll
+        for (int e4 = 0; e4 < LCLA_D / 4; ++e4) {
+            float4 qv[4], pv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+                qv[a] = *reinterpret_cast<const float4 *>(qt + ((otq + a) * LCLA_HG + ohh) * LCLA_D + e4 * 4);
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                pv[m] = *reinterpret_cast<const float4 *>(PT + ohh * LCLA_D * LCLA_D + (e4 * 4 + m) * LCLA_D + c0);
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const float qq[4] = {qv[a].x, qv[a].y, qv[a].z, qv[a].w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    acc[a][0] = fmaf(qq[m], pv[m].x, acc[a][0]);
+                    acc[a][1] = fmaf(qq[m], pv[m].y, acc[a][1]);
+                    acc[a][2] = fmaf(qq[m], pv[m].z, acc[a][2]);
+                    acc[a][3] = fmaf(qq[m], pv[m].w, acc[a][3]);
+                }
+            }
+        }
+        if (h0 + ohh < p.H) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int tok = otq + a;
+                if (tok < nt) {
+                    const float r = inv[tok * LCLA_HG + ohh];
+                    float o[4] = {acc[a][0] * r, acc[a][1] * r, acc[a][2] * r, acc[a][3] * r};
+                    store4(out + (((size_t)b * p.N + (size_t)(t + tok)) * p.H + (h0 + ohh)) * LCLA_D + c0, o);
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pass C, chunk mode (block_len <= LCLA_T): tiles of whole blocks.  Each
+// segment walks its tiles in order with a running state R (exclusive prefix
+// at the tile start):
+//   num_i = R_S q~_i + sum_{j in tile, blk(j) <= blk(i)} v_j (k~_j . q~_i)
+//   den_i = (R_z + sum_{same j} phi(k_j)) . phi(q_i) + eps
+// then R += the tile's (S, z).  grid (nseg, ngroups, B), 256 threads.
+// ---------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(256)
+pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                  const float *__restrict__ rcos, const float *__restrict__ rsin, const LclaPlan p,
+                  const float *__restrict__ pref, const float eps, Tin *__restrict__ out)
+{
+    using G = Geo<Tin>;
+    extern __shared__ __align__(128) unsigned char sm[];
+    unsigned char *qraw_b = sm;
+    unsigned char *kraw_b = qraw_b + G::TILE_IN;
+    unsigned char *vraw_b = kraw_b + G::TILE_IN;
+    unsigned char *ct_b = vraw_b + G::TILE_IN;
+    unsigned char *st_b = ct_b + G::TILE_TAB;
+    float *qt = reinterpret_cast<float *>(st_b + G::TILE_TAB);        // [T][HG][D] rotated q
+    float *kt = qt + LCLA_T * LCLA_HG * LCLA_D;                       // rotated k
+    float *fq = kt + LCLA_T * LCLA_HG * LCLA_D;                       // phi(q)
+    float *fk = fq + LCLA_T * LCLA_HG * LCLA_D;                       // phi(k), then its running sum
+    float *sc = fk + LCLA_T * LCLA_HG * LCLA_D;                       // [HG][T j][T i] scores / reduction
+    float *RT = sc + LCLA_HG * LCLA_T * LCLA_T;                       // [HG][D e][D c]
+    float *Rz = RT + LCLA_HG * LCLA_D * LCLA_D;                       // [HG][D]
+
+    const int s = blockIdx.x, h0 = blockIdx.y * LCLA_HG, b = blockIdx.z;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const LclaSeg g = lcla_segment(p, s);
+    const int T = p.T, L = p.L;
+    const int ntile = (g.t1 - g.t0 + T - 1) / T;
+    if (ntile <= 0) return;
+
+    for (int x = tid; x < LCLA_HG * LCLA_SZ; x += 256) {
+        const int hh = x / LCLA_SZ, e = x - hh * LCLA_SZ;
+        float val = 0.f;
+        if (h0 + hh < p.H) val = pref[(((size_t)s * p.B + b) * p.H + (h0 + hh)) * LCLA_SZ + e];
+        if (e < LCLA_D * LCLA_D) RT[hh * LCLA_D * LCLA_D + (e & 31) * LCLA_D + (e >> 5)] = val;
+        else Rz[hh * LCLA_D + (e - LCLA_D * LCLA_D)] = val;
+    }
+
+    const int ohh = w >> 2, otq = (w & 3) * 16 + (lane >> 3) * 4;
+    const int c0 = (lane & 7) * 4;
+
+    for (int i = 0; i < ntile; ++i) {
+        const int t = g.t0 + i * T, nt = min(T, g.t1 - t);
+        issue_rows<Tin>(qraw_b, q, p, b, t, nt, h0, tid, 256);
+        issue_rows<Tin>(kraw_b, k, p, b, t, nt, h0, tid, 256);
+        issue_rows<Tin>(vraw_b, v, p, b, t, nt, h0, tid, 256);
+        issue_table(ct_b, rcos, t, nt, tid, 256);
+        issue_table(st_b, rsin, t, nt, tid, 256);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+        const Tin *qraw = reinterpret_cast<const Tin *>(qraw_b);
+        const Tin *kraw = reinterpret_cast<const Tin *>(kraw_b);
+        const Tin *vraw = reinterpret_cast<const Tin *>(vraw_b);
+        const float *ct = reinterpret_cast<const float *>(ct_b);
+        const float *st = reinterpret_cast<const float *>(st_b);
+
+        // prologue for q and k (rows past nt are zero-filled, so they give zeros)
+        for (int it = tid; it < LCLA_T * LCLA_HG * 4; it += 256) {
+            const int tok = it >> 3, hh = (it >> 2) & 1, qtr = it & 3;
+            const float4 c4 = reinterpret_cast<const float4 *>(ct + tok * (LCLA_D / 2))[qtr];
+            const float4 s4 = reinterpret_cast<const float4 *>(st + tok * (LCLA_D / 2))[qtr];
+            const int o = (tok * LCLA_HG + hh) * LCLA_D + qtr * 8;
+            float x[8], f[8], y[8];
+            load8(qraw + o, x);
+            relu_rope8(x, c4, s4, f, y);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { fq[o + j] = f[j]; qt[o + j] = y[j]; }
+            load8(kraw + o, x);
+            relu_rope8(x, c4, s4, f, y);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { fk[o + j] = f[j]; kt[o + j] = y[j]; }
+        }
+        __syncthreads();
+
+        // scores sc[hh][j][i] = [blk(j) <= blk(i)] (k~_j . q~_i), 4x4 blocks
+        for (int blkid = tid; blkid < LCLA_HG * 16 * 16; blkid += 256) {
+            const int hh = blkid >> 8, ib = (blkid >> 4) & 15, jb = blkid & 15;
+            float a[4][4];
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) a[ii][jj] = 0.f;
+#pragma unroll
+            for (int e4 = 0; e4 < LCLA_D / 4; ++e4) {
+                float4 qv[4], kv[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    qv[x] = *reinterpret_cast<const float4 *>(qt + ((ib * 4 + x) * LCLA_HG + hh) * LCLA_D + e4 * 4);
+                    kv[x] = *reinterpret_cast<const float4 *>(kt + ((jb * 4 + x) * LCLA_HG + hh) * LCLA_D + e4 * 4);
+                }
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        a[ii][jj] += qv[ii].x * kv[jj].x + qv[ii].y * kv[jj].y +
+                                     qv[ii].z * kv[jj].z + qv[ii].w * kv[jj].w;
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = jb * 4 + jj;
+                float o4[4];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) {
+                    const int i2 = ib * 4 + ii;
+                    o4[ii] = (j < nt && (j / L) <= (i2 / L)) ? a[ii][jj] : 0.f;
+                }
+                *reinterpret_cast<float4 *>(sc + (hh * LCLA_T + j) * LCLA_T + ib * 4) =
+                    make_float4(o4[0], o4[1], o4[2], o4[3]);
+            }
+        }
+        // running key sum over the tile, in token order, one thread per (head, dim)
+        if (tid < LCLA_HG * LCLA_D) {
+            const int hh = tid >> 5, e = tid & 31;
+            float run = 0.f;
+            for (int j = 0; j < nt; ++j) {
+                run += fk[(j * LCLA_HG + hh) * LCLA_D + e];
+                fk[(j * LCLA_HG + hh) * LCLA_D + e] = run;
+            }
+        }
+        __syncthreads();
+
+        // outputs
+        float acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+        for (int e4 = 0; e4 < LCLA_D / 4; ++e4) {      // carried state
+            float4 qv[4], pv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+                qv[a] = *reinterpret_cast<const float4 *>(qt + ((otq + a) * LCLA_HG + ohh) * LCLA_D + e4 * 4);
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                pv[m] = *reinterpret_cast<const float4 *>(RT + ohh * LCLA_D * LCLA_D + (e4 * 4 + m) * LCLA_D + c0);
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const float qq[4] = {qv[a].x, qv[a].y, qv[a].z, qv[a].w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    acc[a][0] = fmaf(qq[m], pv[m].x, acc[a][0]);
+                    acc[a][1] = fmaf(qq[m], pv[m].y, acc[a][1]);
+                    acc[a][2] = fmaf(qq[m], pv[m].z, acc[a][2]);
+                    acc[a][3] = fmaf(qq[m], pv[m].w, acc[a][3]);
+                }
+            }
+        }
+        for (int j = 0; j < nt; ++j) {                 // masked in-tile term
+            const float4 sv = *reinterpret_cast<const float4 *>(sc + (ohh * LCLA_T + j) * LCLA_T + otq);
+            float vv[4];
+            load4(vraw + (j * LCLA_HG + ohh) * LCLA_D + c0, vv);
+            const float ss[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(ss[a], vv[c], acc[a][c]);
+        }
+        // denominators: the 8 lanes sharing these 4 tokens split the key dims
+        float den[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int tok = otq + a;
+            const int last = min(nt, (tok / L + 1) * L) - 1;   // last in-tile token of tok's block
+            const int lc = last < 0 ? 0 : last;
+            float dp = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int e = c0 + m;
+                const float zt = Rz[ohh * LCLA_D + e] + fk[(lc * LCLA_HG + ohh) * LCLA_D + e];
+                dp = fmaf(zt, fq[(tok * LCLA_HG + ohh) * LCLA_D + e], dp);
+            }
+            dp += __shfl_xor_sync(0xffffffffu, dp, 1);
+            dp += __shfl_xor_sync(0xffffffffu, dp, 2);
+            dp += __shfl_xor_sync(0xffffffffu, dp, 4);
+            den[a] = dp + eps;
+        }
+        if (h0 + ohh < p.H) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int tok = otq + a;
+                if (tok < nt) {
+                    const float r = 1.0f / den[a];
+                    float o[4] = {acc[a][0] * r, acc[a][1] * r, acc[a][2] * r, acc[a][3] * r};
+                    store4(out + (((size_t)b * p.N + (size_t)(t + tok)) * p.H + (h0 + ohh)) * LCLA_D + c0, o);
+                }
+            }
+        }
+        __syncthreads();
+
+        // R += tile state: per-warp partial over 16 tokens, fixed-order sum
+        {
+            const int rc0 = (lane >> 2) * 4, re0 = (lane & 3) * 8, rtq = (w & 3) * 16;
+            float ra[4][8];
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ra[ii][j] = 0.f;
+            for (int tt = 0; tt < 16; ++tt) {
+                const int tok = rtq + tt;
+                float vv[4];
+                load4(vraw + (tok * LCLA_HG + ohh) * LCLA_D + rc0, vv);
+                const float4 ka = *reinterpret_cast<const float4 *>(kt + (tok * LCLA_HG + ohh) * LCLA_D + re0);
+                const float4 kb = *reinterpret_cast<const float4 *>(kt + (tok * LCLA_HG + ohh) * LCLA_D + re0 + 4);
+                const float kk[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) ra[ii][j] = fmaf(vv[ii], kk[j], ra[ii][j]);
+            }
+            float *red = sc;                                 // [8 warps][D c][D e]
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) red[w * LCLA_D * LCLA_D + (rc0 + ii) * LCLA_D + re0 + j] = ra[ii][j];
+        }
+        __syncthreads();
+        for (int x = tid; x < LCLA_HG * LCLA_D * LCLA_D; x += 256) {
+            const int hh = x >> 10, ce = x & 1023, c = ce >> 5, e = ce & 31;
+            const float *r = sc + (hh * 4) * LCLA_D * LCLA_D + ce;
+            const float add = ((r[0] + r[LCLA_D * LCLA_D]) + r[2 * LCLA_D * LCLA_D]) + r[3 * LCLA_D * LCLA_D];
+            RT[hh * LCLA_D * LCLA_D + e * LCLA_D + c] += add;
+        }
+        if (tid < LCLA_HG * LCLA_D && nt > 0) {
+            const int hh = tid >> 5, e = tid & 31;
+            Rz[hh * LCLA_D + e] += fk[((nt - 1) * LCLA_HG + hh) * LCLA_D + e];
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Scan: partials -> prefixes, one CTA per (b, h), 264 threads x float4.
+// Block mode: pref[blk] = state_in + sum of all segments of blocks <= blk.
+// Chunk mode: pref[s]   = state_in + sum of segments < s.
+// state_out (may equal state_in) receives the total.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(264)
+scan_states(const LclaPlan p, const float *__restrict__ part, float *__restrict__ pref,
+            const float *state_in, float *state_out)
+{
+    const size_t bh = blockIdx.x;
+    const int tid = threadIdx.x;
+    const size_t stride = (size_t)p.B * p.H * (LCLA_SZ / 4);   // float4 per segment slice
+    const float4 *P = reinterpret_cast<const float4 *>(part) + bh * (LCLA_SZ / 4) + tid;
+    float4 *Q = reinterpret_cast<float4 *>(pref) + bh * (LCLA_SZ / 4) + tid;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (state_in) acc = reinterpret_cast<const float4 *>(state_in + bh * LCLA_SZ)[tid];
+    if (!p.chunk) {
+        for (int blk = 0; blk < p.nb; ++blk) {
+#pragma unroll 4
+            for (int j = 0; j < p.nsb; ++j) {
+                const float4 x = P[((size_t)blk * p.nsb + j) * stride];
+                acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+            }
+            Q[(size_t)blk * stride] = acc;
+        }
+    } else {
+#pragma unroll 4
+        for (int s = 0; s < p.nseg; ++s) {
+            Q[(size_t)s * stride] = acc;
+            const float4 x = P[(size_t)s * stride];
+            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+        }
+    }
+    if (state_out) reinterpret_cast<float4 *>(state_out + bh * LCLA_SZ)[tid] = acc;
+}
+
+}  // namespace lcla

@@ -1,0 +1,70 @@
+// lcla_plan.h -- how one call is cut into work units (host and device).
+//
+// Tokens of one (b, h) form blocks of block_len tokens; a token attends to
+// its own block and every earlier block ("Implementing Block Causal Linear
+// Attention for Long Video Generation with Sana", section "Chunk-Wise
+// Causality").  The kernels cut the sequence into *segments*, contiguous token
+// ranges that either
+//   - lie inside one block (block mode, block_len > LCLA_T): every token of
+//     the segment uses the inclusive prefix state of its block; or
+//   - hold whole blocks only (chunk mode, block_len <= LCLA_T): tiles of
+//     T = (LCLA_T / block_len) * block_len tokens, where a token uses the
+//     exclusive prefix at the tile start plus a masked term inside the tile.
+// Pass A reduces each segment to a partial state, the scan turns partials
+// into prefixes, pass C produces the outputs.
+#pragma once
+#include <stddef.h>
+
+#define LCLA_D 32                              // head dim served
+#define LCLA_HG 2                              // heads per CTA (FFMA path)
+#define LCLA_T 64                              // tokens per tile (FFMA path)
+#define LCLA_SZ ((LCLA_D + 1) * LCLA_D)        // floats per (S, z) state
+#define LCLA_TARGET_CTAS (148 * 4)             // CTAs per pass the plan aims for
+
+struct LclaPlan {
+    int B, H, N, L, dtype;
+    int chunk;     // 0: block mode, 1: chunk mode
+    int T;         // chunk mode: tokens per tile (whole blocks); block mode: LCLA_T
+    int nb;        // blocks
+    int nsb;       // block mode: segments per block
+    int tps;       // chunk mode: tiles per segment
+    int nseg;      // segments
+    int npref;     // prefix entries: block mode nb, chunk mode nseg
+    int ngroups;   // head groups of LCLA_HG heads
+    size_t part_off, pref_off, ws_bytes;   // workspace layout (bytes)
+};
+
+struct LclaSeg {
+    int t0, t1;    // token range [t0, t1), possibly empty
+    int blk;       // block mode: block index; chunk mode: -1
+};
+
+#ifdef __CUDACC__
+#define LCLA_HD __host__ __device__ __forceinline__
+#else
+#define LCLA_HD inline
+#endif
+
+LCLA_HD long long lcla_min_ll(long long a, long long b) { return a < b ? a : b; }
+
+// Token range of segment s.
+LCLA_HD LclaSeg lcla_segment(const LclaPlan &p, int s)
+{
+    LclaSeg g;
+    if (!p.chunk) {
+        g.blk = s / p.nsb;
+        const long long j = s - (long long)g.blk * p.nsb;
+        const long long b0 = (long long)g.blk * p.L;
+        const long long bl = lcla_min_ll(p.L, p.N - b0);
+        const long long nt = (bl + LCLA_T - 1) / LCLA_T;          // tiles in this block
+        const long long per = (nt + p.nsb - 1) / p.nsb;          // tiles per segment
+        g.t0 = (int)(b0 + lcla_min_ll(j * per * LCLA_T, bl));
+        g.t1 = (int)(b0 + lcla_min_ll((j + 1) * per * LCLA_T, bl));
+    } else {
+        const long long span = (long long)p.tps * p.T;
+        g.t0 = (int)lcla_min_ll((long long)s * span, p.N);
+        g.t1 = (int)lcla_min_ll((long long)g.t0 + span, p.N);
+        g.blk = -1;
+    }
+    return g;
+}

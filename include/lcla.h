@@ -1,0 +1,164 @@
+/*
+ * lcla.h -- block-causal ReLU linear attention with a carried fp32 state,
+ * for NVIDIA B200 (sm_100a).  C ABI: plain pointers and sizes only.
+ *
+ * The operation ("Implementing Block Causal Linear Attention for Long Video
+ * Generation with Sana": sections "The Linear Attention Kernel", "Rotary
+ * Position Embeddings", "Chunk-Wise Causality"; "Block Causal Linear
+ * Attention" note: "What SANA-Video Actually Uses"; "[feat] LongSANA" PR:
+ * causal linear attention KV cache).  Per batch entry b and head h, with
+ * phi = ReLU, R_n the rotary embedding at token n (interleaved pairs (2p,2p+1),
+ * (x,y) -> (x c - y s, x s + y c), c = rope_cos[n][p], s = rope_sin[n][p]) and
+ * blk(n) = n / block_len:
+ *
+ *   out_i = sum_{j: blk(j) <= blk(i)} v_j (R_j phi(k_j) . R_i phi(q_i))
+ *           / ( sum_{same j} phi(k_j) . phi(q_i) + eps )
+ *
+ * i.e. a token attends to every token of its own block (both directions) and
+ * of all earlier blocks.  The carried state of one (b, h) is
+ *   S[c][e] = sum_j v_j[c] (R_j phi(k_j))[e]      (d x d, row = value dim)
+ *   z[e]    = sum_j phi(k_j)[e]                     (d, unrotated key sum)
+ * stored as float32 [d+1][d]: rows 0..d-1 hold S, row d holds z.
+ *
+ * Layouts (row-major, C order):
+ *   q, k, v, out        [B, N, H, d], element type `dtype` (out has q's type)
+ *   rope_cos, rope_sin  [N, d/2] float32, shared by every b and h
+ *   state               [B, H, d+1, d] float32
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     allocates nothing, keeps no per-call state between calls, and never
+ *     frees caller memory.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.  Results are valid
+ *     once the stream has reached the work.
+ *   - Arguments are validated before anything is enqueued; on any error code
+ *     other than LCLA_ERR_CUDA nothing was enqueued and no memory was touched.
+ *   - Every array pointer must be 16-byte aligned (LCLA_ERR_MISALIGNED).
+ *   - d must be 32 (other head dims: LCLA_ERR_UNSUPPORTED).
+ *   - `out` must not overlap q, k, v, the tables, the state or the workspace
+ *     (LCLA_ERR_INVALID_ARG).
+ *   - eps must be finite and >= 0.
+ *   - The results do not depend on the stream or on run-to-run timing: the
+ *     kernels use no floating-point atomics, so identical calls give
+ *     bit-identical outputs.
+ */
+#ifndef LCLA_H
+#define LCLA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define LCLA_API __attribute__((visibility("default")))
+#else
+#define LCLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LCLA_OK = 0,
+    LCLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad dtype, overlap, bad eps */
+    LCLA_ERR_UNSUPPORTED = 2,   /* valid request this build does not serve (d != 32, N > 2^30) */
+    LCLA_ERR_MISALIGNED = 3,    /* an array pointer is not 16-byte aligned */
+    LCLA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the query says */
+    LCLA_ERR_CUDA = 5           /* a CUDA launch failed; see cudaGetLastError */
+} lcla_status;
+
+typedef enum {
+    LCLA_BF16 = 0,              /* q, k, v, out are bfloat16 */
+    LCLA_F32 = 1                /* q, k, v, out are float32 */
+} lcla_dtype;
+
+/*
+ * Workspace bytes lcla_forward needs for this problem (0 when the arguments
+ * are invalid).  Depends only on the arguments, never on the device.
+ */
+LCLA_API size_t lcla_forward_workspace_bytes(int B, int H, int N, int d, int block_len, int dtype);
+
+/*
+ * Whole-sequence forward.
+ *   q, k, v     [B, N, H, d] device, dtype.  Read only.
+ *   rope_cos/sin [N, d/2] float32 device.  Read only.
+ *   B, H >= 1; N >= 0 (N = 0: no outputs, state_out set to zero);
+ *   block_len >= 1 (the last block holds the N mod block_len leftover tokens).
+ *   eps         added to every denominator.
+ *   out         [B, N, H, d] device, dtype.  Written.
+ *   state_out   [B, H, d+1, d] float32 device, or NULL.  Written with the
+ *               state after the last block (S and z summed over all tokens).
+ *   workspace   device scratch of at least lcla_forward_workspace_bytes(...)
+ *               bytes, 16-byte aligned (may be NULL when that is 0).  Its
+ *               contents on entry are ignored; it must not be shared with
+ *               another call that is in flight at the same time.
+ * Returns an lcla_status.
+ */
+LCLA_API int lcla_forward(const void *q, const void *k, const void *v,
+                 const float *rope_cos, const float *rope_sin,
+                 int B, int H, int N, int d, int block_len, float eps,
+                 void *out, float *state_out, int dtype,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * lcla_forward plus pass timing: `events` points to 4 cudaEvent_t handles
+ * created by the caller (cudaEventDefault flags); they are recorded on
+ * `stream` before pass A (partial states), before the scan, before pass C
+ * (outputs) and after pass C, so cudaEventElapsedTime gives each pass's
+ * device time.  events == NULL behaves exactly like lcla_forward.  Same
+ * arguments, ownership and errors as lcla_forward.
+ */
+LCLA_API int lcla_forward_timed(const void *q, const void *k, const void *v,
+                 const float *rope_cos, const float *rope_sin,
+                 int B, int H, int N, int d, int block_len, float eps,
+                 void *out, float *state_out, int dtype,
+                 void *workspace, size_t workspace_bytes, void *stream,
+                 void *const *events);
+
+/* Workspace bytes lcla_step needs (0 when the arguments are invalid). */
+LCLA_API size_t lcla_step_workspace_bytes(int B, int H, int L, int d, int dtype);
+
+/*
+ * Streaming step: one block of L tokens against the carried state
+ * ("[feat] LongSANA" PR: multi-step denoising per chunk against the cache,
+ * and the cache's enable_save switch).
+ *   q, k, v     [B, L, H, d] device, dtype: the block's tokens.
+ *   cos/sin     [L, d/2] float32 device: table rows at the block's absolute
+ *               positions.
+ *   L >= 0 (L = 0: nothing is done).
+ *   state       [B, H, d+1, d] float32 device, in/out.  P = state + (S, z)
+ *               of this block; every output uses P.  save != 0: state
+ *               becomes P.  save == 0: state is not written (bit-unchanged),
+ *               so the same block can be evaluated again, e.g. once per
+ *               denoising step, before a final call with save = 1.
+ *   out         [B, L, H, d] device, dtype.  Written.
+ *   workspace   as for lcla_forward, sized by lcla_step_workspace_bytes.
+ * Returns an lcla_status.
+ */
+LCLA_API int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk,
+              const float *cos_blk, const float *sin_blk,
+              int B, int H, int L, int d, float eps,
+              float *state, int save, void *out, int dtype,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * How lcla_forward cuts this problem, for benchmarks and tests: writes
+ * info[0] = 1 when tiles hold whole blocks (block_len <= 64), else 0;
+ * info[1] = segments (partial states written by the first pass);
+ * info[2] = prefix states (blocks, or segments when info[0] = 1);
+ * info[3] = tokens per tile.  Returns an lcla_status; touches no device.
+ */
+LCLA_API int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,
+                                    int *info);
+
+/* Static, human-readable name of a status code. */
+LCLA_API const char *lcla_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+LCLA_API int lcla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCLA_H */

@@ -180,11 +180,32 @@ int lcla_oracle_masked(const void *q, const void *k, const void *v, int dtype,
     return 0;
 }
 
+/* (token, output slot) pair: requested rows are visited in token order. */
+typedef struct { int64_t tok, slot; } row_ref;
+
+static int row_ref_cmp(const void *a, const void *b)
+{
+    const row_ref *x = (const row_ref *)a, *y = (const row_ref *)b;
+    return (x->tok > y->tok) - (x->tok < y->tok);
+}
+
+/* out_i = (P S-part . R_i phi(q_i)) / (P z-part . phi(q_i) + eps) */
+static void eval_row(const void *q, int dtype, const float *cs, const float *sn, int N, int H,
+                     int d, int b, int h, long i, const double *P, double eps, double *o)
+{
+    double qf[256], qr[256];
+    load_row(q, dtype, N, H, d, b, i, h, qf);
+    apply_relu(qf, d);
+    rotate(qf, cs, sn, i, d, qr);
+    double den = dot(P + (size_t)d * d, qf, d) + eps;
+    for (int c = 0; c < d; ++c) o[c] = dot(P + (size_t)c * d, qr, d) / den;
+}
+
 /*
  * Block-recurrence form.  For each (b, h): start from state_in (zero when
- * NULL), add each block's local state (S_blk, z_blk) in block order, keep the
- * inclusive running sum P_blk, and evaluate every requested token of block blk
- * against P_blk.
+ * NULL), add each block's local state (S_blk, z_blk) in block order to the
+ * running sum P, and right after block blk evaluate that block's requested
+ * tokens against P (the inclusive sum through blk).
  *
  * state_in     [B, H, d+1, d] or NULL.
  * rows, nrows  as in the masked form; out [B, nrows, H, d] or NULL.
@@ -205,16 +226,23 @@ int lcla_oracle_recurrence(const void *q, const void *k, const void *v, int dtyp
         if (rows[r] < 0 || rows[r] >= N) return -1;
     const long nb = ((long)N + block_len - 1) / block_len;
     const size_t sz = (size_t)(d + 1) * d;
+    row_ref *order = (row_ref *)malloc(sizeof(row_ref) * (size_t)(nrows > 0 ? nrows : 1));
+    if (!order) return -1;
+    for (int64_t r = 0; r < nrows; ++r) {
+        order[r].tok = rows ? rows[r] : r;
+        order[r].slot = r;
+    }
+    if (rows) qsort(order, (size_t)nrows, sizeof(row_ref), row_ref_cmp);
     int failed = 0;
 
     #pragma omp parallel for schedule(dynamic, 1) collapse(2)
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H; ++h) {
-            double *P = (double *)calloc((size_t)nb * sz, sizeof(double));
             double *acc = (double *)calloc(sz, sizeof(double));
-            if (!P || !acc) { free(P); free(acc); failed = 1; continue; }
+            if (!acc) { failed = 1; continue; }
             if (state_in) memcpy(acc, state_in + ((size_t)b * H + h) * sz, sz * sizeof(double));
             double kf[256], kr[256], vj[256];
+            int64_t next = 0;    /* next entry of order[] to evaluate */
             for (long blk = 0; blk < nb; ++blk) {
                 long j0 = blk * (long)block_len, j1 = j0 + block_len;
                 if (j1 > N) j1 = N;
@@ -227,26 +255,17 @@ int lcla_oracle_recurrence(const void *q, const void *k, const void *v, int dtyp
                         for (int e = 0; e < d; ++e) acc[(size_t)c * d + e] += vj[c] * kr[e];
                     for (int e = 0; e < d; ++e) acc[(size_t)d * d + e] += kf[e];
                 }
-                memcpy(P + (size_t)blk * sz, acc, sz * sizeof(double));
+                if (prefix)
+                    memcpy(prefix + (((size_t)b * H + h) * nb + blk) * sz, acc, sz * sizeof(double));
+                for (; out && next < nrows && order[next].tok < j1; ++next)
+                    eval_row(q, dtype, rope_cos, rope_sin, N, H, d, b, h, (long)order[next].tok,
+                             acc, eps,
+                             out + (((size_t)b * nrows + (size_t)order[next].slot) * H + h) * (size_t)d);
             }
             if (state_out) memcpy(state_out + ((size_t)b * H + h) * sz, acc, sz * sizeof(double));
-            if (prefix) memcpy(prefix + ((size_t)b * H + h) * nb * sz, P, (size_t)nb * sz * sizeof(double));
-            if (out) {
-                double qf[256], qr[256];
-                for (int64_t r = 0; r < nrows; ++r) {
-                    long i = rows ? (long)rows[r] : (long)r;
-                    const double *Pi = P + (size_t)(i / block_len) * sz;
-                    load_row(q, dtype, N, H, d, b, i, h, qf);
-                    apply_relu(qf, d);
-                    rotate(qf, rope_cos, rope_sin, i, d, qr);
-                    double den = dot(Pi + (size_t)d * d, qf, d) + eps;
-                    double *o = out + (((size_t)b * nrows + (size_t)r) * H + h) * (size_t)d;
-                    for (int c = 0; c < d; ++c) o[c] = dot(Pi + (size_t)c * d, qr, d) / den;
-                }
-            }
-            free(P);
             free(acc);
         }
+    free(order);
     return failed ? -1 : 0;
 }
 

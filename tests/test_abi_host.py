@@ -1,0 +1,107 @@
+"""The C-ABI library on the host: it loads, exports every declared entry
+point, answers workspace queries, and rejects invalid calls before touching
+the GPU (every call here fails validation, so no kernel is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_causal_relu_b200 as lcla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA = range(6)
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "lcla.h")).read()
+    return sorted(set(re.findall(r"LCLA_API\s+[\w\s\*]+?\b(lcla_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert {"lcla_forward", "lcla_step", "lcla_forward_workspace_bytes",
+            "lcla_step_workspace_bytes", "lcla_status_string", "lcla_version"} <= set(names)
+    lib = ctypes.CDLL(lcla.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version():
+    for s in range(6):
+        assert lcla.lib.lcla_status_string(s)
+    assert b"unknown" in lcla.lib.lcla_status_string(99)
+    assert lcla.lib.lcla_version() >= 100
+
+
+def test_workspace_queries():
+    f = lcla.forward_workspace_bytes
+    assert f(1, 70, 32760, 32, 4680, lcla.BF16) > 0
+    assert f(1, 70, 32760, 32, 4680, lcla.BF16) % 256 == 0
+    assert f(1, 16, 65536, 32, 1, lcla.F32) > 0
+    assert f(1, 1, 0, 32, 4, lcla.BF16) == 0          # empty sequence needs nothing
+    assert f(0, 1, 10, 32, 4, lcla.BF16) == 0          # invalid -> 0
+    assert f(1, 1, 10, 64, 4, lcla.BF16) == 0          # unsupported -> 0
+    assert f(1, 1, 10, 32, 0, lcla.BF16) == 0
+    assert f(1, 1, 10, 32, 4, 7) == 0
+    # independent of anything but the arguments
+    assert f(2, 70, 63960, 32, 4680, 0) == f(2, 70, 63960, 32, 4680, 0)
+    assert lcla.step_workspace_bytes(2, 70, 4680, 32, lcla.BF16) > 0
+    assert lcla.step_workspace_bytes(2, 70, 0, 32, lcla.BF16) == 0
+
+
+A = 1 << 20   # fake, 16-byte aligned "device" addresses: validation never dereferences
+
+
+def fwd(**kw):
+    args = dict(q=A, k=2 * A, v=3 * A, c=4 * A, s=5 * A, B=1, H=2, N=100, d=32, L=10, eps=1e-8,
+                out=6 * A, st=7 * A, dtype=0, ws=8 * A, wsb=1 << 20, stream=None)
+    args.update(kw)
+    return lcla.lib.lcla_forward(args["q"], args["k"], args["v"], args["c"], args["s"], args["B"],
+                                 args["H"], args["N"], args["d"], args["L"], args["eps"],
+                                 args["out"], args["st"], args["dtype"], args["ws"], args["wsb"],
+                                 args["stream"])
+
+
+def stp(**kw):
+    args = dict(q=A, k=2 * A, v=3 * A, c=4 * A, s=5 * A, B=1, H=2, L=100, d=32, eps=1e-8,
+                st=7 * A, save=1, out=6 * A, dtype=0, ws=8 * A, wsb=1 << 20, stream=None)
+    args.update(kw)
+    return lcla.lib.lcla_step(args["q"], args["k"], args["v"], args["c"], args["s"], args["B"],
+                              args["H"], args["L"], args["d"], args["eps"], args["st"], args["save"],
+                              args["out"], args["dtype"], args["ws"], args["wsb"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(k=None), INVALID), (dict(v=None), INVALID),
+    (dict(c=None), INVALID), (dict(s=None), INVALID), (dict(out=None), INVALID),
+    (dict(N=-1), INVALID), (dict(B=0), INVALID), (dict(H=0), INVALID), (dict(B=-3), INVALID),
+    (dict(L=0), INVALID), (dict(L=-5), INVALID), (dict(d=0), INVALID), (dict(d=31), INVALID),
+    (dict(d=64), UNSUPPORTED), (dict(d=16), UNSUPPORTED), (dict(N=(1 << 30) + 1), UNSUPPORTED),
+    (dict(dtype=2), INVALID), (dict(dtype=-1), INVALID),
+    (dict(eps=-1.0), INVALID), (dict(eps=float("nan")), INVALID), (dict(eps=float("inf")), INVALID),
+    (dict(q=A + 8), MISALIGNED), (dict(k=2 * A + 4), MISALIGNED), (dict(v=3 * A + 2), MISALIGNED),
+    (dict(c=4 * A + 8), MISALIGNED), (dict(out=6 * A + 1), MISALIGNED), (dict(st=7 * A + 4), MISALIGNED),
+    (dict(ws=8 * A + 8), MISALIGNED),
+    (dict(ws=None), WORKSPACE), (dict(wsb=16), WORKSPACE),
+    (dict(out=A), INVALID), (dict(out=2 * A + 64), INVALID), (dict(out=3 * A - 64), INVALID),
+    (dict(out=4 * A), INVALID), (dict(out=7 * A), INVALID), (dict(out=8 * A + 4096), INVALID),
+    (dict(ws=A), INVALID), (dict(st=A + 256), INVALID),
+])
+def test_forward_rejects(kw, code):
+    assert fwd(**kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(st=None), INVALID), (dict(q=None), INVALID), (dict(L=-1), INVALID), (dict(B=0), INVALID),
+    (dict(d=64), UNSUPPORTED), (dict(dtype=5), INVALID), (dict(st=7 * A + 8), MISALIGNED),
+    (dict(ws=None), WORKSPACE), (dict(out=3 * A), INVALID), (dict(st=5 * A), INVALID),
+    (dict(eps=-0.5), INVALID),
+])
+def test_step_rejects(kw, code):
+    assert stp(**kw) == code
+
+
+def test_trivial_calls_need_no_gpu():
+    # an empty block is a valid no-op and touches nothing
+    assert stp(L=0, q=None, k=None, v=None, c=None, s=None, out=None, ws=None, wsb=0) == OK

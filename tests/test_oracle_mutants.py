@@ -43,14 +43,11 @@ MUTANTS = {
     "recurrence_transposed_state": [("acc[(size_t)c * d + e] += vj[c] * kr[e];",
                                      "acc[(size_t)e * d + c] += vj[c] * kr[e];")],
     "recurrence_rotated_key_sum": [("acc[(size_t)d * d + e] += kf[e];", "acc[(size_t)d * d + e] += kr[e];")],
-    "recurrence_dropped_eps": [("double den = dot(Pi + (size_t)d * d, qf, d) + eps;",
-                                "double den = dot(Pi + (size_t)d * d, qf, d);")],
-    "recurrence_exclusive_prefix": [("const double *Pi = P + (size_t)(i / block_len) * sz;",
-                                     "const double *Pi = P + (size_t)(i / block_len > 0 ? i / block_len - 1 : 0) * sz;")],
-    "recurrence_unrotated_query": [("                    rotate(qf, rope_cos, rope_sin, i, d, qr);\n"
-                                    "                    double den = dot(Pi",
-                                    "                    rotate(qf, rope_cos, rope_sin, 0, d, qr);\n"
-                                    "                    double den = dot(Pi")],
+    "recurrence_dropped_eps": [("double den = dot(P + (size_t)d * d, qf, d) + eps;",
+                                "double den = dot(P + (size_t)d * d, qf, d);")],
+    "recurrence_exclusive_prefix": [("order[next].tok < j1;", "order[next].tok < j0;")],
+    "recurrence_unrotated_query": [("    rotate(qf, cs, sn, i, d, qr);\n    double den = dot(P",
+                                    "    rotate(qf, cs, sn, 0, d, qr);\n    double den = dot(P")],
     # step route
     "step_ignores_carried_state": [("S[x] += st[x];", "S[x] += 0.0 * st[x];")],
     "step_save_inverted": [("if (save) memcpy(st, S,", "if (!save) memcpy(st, S,")],
