@@ -30,15 +30,16 @@ def ulp(x: np.ndarray, dtype: str) -> np.ndarray:
     return np.exp2(np.floor(np.log2(ax)) - mant)
 
 
-def output_excess(o: np.ndarray, r: np.ndarray, dtype: str) -> np.ndarray:
+def output_excess(o: np.ndarray, r: np.ndarray, dtype: str, ulps: float = 0.5) -> np.ndarray:
     """Per-row worst excess of the error over its allowance, divided by the
     row scale; values <= tol pass.  Rows with zero scale give 0 when exact and
-    +inf otherwise."""
+    +inf otherwise.  ``ulps`` is the rounding allowance in output ulps: 1/2
+    against the unrounded oracle, 1 when both sides are rounded outputs."""
     o = np.asarray(o, np.float64)
     r = np.asarray(r, np.float64)
     assert o.shape == r.shape, (o.shape, r.shape)
     scale = np.abs(r).max(axis=-1)
-    err = np.abs(o - r) - 0.5 * ulp(np.maximum(np.abs(o), np.abs(r)), dtype)
+    err = np.abs(o - r) - ulps * ulp(np.maximum(np.abs(o), np.abs(r)), dtype)
     worst = np.maximum(err.max(axis=-1), 0.0)
     with np.errstate(divide="ignore", invalid="ignore"):
         rel = np.where(scale > 0, worst / np.where(scale > 0, scale, 1.0),
@@ -46,8 +47,8 @@ def output_excess(o: np.ndarray, r: np.ndarray, dtype: str) -> np.ndarray:
     return rel
 
 
-def check_outputs(o, r, dtype: str, what: str = "") -> float:
-    rel = output_excess(o, r, dtype)
+def check_outputs(o, r, dtype: str, what: str = "", ulps: float = 0.5) -> float:
+    rel = output_excess(o, r, dtype, ulps)
     worst = float(rel.max()) if rel.size else 0.0
     if not np.isfinite(o).all():
         raise AssertionError(f"{what}: non-finite outputs")
