@@ -102,10 +102,10 @@ def step_workspace_bytes(B: int, H: int, L: int, d: int, dtype: int) -> int:
 
 def plan_info(B: int, H: int, N: int, d: int, block_len: int, dtype: int) -> dict:
     """The library's cut of a forward problem (see ``lcla_forward_plan_info``)."""
-    info = (ctypes.c_int * 4)()
+    info = (ctypes.c_int * 5)()
     _check(lib.lcla_forward_plan_info(B, H, N, d, block_len, dtype, info))
     return {"chunk_mode": bool(info[0]), "segments": info[1], "prefixes": info[2],
-            "tile_tokens": info[3]}
+            "tile_tokens": info[3], "tensor_cores": bool(info[4])}
 
 
 def _stream(stream, device) -> int:

@@ -4,14 +4,19 @@
 // the work plan, and launches pass A (segment partial states), the scan
 // (prefix states, carried state in/out) and pass C (outputs) on the caller's
 // stream.  Allocates nothing.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "lcla.h"
 #include "lcla_ffma.cuh"
 #include "lcla_plan.h"
+#include "lcla_tc.cuh"
 
 namespace {
 
@@ -32,7 +37,7 @@ int check_shape(int B, int H, int N, int d, int L, int dtype)
 }
 
 // Cut the problem into segments (see lcla_plan.h) and lay out the workspace:
-// [part: nseg x B x H x (d+1) x d fp32][pref: npref x B x H x (d+1) x d fp32].
+// [status word, 256 B][part: nseg x B x H x (d+1) x d fp32][pref: npref x B x H x (d+1) x d fp32].
 LclaPlan make_plan(int B, int H, int N, int L, int dtype)
 {
     LclaPlan p;
@@ -44,9 +49,26 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
     const long long units = (long long)p.ngroups * B;
     if (L > LCLA_T) {
         p.chunk = 0;
-        p.T = LCLA_T;
-        const long long tpb = ((long long)(L < N ? L : N) + LCLA_T - 1) / LCLA_T;   // tiles per full block
-        long long nsb = (LCLA_TARGET_CTAS + units * p.nb - 1) / (units * p.nb);
+        p.tc = dtype == LCLA_BF16;
+        p.T = p.tc ? LCLA_TC_T : LCLA_T;
+        const long long tpb = ((long long)(L < N ? L : N) + p.T - 1) / p.T;   // tiles per full block
+        long long nsb;
+        if (p.tc) {
+            // One resident CTA per SM: the smallest split whose CTA count fills
+            // at least one wave and whose last wave is >= 90% full.
+            const long long base = units * p.nb;
+            long long best = 1;
+            double best_eff = 0.0;
+            for (nsb = 1; nsb <= tpb && nsb <= 64; ++nsb) {
+                const double waves = (double)(base * nsb) / LCLA_SMS;
+                const double eff = waves / (double)(long long)(waves + 0.999999);
+                if (eff > best_eff + 1e-9) { best_eff = eff; best = nsb; }
+                if (waves >= 0.9 && eff >= 0.9) { best = nsb; break; }
+            }
+            nsb = best;
+        } else {
+            nsb = (LCLA_TARGET_CTAS + units * p.nb - 1) / (units * p.nb);
+        }
         if (nsb > tpb) nsb = tpb;
         if (nsb < 1) nsb = 1;
         p.nsb = (int)nsb;
@@ -64,8 +86,8 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
         p.npref = p.nseg;
     }
     const size_t slice = (size_t)B * H * LCLA_SZ * sizeof(float);
-    p.part_off = 0;
-    p.pref_off = round_up((size_t)p.nseg * slice);
+    p.part_off = kAlign;
+    p.pref_off = p.part_off + round_up((size_t)p.nseg * slice);
     p.ws_bytes = p.pref_off + round_up((size_t)p.npref * slice);
     return p;
 }
@@ -86,6 +108,79 @@ void set_smem(F *kernel, int bytes)
     cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// [B, N, H*d] bf16 viewed as a 3-D tensor; box = 2 heads x 128 tokens, 128-byte swizzle.
+bool map_tokens(CUtensorMap *m, const void *base, int B, int N, int H)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)H * LCLA_D, (cuuint64_t)N, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)H * LCLA_D * 2, (cuuint64_t)N * H * LCLA_D * 2};
+    cuuint32_t box[3] = {LCLA_HG * LCLA_D, LCLA_TC_T, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [N, d/2] fp32 rotary table; box = 128 tokens, 64-byte swizzle.
+bool map_table(CUtensorMap *m, const float *base, int N)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {LCLA_D / 2, (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)(LCLA_D / 2) * 4};
+    cuuint32_t box[2] = {LCLA_D / 2, LCLA_TC_T};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor-core path: returns false (nothing enqueued) when a tensor map cannot
+// be encoded, so that the caller can run the CUDA-core kernels instead.
+bool launch_tc(const void *q, const void *k, const void *v, const float *rc, const float *rs,
+               const LclaPlan &p, float eps, void *out, const float *state_in, float *state_out,
+               unsigned char *ws, cudaStream_t st, cudaEvent_t const *ev, int *rc_out)
+{
+    CUtensorMap mq, mk, mv, mo, mc, ms;
+    if (!map_tokens(&mq, q, p.B, p.N, p.H) || !map_tokens(&mk, k, p.B, p.N, p.H) ||
+        !map_tokens(&mv, v, p.B, p.N, p.H) || !map_tokens(&mo, out, p.B, p.N, p.H) ||
+        !map_table(&mc, rc, p.N) || !map_table(&ms, rs, p.N))
+        return false;
+    float *part = reinterpret_cast<float *>(ws + p.part_off);
+    float *pref = reinterpret_cast<float *>(ws + p.pref_off);
+    int *status = reinterpret_cast<int *>(ws);
+    const dim3 grid(p.nseg, p.ngroups, p.B);
+    set_smem(lcla::tc::pass_a_tc, lcla::tc::LayA::BYTES);
+    set_smem(lcla::tc::pass_c_tc, lcla::tc::LayC::BYTES);
+    cudaMemsetAsync(status, 0, sizeof(int), st);
+    if (ev) cudaEventRecord(ev[0], st);
+    lcla::tc::pass_a_tc<<<grid, 256, lcla::tc::LayA::BYTES, st>>>(mk, mv, mc, ms, p, part, status);
+    if (ev) cudaEventRecord(ev[1], st);
+    lcla::scan_states<<<p.B * p.H, 264, 0, st>>>(p, part, pref, state_in, state_out);
+    if (ev) cudaEventRecord(ev[2], st);
+    lcla::tc::pass_c_tc<<<grid, 256, lcla::tc::LayC::BYTES, st>>>(mq, mc, ms, mo, p, pref, eps,
+                                                                  (__nv_bfloat16 *)out, status);
+    if (ev) cudaEventRecord(ev[3], st);
+    *rc_out = cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
+    return true;
+}
+
 template <typename Tin>
 int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const float *rs,
                const LclaPlan &p, float eps, Tin *out, const float *state_in, float *state_out,
@@ -95,6 +190,7 @@ int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const 
     float *part = reinterpret_cast<float *>(ws + p.part_off);
     float *pref = reinterpret_cast<float *>(ws + p.pref_off);
     const dim3 grid(p.nseg, p.ngroups, p.B);
+    cudaMemsetAsync(ws, 0, sizeof(int), st);   // status word (no CUDA-core kernel sets it)
 
     const int smem_a = 2 * (2 * G::TILE_IN + 2 * G::TILE_TAB) + G::TILE_F;
     set_smem(lcla::pass_a_ffma<Tin>, smem_a);
@@ -125,6 +221,11 @@ int run(const void *q, const void *k, const void *v, const float *rc, const floa
         const LclaPlan &p, float eps, void *out, const float *state_in, float *state_out,
         void *ws, cudaStream_t st, cudaEvent_t const *ev = nullptr)
 {
+    if (p.tc) {
+        int status = LCLA_OK;
+        if (launch_tc(q, k, v, rc, rs, p, eps, out, state_in, state_out, (unsigned char *)ws, st, ev, &status))
+            return status;
+    }
     if (p.dtype == LCLA_BF16)
         return launch_all<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
                                          (const __nv_bfloat16 *)v, rc, rs, p, eps,
@@ -245,6 +346,7 @@ int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,
     info[1] = p.nseg;
     info[2] = p.npref;
     info[3] = p.T;
+    info[4] = p.tc;
     return LCLA_OK;
 }
 

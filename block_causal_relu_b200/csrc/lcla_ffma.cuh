@@ -630,6 +630,7 @@ __global__ void __launch_bounds__(264)
 scan_states(const LclaPlan p, const float *__restrict__ part, float *__restrict__ pref,
             const float *state_in, float *state_out)
 {
+    constexpr int BATCH = 16;   // partials loaded before they are summed (independent loads in flight)
     const size_t bh = blockIdx.x;
     const int tid = threadIdx.x;
     const size_t stride = (size_t)p.B * p.H * (LCLA_SZ / 4);   // float4 per segment slice
@@ -637,21 +638,22 @@ scan_states(const LclaPlan p, const float *__restrict__ part, float *__restrict_
     float4 *Q = reinterpret_cast<float4 *>(pref) + bh * (LCLA_SZ / 4) + tid;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (state_in) acc = reinterpret_cast<const float4 *>(state_in + bh * LCLA_SZ)[tid];
-    if (!p.chunk) {
-        for (int blk = 0; blk < p.nb; ++blk) {
-#pragma unroll 4
-            for (int j = 0; j < p.nsb; ++j) {
-                const float4 x = P[((size_t)blk * p.nsb + j) * stride];
-                acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+    // Segments are summed in index order.  Block mode writes the running sum
+    // after the last segment of every block (inclusive prefix per block);
+    // chunk mode writes it before every segment (exclusive prefix).
+    for (int s0 = 0; s0 < p.nseg; s0 += BATCH) {
+        float4 x[BATCH];
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j)
+            if (s0 + j < p.nseg) x[j] = P[(size_t)(s0 + j) * stride];
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) {
+            const int s = s0 + j;
+            if (s < p.nseg) {
+                if (p.chunk) Q[(size_t)s * stride] = acc;
+                acc.x += x[j].x; acc.y += x[j].y; acc.z += x[j].z; acc.w += x[j].w;
+                if (!p.chunk && (s + 1) % p.nsb == 0) Q[(size_t)(s / p.nsb) * stride] = acc;
             }
-            Q[(size_t)blk * stride] = acc;
-        }
-    } else {
-#pragma unroll 4
-        for (int s = 0; s < p.nseg; ++s) {
-            Q[(size_t)s * stride] = acc;
-            const float4 x = P[(size_t)s * stride];
-            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
         }
     }
     if (state_out) reinterpret_cast<float4 *>(state_out + bh * LCLA_SZ)[tid] = acc;

@@ -16,15 +16,18 @@
 #include <stddef.h>
 
 #define LCLA_D 32                              // head dim served
-#define LCLA_HG 2                              // heads per CTA (FFMA path)
-#define LCLA_T 64                              // tokens per tile (FFMA path)
+#define LCLA_HG 2                              // heads per CTA (both paths)
+#define LCLA_T 64                              // tokens per tile (CUDA-core path)
+#define LCLA_TC_T 128                          // tokens per tile (tensor-core path)
 #define LCLA_SZ ((LCLA_D + 1) * LCLA_D)        // floats per (S, z) state
-#define LCLA_TARGET_CTAS (148 * 4)             // CTAs per pass the plan aims for
+#define LCLA_SMS 148                           // B200 streaming multiprocessors
+#define LCLA_TARGET_CTAS (LCLA_SMS * 4)        // CTAs per pass the CUDA-core plan aims for
 
 struct LclaPlan {
     int B, H, N, L, dtype;
     int chunk;     // 0: block mode, 1: chunk mode
-    int T;         // chunk mode: tokens per tile (whole blocks); block mode: LCLA_T
+    int tc;        // 1: tensor-core kernels (bf16, block mode), 0: CUDA-core kernels
+    int T;         // chunk mode: tokens per tile (whole blocks); block mode: tile tokens
     int nb;        // blocks
     int nsb;       // block mode: segments per block
     int tps;       // chunk mode: tiles per segment
@@ -56,10 +59,10 @@ LCLA_HD LclaSeg lcla_segment(const LclaPlan &p, int s)
         const long long j = s - (long long)g.blk * p.nsb;
         const long long b0 = (long long)g.blk * p.L;
         const long long bl = lcla_min_ll(p.L, p.N - b0);
-        const long long nt = (bl + LCLA_T - 1) / LCLA_T;          // tiles in this block
+        const long long nt = (bl + p.T - 1) / p.T;               // tiles in this block
         const long long per = (nt + p.nsb - 1) / p.nsb;          // tiles per segment
-        g.t0 = (int)(b0 + lcla_min_ll(j * per * LCLA_T, bl));
-        g.t1 = (int)(b0 + lcla_min_ll((j + 1) * per * LCLA_T, bl));
+        g.t0 = (int)(b0 + lcla_min_ll(j * per * p.T, bl));
+        g.t1 = (int)(b0 + lcla_min_ll((j + 1) * per * p.T, bl));
     } else {
         const long long span = (long long)p.tps * p.T;
         g.t0 = (int)lcla_min_ll((long long)s * span, p.N);

@@ -146,7 +146,9 @@ LCLA_API int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk,
  * info[0] = 1 when tiles hold whole blocks (block_len <= 64), else 0;
  * info[1] = segments (partial states written by the first pass);
  * info[2] = prefix states (blocks, or segments when info[0] = 1);
- * info[3] = tokens per tile.  Returns an lcla_status; touches no device.
+ * info[3] = tokens per tile; info[4] = 1 when the tensor-core kernels run
+ * (bf16 with block_len > 64), else 0.  `info` holds 5 ints.  Returns an
+ * lcla_status; touches no device.
  */
 LCLA_API int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,
                                     int *info);
