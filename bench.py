@@ -291,11 +291,12 @@ def main():
     for _ in range(W):
         step()
     barrier()
+    # timed region 1: the headline number, plain calls back to back
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(device) as clk:
         e0.record(stream)
         for i in range(K):
-            step(evs[i])
+            step()
         e1.record(stream)
         torch.cuda.synchronize(device)
     barrier()
@@ -303,6 +304,12 @@ def main():
     ms = ms_total / K
     units = spec.token_heads
     value = world * units * K / (ms_total / 1e3)
+    # timed region 2: the same steps with events recorded between the passes
+    # (lcla_forward_timed) for the per-kernel durations of the roofline
+    for i in range(K):
+        step(evs[i])
+    torch.cuda.synchronize(device)
+    barrier()
 
     # per-pass device times over the timed region
     pa = [r[0].elapsed_time(r[1]) for r in evs]

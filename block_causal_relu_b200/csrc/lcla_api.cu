@@ -31,7 +31,7 @@ int check_shape(int B, int H, int N, int d, int L, int dtype)
     if (d & 1) return LCLA_ERR_INVALID_ARG;
     if (d != LCLA_D) return LCLA_ERR_UNSUPPORTED;
     if (N > (1 << 30)) return LCLA_ERR_UNSUPPORTED;
-    if (B > 65535 || (H + LCLA_HG - 1) / LCLA_HG > 65535) return LCLA_ERR_UNSUPPORTED;
+    if (B > 65535) return LCLA_ERR_UNSUPPORTED;
     if ((long long)B * H > 0x7fffffffLL) return LCLA_ERR_UNSUPPORTED;
     return LCLA_OK;
 }
@@ -54,13 +54,13 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
         const long long tpb = ((long long)(L < N ? L : N) + p.T - 1) / p.T;   // tiles per full block
         long long nsb;
         if (p.tc) {
-            // One resident CTA per SM: the smallest split whose CTA count fills
-            // at least one wave and whose last wave is >= 90% full.
+            // LCLA_TC_RESIDENT CTAs per SM: the smallest split whose CTA count
+            // fills at least one wave and whose last wave is >= 90% full.
             const long long base = units * p.nb;
             long long best = 1;
             double best_eff = 0.0;
             for (nsb = 1; nsb <= tpb && nsb <= 64; ++nsb) {
-                const double waves = (double)(base * nsb) / LCLA_SMS;
+                const double waves = (double)(base * nsb) / (LCLA_SMS * LCLA_TC_RESIDENT);
                 const double eff = waves / (double)(long long)(waves + 0.999999);
                 if (eff > best_eff + 1e-9) { best_eff = eff; best = nsb; }
                 if (waves >= 0.9 && eff >= 0.9) { best = nsb; break; }
@@ -92,6 +92,9 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
     return p;
 }
 
+// The launch grid flattens (segment, head group) into blockIdx.x.
+bool grid_fits(const LclaPlan &p) { return (long long)p.nseg * p.ngroups <= 0x7fffffffLL; }
+
 bool misaligned(const void *ptr) { return ((uintptr_t)ptr & 15u) != 0; }
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb)
@@ -99,6 +102,31 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb)
     if (!a || !b || !na || !nb) return false;
     const uintptr_t a0 = (uintptr_t)a, a1 = a0 + na, b0 = (uintptr_t)b, b1 = b0 + nb;
     return a0 < b1 && b0 < a1;
+}
+
+// Launch with programmatic dependent launch: the kernel may start while the
+// previous kernel of the stream finishes; it calls griddepcontrol.wait before
+// reading anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+unsigned scan_blocks(const LclaPlan &p)
+{
+    const size_t n = (size_t)p.B * p.H * LCLA_SZ;
+    return (unsigned)((n + lcla::SCAN_THREADS - 1) / lcla::SCAN_THREADS);
 }
 
 template <typename F>
@@ -165,17 +193,18 @@ bool launch_tc(const void *q, const void *k, const void *v, const float *rc, con
     float *part = reinterpret_cast<float *>(ws + p.part_off);
     float *pref = reinterpret_cast<float *>(ws + p.pref_off);
     int *status = reinterpret_cast<int *>(ws);
-    const dim3 grid(p.nseg, p.ngroups, p.B);
+    const dim3 grid(p.nseg * p.ngroups, p.B);
     set_smem(lcla::tc::pass_a_tc, lcla::tc::LayA::BYTES);
     set_smem(lcla::tc::pass_c_tc, lcla::tc::LayC::BYTES);
     cudaMemsetAsync(status, 0, sizeof(int), st);
     if (ev) cudaEventRecord(ev[0], st);
     lcla::tc::pass_a_tc<<<grid, 256, lcla::tc::LayA::BYTES, st>>>(mk, mv, mc, ms, p, part, status);
     if (ev) cudaEventRecord(ev[1], st);
-    lcla::scan_states<<<p.B * p.H, 264, 0, st>>>(p, part, pref, state_in, state_out);
+    launch_pdl(lcla::scan_states, dim3(scan_blocks(p)), dim3(lcla::SCAN_THREADS), 0, st, p, part, pref,
+               state_in, state_out);
     if (ev) cudaEventRecord(ev[2], st);
-    lcla::tc::pass_c_tc<<<grid, 256, lcla::tc::LayC::BYTES, st>>>(mq, mc, ms, mo, p, pref, eps,
-                                                                  (__nv_bfloat16 *)out, status);
+    launch_pdl(lcla::tc::pass_c_tc, grid, dim3(256), lcla::tc::LayC::BYTES, st, mq, mc, ms, mo, p,
+               (const float *)pref, eps, (__nv_bfloat16 *)out, status);
     if (ev) cudaEventRecord(ev[3], st);
     *rc_out = cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
     return true;
@@ -189,7 +218,7 @@ int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const 
     using G = lcla::Geo<Tin>;
     float *part = reinterpret_cast<float *>(ws + p.part_off);
     float *pref = reinterpret_cast<float *>(ws + p.pref_off);
-    const dim3 grid(p.nseg, p.ngroups, p.B);
+    const dim3 grid(p.nseg * p.ngroups, p.B);
     cudaMemsetAsync(ws, 0, sizeof(int), st);   // status word (no CUDA-core kernel sets it)
 
     const int smem_a = 2 * (2 * G::TILE_IN + 2 * G::TILE_TAB) + G::TILE_F;
@@ -198,19 +227,21 @@ int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const 
     lcla::pass_a_ffma<Tin><<<grid, 256, smem_a, st>>>(k, v, rc, rs, p, part);
 
     if (ev) cudaEventRecord(ev[1], st);
-    lcla::scan_states<<<p.B * p.H, 264, 0, st>>>(p, part, pref, state_in, state_out);
+    launch_pdl(lcla::scan_states, dim3(scan_blocks(p)), dim3(lcla::SCAN_THREADS), 0, st, p, part, pref,
+               state_in, state_out);
     if (ev) cudaEventRecord(ev[2], st);
 
     if (!p.chunk) {
         const int smem_c = 2 * (G::TILE_IN + 2 * G::TILE_TAB) + G::TILE_F +
                            (LCLA_HG * LCLA_D * LCLA_D + LCLA_HG * LCLA_D + LCLA_T * LCLA_HG) * 4;
         set_smem(lcla::pass_c_ffma<Tin>, smem_c);
-        lcla::pass_c_ffma<Tin><<<grid, 256, smem_c, st>>>(q, rc, rs, p, pref, eps, out);
+        launch_pdl(lcla::pass_c_ffma<Tin>, grid, dim3(256), smem_c, st, q, rc, rs, p, (const float *)pref, eps, out);
     } else {
         const int smem_c = 3 * G::TILE_IN + 2 * G::TILE_TAB + 4 * G::TILE_F +
                            (LCLA_HG * LCLA_T * LCLA_T + LCLA_HG * LCLA_D * LCLA_D + LCLA_HG * LCLA_D) * 4;
         set_smem(lcla::pass_c_chunk_ffma<Tin>, smem_c);
-        lcla::pass_c_chunk_ffma<Tin><<<grid, 256, smem_c, st>>>(q, k, v, rc, rs, p, pref, eps, out);
+        launch_pdl(lcla::pass_c_chunk_ffma<Tin>, grid, dim3(256), smem_c, st, q, k, v, rc, rs, p,
+                   (const float *)pref, eps, out);
     }
     if (ev) cudaEventRecord(ev[3], st);
     return cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
@@ -278,13 +309,15 @@ extern "C" {
 size_t lcla_forward_workspace_bytes(int B, int H, int N, int d, int block_len, int dtype)
 {
     if (check_shape(B, H, N, d, block_len, dtype) != LCLA_OK) return 0;
-    return make_plan(B, H, N, block_len, dtype).ws_bytes;
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    return grid_fits(p) ? p.ws_bytes : 0;
 }
 
 size_t lcla_step_workspace_bytes(int B, int H, int L, int d, int dtype)
 {
     if (check_shape(B, H, L, d, L < 1 ? 1 : L, dtype) != LCLA_OK) return 0;
-    return make_plan(B, H, L, L < 1 ? 1 : L, dtype).ws_bytes;
+    const LclaPlan p = make_plan(B, H, L, L < 1 ? 1 : L, dtype);
+    return grid_fits(p) ? p.ws_bytes : 0;
 }
 
 int lcla_forward_timed(const void *q, const void *k, const void *v, const float *rope_cos,
@@ -295,6 +328,7 @@ int lcla_forward_timed(const void *q, const void *k, const void *v, const float 
     int rc = check_shape(B, H, N, d, block_len, dtype);
     if (rc != LCLA_OK) return rc;
     const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
     rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, dtype, eps,
                        workspace, workspace_bytes, p.ws_bytes);
     if (rc != LCLA_OK) return rc;
@@ -327,6 +361,7 @@ int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk, const flo
     int rc = check_shape(B, H, L, d, L < 1 ? 1 : L, dtype);
     if (rc != LCLA_OK) return rc;
     const LclaPlan p = make_plan(B, H, L, L < 1 ? 1 : L, dtype);
+    if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
     rc = check_buffers(q_blk, k_blk, v_blk, cos_blk, sin_blk, out, state, true, B, H, L, dtype, eps,
                        workspace, workspace_bytes, p.ws_bytes);
     if (rc != LCLA_OK) return rc;
@@ -342,6 +377,7 @@ int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,
     if (rc != LCLA_OK) return rc;
     if (!info) return LCLA_ERR_INVALID_ARG;
     const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
     info[0] = p.chunk;
     info[1] = p.nseg;
     info[2] = p.npref;

@@ -37,6 +37,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
+// Programmatic dependent launch: wait until the preceding kernel of the
+// stream has completed (no-op when launched without the attribute), and let
+// the next kernel of the stream start its launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ReLU written as a comparison so that NaN passes through.
 __device__ __forceinline__ float relu(float x) { return x < 0.f ? 0.f : x; }
 
@@ -158,7 +164,7 @@ pass_a_ffma(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
     extern __shared__ __align__(128) unsigned char sm[];
     float *kt = reinterpret_cast<float *>(sm + 2 * STAGE);   // [T][HG][D] rotated features
 
-    const int s = blockIdx.x, h0 = blockIdx.y * LCLA_HG, b = blockIdx.z;
+    const int s = blockIdx.x / p.ngroups, h0 = (blockIdx.x % p.ngroups) * LCLA_HG, b = blockIdx.y;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const LclaSeg g = lcla_segment(p, s);
     const int ntile = (g.t1 - g.t0 + LCLA_T - 1) / LCLA_T;
@@ -234,6 +240,7 @@ pass_a_ffma(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
         __syncthreads();
     }
 
+    pdl_trigger();
     // fixed-order reduction of the 4 warps of each head and of the key sums
     float *red = reinterpret_cast<float *>(sm);                 // [8][D][D]
     float *zred = red + 8 * LCLA_D * LCLA_D;                     // [256][8]
@@ -279,11 +286,12 @@ pass_c_ffma(const Tin *__restrict__ q, const float *__restrict__ rcos, const flo
     float *zz = PT + LCLA_HG * LCLA_D * LCLA_D;                       // [HG][D]
     float *inv = zz + LCLA_HG * LCLA_D;                               // [T][HG]
 
-    const int s = blockIdx.x, h0 = blockIdx.y * LCLA_HG, b = blockIdx.z;
+    const int s = blockIdx.x / p.ngroups, h0 = (blockIdx.x % p.ngroups) * LCLA_HG, b = blockIdx.y;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const LclaSeg g = lcla_segment(p, s);
     const int ntile = (g.t1 - g.t0 + LCLA_T - 1) / LCLA_T;
     if (ntile <= 0) return;
+    pdl_wait();
 
     // prefix state of this block, transposed to [e][c]
     for (int x = tid; x < LCLA_HG * LCLA_SZ; x += 256) {
@@ -412,12 +420,13 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
     float *RT = sc + LCLA_HG * LCLA_T * LCLA_T;                       // [HG][D e][D c]
     float *Rz = RT + LCLA_HG * LCLA_D * LCLA_D;                       // [HG][D]
 
-    const int s = blockIdx.x, h0 = blockIdx.y * LCLA_HG, b = blockIdx.z;
+    const int s = blockIdx.x / p.ngroups, h0 = (blockIdx.x % p.ngroups) * LCLA_HG, b = blockIdx.y;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const LclaSeg g = lcla_segment(p, s);
     const int T = p.T, L = p.L;
     const int ntile = (g.t1 - g.t0 + T - 1) / T;
     if (ntile <= 0) return;
+    pdl_wait();
 
     for (int x = tid; x < LCLA_HG * LCLA_SZ; x += 256) {
         const int hh = x / LCLA_SZ, e = x - hh * LCLA_SZ;
@@ -621,42 +630,42 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
 }
 
 // ---------------------------------------------------------------------------
-// Scan: partials -> prefixes, one CTA per (b, h), 264 threads x float4.
+// Scan: partials -> prefixes, one thread per state element (b, h, x) with
+// x < (D+1)*D; the segment partials are loaded in batches of independent
+// loads and summed in segment order.
 // Block mode: pref[blk] = state_in + sum of all segments of blocks <= blk.
 // Chunk mode: pref[s]   = state_in + sum of segments < s.
 // state_out (may equal state_in) receives the total.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(264)
+constexpr int SCAN_THREADS = 256;
+
+__global__ void __launch_bounds__(SCAN_THREADS)
 scan_states(const LclaPlan p, const float *__restrict__ part, float *__restrict__ pref,
             const float *state_in, float *state_out)
 {
-    constexpr int BATCH = 16;   // partials loaded before they are summed (independent loads in flight)
-    const size_t bh = blockIdx.x;
-    const int tid = threadIdx.x;
-    const size_t stride = (size_t)p.B * p.H * (LCLA_SZ / 4);   // float4 per segment slice
-    const float4 *P = reinterpret_cast<const float4 *>(part) + bh * (LCLA_SZ / 4) + tid;
-    float4 *Q = reinterpret_cast<float4 *>(pref) + bh * (LCLA_SZ / 4) + tid;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (state_in) acc = reinterpret_cast<const float4 *>(state_in + bh * LCLA_SZ)[tid];
-    // Segments are summed in index order.  Block mode writes the running sum
-    // after the last segment of every block (inclusive prefix per block);
-    // chunk mode writes it before every segment (exclusive prefix).
+    constexpr int BATCH = 16;
+    const size_t n = (size_t)p.B * p.H * LCLA_SZ;                // elements of one slice
+    const size_t x = (size_t)blockIdx.x * SCAN_THREADS + threadIdx.x;
+    pdl_wait();
+    pdl_trigger();
+    if (x >= n) return;
+    float acc = state_in ? state_in[x] : 0.f;
     for (int s0 = 0; s0 < p.nseg; s0 += BATCH) {
-        float4 x[BATCH];
+        float v[BATCH];
 #pragma unroll
         for (int j = 0; j < BATCH; ++j)
-            if (s0 + j < p.nseg) x[j] = P[(size_t)(s0 + j) * stride];
+            if (s0 + j < p.nseg) v[j] = __ldcg(part + (size_t)(s0 + j) * n + x);
 #pragma unroll
         for (int j = 0; j < BATCH; ++j) {
             const int s = s0 + j;
             if (s < p.nseg) {
-                if (p.chunk) Q[(size_t)s * stride] = acc;
-                acc.x += x[j].x; acc.y += x[j].y; acc.z += x[j].z; acc.w += x[j].w;
-                if (!p.chunk && (s + 1) % p.nsb == 0) Q[(size_t)(s / p.nsb) * stride] = acc;
+                if (p.chunk) pref[(size_t)s * n + x] = acc;
+                acc += v[j];
+                if (!p.chunk && (s + 1) % p.nsb == 0) pref[(size_t)(s / p.nsb) * n + x] = acc;
             }
         }
     }
-    if (state_out) reinterpret_cast<float4 *>(state_out + bh * LCLA_SZ)[tid] = acc;
+    if (state_out) state_out[x] = acc;
 }
 
 }  // namespace lcla

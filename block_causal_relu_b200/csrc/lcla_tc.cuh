@@ -7,8 +7,12 @@
 // ReLU features), with the d x d contractions on the 5th-generation tensor
 // cores:
 //
-// Pass A, per CTA = (segment inside one block, head pair, batch entry), tiles
-// of 128 tokens.  The rotated keys are split into bf16 hi + lo parts
+// Two CTAs of 256 threads reside on each SM (about 105 KB of shared memory
+// each), so one CTA's barriers overlap the other's work.  Tiles hold 64
+// tokens; two threads share each (token, head) row, 16 elements each.
+//
+// Pass A, per CTA = (segment inside one block, head pair, batch entry).  The
+// rotated keys are split into bf16 hi + lo parts
 // (k~ = hi + lo to 2^-16 relative) and stacked as the 128 rows of the MMA's A
 // operand, [hi_h0; lo_h0; hi_h1; lo_h1] (MN-major, written by the threads);
 // V of the two heads is the B operand exactly as TMA lands it (MN-major,
@@ -20,11 +24,13 @@
 // cores from the same ReLU features.
 //
 // Pass C, per CTA = (segment, head pair, batch entry): the block's prefix
-// state P is split once into bf16 hi + lo and staged as the B operand
-// (K-major); per 128-token tile the rotated queries, split into hi + lo, form
-// the A operand (K-major) and
-//   D[tok][c] = q~hi.Phi + q~lo.Phi + q~hi.Plo   (6 MMAs of K = 16 per head)
-// is scaled by 1 / (z . phi(q) + eps) and stored through TMA.
+// state P of both heads is split once into bf16 hi + lo and staged as the B
+// operand (K-major rows (head, c) = [P hi | P lo]); per 64-token tile the
+// rotated queries of both heads, split into hi + lo, are the 128 rows
+// (head, token) of the A operand (K-major) and
+//   D[(h,tok)][(h',c)] = q~hi.Phi + q~lo.Phi + q~hi.Plo   (6 MMAs of K = 16)
+// (blocks h = h' used) is scaled by 1 / (z . phi(q) + eps) and stored
+// through TMA.
 //
 // Every wait on an mbarrier is bounded (LCLA_TC_WAIT_NS of globaltimer); a
 // timeout is voted across the CTA, the CTA waits (bounded) for its own
@@ -194,40 +200,57 @@ __device__ __forceinline__ void rope_split(const float *f, const float *cv, cons
     }
 }
 
-// Head h's 32 bf16 of row r of a [128][64] bf16 tile with 128-byte swizzle.
-__device__ __forceinline__ void load_head_row(const unsigned char *tile, int r, int h, float *x)
+// ReLU on two packed bf16 (NaN passes through).
+__device__ __forceinline__ uint32_t relu2(uint32_t w)
+{
+    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162 *>(&w);
+    x = __hmax2_nan(x, __floats2bfloat162_rn(0.f, 0.f));
+    return bf2_bits(x);
+}
+
+// Elements [16f, 16f+16) of head h in row r of a [64][64] bf16 tile with
+// 128-byte swizzle, as 8 packed bf16 pairs.
+__device__ __forceinline__ void load_half_row(const unsigned char *tile, int r, int h, int f, uint32_t *w)
 {
     const int sw = r & 7;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(tile + r * 128 + (((4 * h + j) ^ sw) << 4));
-        x[8 * j + 0] = bf_lo(u.x); x[8 * j + 1] = bf_hi(u.x);
-        x[8 * j + 2] = bf_lo(u.y); x[8 * j + 3] = bf_hi(u.y);
-        x[8 * j + 4] = bf_lo(u.z); x[8 * j + 5] = bf_hi(u.z);
-        x[8 * j + 6] = bf_lo(u.w); x[8 * j + 7] = bf_hi(u.w);
-    }
+    const uint4 a = *reinterpret_cast<const uint4 *>(tile + r * 128 + (((4 * h + 2 * f) ^ sw) << 4));
+    const uint4 b = *reinterpret_cast<const uint4 *>(tile + r * 128 + (((4 * h + 2 * f + 1) ^ sw) << 4));
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
 }
-// Row r of a [128][16] fp32 table tile with 64-byte swizzle.
-__device__ __forceinline__ void load_table_row(const unsigned char *tile, int r, float *x)
+// Pairs [8f, 8f+8) of row r of a [64][16] fp32 table tile with 64-byte swizzle.
+__device__ __forceinline__ void load_half_table(const unsigned char *tile, int r, int f, float *x)
 {
     const int sw = (r >> 1) & 3;
+    const float4 a = *reinterpret_cast<const float4 *>(tile + r * 64 + (((2 * f) ^ sw) << 4));
+    const float4 b = *reinterpret_cast<const float4 *>(tile + r * 64 + (((2 * f + 1) ^ sw) << 4));
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+// Rotate 8 pairs of (packed bf16) ReLU features and split each rotated value
+// into bf16 hi + lo (packed pairs).
+__device__ __forceinline__ void rope_split8(const uint32_t *fw, const float *cv, const float *sv, uint32_t *hi,
+                                            uint32_t *lo)
+{
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float4 a = *reinterpret_cast<const float4 *>(tile + r * 64 + ((j ^ sw) << 4));
-        x[4 * j + 0] = a.x; x[4 * j + 1] = a.y; x[4 * j + 2] = a.z; x[4 * j + 3] = a.w;
+    for (int p = 0; p < 8; ++p) {
+        const float a = bf_lo(fw[p]), b = bf_hi(fw[p]);
+        const float y0 = a * cv[p] - b * sv[p];
+        const float y1 = a * sv[p] + b * cv[p];
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+        const float2 hf = __bfloat1622float2(h2);
+        hi[p] = bf2_bits(h2);
+        lo[p] = bf2_bits(__floats2bfloat162_rn(y0 - hf.x, y1 - hf.y));
     }
 }
-// Row r of a 128-byte-swizzled operand row block: chunks 0-3 <- hi, 4-7 <- lo.
-__device__ __forceinline__ void store_hi_lo_row(unsigned char *tile, int r, const uint32_t *hi, const uint32_t *lo)
+// Half f of operand row r (128 B, 128-byte swizzle): hi -> chunks 2f, 2f+1; lo -> chunks 4+2f, 5+2f.
+__device__ __forceinline__ void store_half_hi_lo(unsigned char *tile, int r, int f, const uint32_t *hi,
+                                                 const uint32_t *lo)
 {
     const int sw = r & 7;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        *reinterpret_cast<uint4 *>(tile + r * 128 + ((j ^ sw) << 4)) =
-            make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
-        *reinterpret_cast<uint4 *>(tile + r * 128 + (((4 + j) ^ sw) << 4)) =
-            make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
-    }
+    unsigned char *row = tile + r * 128;
+    *reinterpret_cast<uint4 *>(row + (((2 * f) ^ sw) << 4)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4 *>(row + (((2 * f + 1) ^ sw) << 4)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+    *reinterpret_cast<uint4 *>(row + (((4 + 2 * f) ^ sw) << 4)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4 *>(row + (((5 + 2 * f) ^ sw) << 4)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
 }
 
 // ---------------------------------------------------------------------------
@@ -235,15 +258,15 @@ __device__ __forceinline__ void store_hi_lo_row(unsigned char *tile, int r, cons
 // ---------------------------------------------------------------------------
 struct LayA {
     static constexpr int STAGES = 3;
-    static constexpr int K_OFF = 0, V_OFF = 16384, C_OFF = 32768, S_OFF = 40960, STAGE = 49152;
-    static constexpr int A_OFF = STAGES * STAGE, A_BYTES = 32768;      // [hi_h0 lo_h0 | hi_h1 lo_h1] x 128 tokens
+    static constexpr int K_OFF = 0, V_OFF = 8192, C_OFF = 16384, S_OFF = 20480, STAGE = 24576;
+    static constexpr int A_OFF = STAGES * STAGE, A_BYTES = 16384;   // per buffer: head 0 | head 1, [64 tok][128 B]
     static constexpr int CTRL = A_OFF + 2 * A_BYTES;
-    static constexpr int BYTES = CTRL + 128 + 1024;                    // + alignment slack
+    static constexpr int BYTES = CTRL + 128 + 1024;                 // + alignment slack
     static constexpr uint32_t TX = STAGE;
     static constexpr uint32_t IDESC = idesc_bf16(128, 64, 1, 1);
 };
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, 2)
 pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
           const __grid_constant__ CUtensorMap mc, const __grid_constant__ CUtensorMap ms,
           const LclaPlan p, float *__restrict__ part, int *__restrict__ status)
@@ -257,7 +280,7 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
     const uint32_t full0 = sb + L::CTRL, done0 = full0 + 8 * L::STAGES;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 64);
 
-    const int s = blockIdx.x, hp = blockIdx.y, b = blockIdx.z;
+    const int s = blockIdx.x / p.ngroups, hp = blockIdx.x % p.ngroups, b = blockIdx.y;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const LclaSeg g = lcla_segment(p, s);
     const int ntile = g.t1 > g.t0 ? (g.t1 - g.t0 + T - 1) / T : 0;
@@ -276,15 +299,12 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
     tc_after();
     const uint32_t tmem = *tslot;
 
-    const int r = ((w & 3) << 5) | lane;    // prologue: token row of the tile
-    const int h = w >> 2;                    // prologue: head of the pair
-    const int q4 = w & 3, ch = w >> 2;       // drain: tensor-memory lane quarter, column half
+    const int r = tid & 63, h = (tid >> 6) & 1, f = tid >> 7;   // prologue: token row, head, half
+    const int q4 = w & 3, ch = w >> 2;                            // drain: lane quarter, column half
 
-    float zacc[32], sacc[16];
+    float zacc[16], sacc[16];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) zacc[j] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) sacc[j] = 0.f;
+    for (int j = 0; j < 16; ++j) zacc[j] = sacc[j] = 0.f;
     int loaded = 0, consumed = 0, issued = 0, drained = 0;
     bool bad = false;
 
@@ -315,34 +335,32 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
         const int t = g.t0 + i * T, nt = min(T, g.t1 - t);
 
         bool ok = bar_wait(full0 + 8 * st, (uint32_t)((i / L::STAGES) & 1));
-        if (__syncthreads_or(!ok)) { bad = true; break; }
-        consumed = i + 1;
-
-        // phi, key sum, rotary, hi/lo split -> A operand rows of token r, head h
-        {
-            const bool valid = r < nt;
-            float f[32], cv[16], sv[16];
-            load_head_row(stg + L::K_OFF, r, h, f);
-            load_table_row(stg + L::C_OFF, r, cv);
-            load_table_row(stg + L::S_OFF, r, sv);
+        {   // phi, key sum, rotary, hi/lo split -> A operand (MN-major) of token r, head h, half f
+            const bool valid = ok && r < nt;
+            uint32_t fw[8], hi[8], lo[8];
+            float cv[8], sv[8];
+            load_half_row(stg + L::K_OFF, r, h, f, fw);
+            load_half_table(stg + L::C_OFF, r, f, cv);
+            load_half_table(stg + L::S_OFF, r, f, sv);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                f[j] = valid ? relu(f[j]) : 0.f;
-                zacc[j] += f[j];
+            for (int j = 0; j < 8; ++j) {
+                fw[j] = valid ? relu2(fw[j]) : 0u;
+                zacc[2 * j] += bf_lo(fw[j]);
+                zacc[2 * j + 1] += bf_hi(fw[j]);
             }
-            uint32_t hi[16], lo[16];
-            rope_split(f, cv, sv, hi, lo);
-            store_hi_lo_row(sm + L::A_OFF + ab * L::A_BYTES + h * 16384, r, hi, lo);
-            if (!valid) {   // rows past the segment belong to another CTA: zero this head's V row
+            rope_split8(fw, cv, sv, hi, lo);
+            store_half_hi_lo(sm + L::A_OFF + ab * L::A_BYTES + h * 8192, r, f, hi, lo);
+            if (!valid) {   // rows past the segment belong to another CTA: zero this half of V
                 const int sw = r & 7;
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    *reinterpret_cast<uint4 *>(stg + L::V_OFF + r * 128 + (((4 * h + j) ^ sw) << 4)) =
-                        make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(stg + L::V_OFF + r * 128 + (((4 * h + 2 * f) ^ sw) << 4)) =
+                    make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(stg + L::V_OFF + r * 128 + (((4 * h + 2 * f + 1) ^ sw) << 4)) =
+                    make_uint4(0u, 0u, 0u, 0u);
             }
         }
         fence_async_smem();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) { bad = true; break; }
+        consumed = i + 1;
 
         if (tid == 0) {
             tc_after();
@@ -351,32 +369,33 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
             const uint32_t v0 = sb + st * L::STAGE + L::V_OFF;
 #pragma unroll
             for (int j = 0; j < T / 16; ++j)
-                mma_bf16(d, desc_sw128(a0 + 2048 * j, 16384, 1024), desc_sw128(v0 + 2048 * j, 16384, 1024),
+                mma_bf16(d, desc_sw128(a0 + 2048 * j, 8192, 1024), desc_sw128(v0 + 2048 * j, 8192, 1024),
                          L::IDESC, j > 0);
             mma_commit(done0 + 8 * ab);
         }
         issued = i + 1;
 
+        ok = true;
         if (i >= 1) {
             ok = bar_wait(done0 + 8 * ((i - 1) & 1), (uint32_t)(((i - 1) >> 1) & 1));
-            if (__syncthreads_or(!ok)) { bad = true; break; }
-            tc_after();
-            drain((i - 1) & 1);
-            drained = i;
+            if (ok) {
+                tc_after();
+                drain((i - 1) & 1);
+            }
         }
         tc_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) { bad = true; break; }
+        drained = i;
         if (tid == 0 && loaded < ntile) { load(loaded); ++loaded; }
     }
     if (!bad && ntile > 0) {
         const bool ok = bar_wait(done0 + 8 * ((ntile - 1) & 1), (uint32_t)(((ntile - 1) >> 1) & 1));
-        if (__syncthreads_or(!ok)) {
-            bad = true;
-        } else {
+        if (ok) {
             tc_after();
             drain((ntile - 1) & 1);
-            drained = ntile;
         }
+        if (__syncthreads_or(!ok)) bad = true;
+        else drained = ntile;
     }
     if (bad && tid == 0) {   // let this CTA's own copies and MMAs finish before leaving
         if (issued > drained) bar_wait(done0 + 8 * ((issued - 1) & 1), (uint32_t)(((issued - 1) >> 1) & 1));
@@ -385,13 +404,14 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
     tc_before();
     __syncthreads();
 
-    // fixed-order reduction: S from the hi and lo quarters, z over the 128 threads of each head
+    pdl_trigger();
+    // fixed-order reduction: S from the hi and lo quarters, z over the 64 threads of each (head, half)
     float *red = reinterpret_cast<float *>(sm);          // [4 quarters][32 e][32 c]
-    float *zred = red + 4 * 32 * 32;                      // [256 threads][33]
+    float *zred = red + 4 * 32 * 32;                      // [256 threads][17]
 #pragma unroll
     for (int j = 0; j < 16; ++j) red[(q4 * 32 + lane) * 32 + ch * 16 + j] = sacc[j];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) zred[tid * 33 + j] = zacc[j];
+    for (int j = 0; j < 16; ++j) zred[tid * 17 + j] = zacc[j];
     __syncthreads();
     const float nanv = __int_as_float(0x7fc00000);
     for (int x = tid; x < LCLA_HG * LCLA_SZ; x += 256) {
@@ -401,9 +421,10 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
             const int c = e >> 5, ee = e & 31;
             val = red[((2 * hh) * 32 + ee) * 32 + c] + red[((2 * hh + 1) * 32 + ee) * 32 + c];
         } else {
-            const int ez = e - LCLA_D * LCLA_D;
+            const int ez = e - LCLA_D * LCLA_D, ff = ez >> 4, j = ez & 15;
+            const float *zr = zred + (ff * 128 + hh * 64) * 17 + j;
             val = 0.f;
-            for (int rr = 0; rr < 128; ++rr) val += zred[(hh * 128 + rr) * 33 + ez];
+            for (int rr = 0; rr < 64; ++rr) val += zr[rr * 17];
         }
         const int head = LCLA_HG * hp + hh;
         if (head < p.H) part[(((size_t)s * p.B + b) * p.H + head) * LCLA_SZ + e] = bad ? nanv : val;
@@ -422,17 +443,18 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
 // ---------------------------------------------------------------------------
 struct LayC {
     static constexpr int STAGES = 4;
-    static constexpr int Q_OFF = 0, C_OFF = 16384, S_OFF = 24576, STAGE = 32768;   // q tile doubles as out tile
-    static constexpr int A_OFF = STAGES * STAGE, A_BYTES = 32768;                  // per buffer: 2 heads x [128][128 B]
-    static constexpr int B_OFF = A_OFF + 2 * A_BYTES;                              // per head: [P hi|P hi] + [P lo|0]
-    static constexpr int Z_OFF = B_OFF + 2 * 8192;
-    static constexpr int CTRL = Z_OFF + 256;
+    static constexpr int Q_OFF = 0, C_OFF = 8192, S_OFF = 12288, STAGE = 16384;
+    static constexpr int A_OFF = STAGES * STAGE;          // [128 rows (head, token)][q~hi | q~lo]
+    static constexpr int O_OFF = A_OFF + 16384;           // out tiles, 2 x [64 tok][128 B]
+    static constexpr int B_OFF = O_OFF + 2 * 8192;        // [64 rows (head, c)][P hi | P lo]
+    static constexpr int D_OFF = B_OFF + 8192;            // denominator halves [2 parity][2 h][2 f][64 r]
+    static constexpr int CTRL = D_OFF + 2048;
     static constexpr int BYTES = CTRL + 128 + 1024;
     static constexpr uint32_t TX = STAGE;
-    static constexpr uint32_t IDESC = idesc_bf16(128, 32, 0, 0);
+    static constexpr uint32_t IDESC = idesc_bf16(128, 64, 0, 0);
 };
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, 2)
 pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mc,
           const __grid_constant__ CUtensorMap ms, const __grid_constant__ CUtensorMap mo,
           const LclaPlan p, const float *__restrict__ pref, const float eps,
@@ -446,9 +468,9 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
     const uint32_t sb = raw + pad;
     const uint32_t full0 = sb + L::CTRL, done0 = full0 + 8 * L::STAGES;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 64);
-    float *zs = reinterpret_cast<float *>(sm + L::Z_OFF);
+    float *dens = reinterpret_cast<float *>(sm + L::D_OFF);
 
-    const int s = blockIdx.x, hp = blockIdx.y, b = blockIdx.z;
+    const int s = blockIdx.x / p.ngroups, hp = blockIdx.x % p.ngroups, b = blockIdx.y;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const LclaSeg g = lcla_segment(p, s);
     const int ntile = g.t1 > g.t0 ? (g.t1 - g.t0 + T - 1) / T : 0;
@@ -463,43 +485,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         tmem_alloc(s32(tslot), 128);
         tmem_relinquish();
     }
-    // prefix state of this block -> B operand [P hi | P hi], [P lo | 0] (K-major), and z
-    for (int x = tid; x < LCLA_HG * LCLA_D * 8; x += 256) {
-        const int hh = x >> 8, c = (x >> 3) & 31, j = x & 7;
-        const int head = LCLA_HG * hp + hh;
-        const float *P = pref + (((size_t)g.blk * p.B + b) * p.H + (head < p.H ? head : 0)) * LCLA_SZ + c * LCLA_D +
-                         8 * (j & 3);
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float y0 = head < p.H ? P[2 * m] : 0.f, y1 = head < p.H ? P[2 * m + 1] : 0.f;
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
-            const float2 hf = __bfloat1622float2(h2);
-            hi[m] = bf2_bits(h2);
-            lo[m] = bf2_bits(__floats2bfloat162_rn(y0 - hf.x, y1 - hf.y));
-        }
-        unsigned char *b1 = sm + L::B_OFF + hh * 8192, *b2 = b1 + 4096;
-        const int off = c * 128 + ((j ^ (c & 7)) << 4);
-        *reinterpret_cast<uint4 *>(b1 + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(b2 + off) = j < 4 ? make_uint4(lo[0], lo[1], lo[2], lo[3]) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (tid < LCLA_HG * LCLA_D) {
-        const int hh = tid >> 5, head = LCLA_HG * hp + hh;
-        zs[tid] = head < p.H ? pref[(((size_t)g.blk * p.B + b) * p.H + head) * LCLA_SZ + LCLA_D * LCLA_D + (tid & 31)] : 0.f;
-    }
-    fence_async_smem();
-    tc_before();
-    __syncthreads();
-    tc_after();
-    const uint32_t tmem = *tslot;
-
-    const int r = ((w & 3) << 5) | lane;   // token row (prologue and epilogue)
-    const int h = w >> 2;                   // head of the pair
-    const int head = LCLA_HG * hp + h;
-    float inv_pend = 0.f;
-    int loaded = 0, consumed = 0, issued = 0, drained = 0;
-    bool bad = false;
-
+    int loaded = 0;
     auto load = [&](int i) {
         const int st = i % L::STAGES;
         const uint32_t base = sb + st * L::STAGE, fb = full0 + 8 * st;
@@ -509,121 +495,150 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         tma_load2(base + L::C_OFF, &mc, fb, 0, t);
         tma_load2(base + L::S_OFF, &ms, fb, 0, t);
     };
-    // outputs of tile i: scale row r of head h and write it to the tile's stage
-    // (full tile, stored by TMA afterwards) or straight to global (partial tile)
+    if (tid == 0) {   // q and the tables are inputs: start streaming them before the prefixes exist
+        for (; loaded < L::STAGES - 1 && loaded < ntile; ++loaded) load(loaded);
+    }
+    pdl_wait();
+    const size_t pbase = ((size_t)g.blk * p.B + b) * p.H;
+    // prefix state of this block -> B operand rows (head, c) = [P hi | P lo] (K-major)
+    for (int x = tid; x < 64 * 8; x += 256) {
+        const int n = x >> 3, j = x & 7, hh = n >> 5, c = n & 31;
+        const int head = LCLA_HG * hp + hh;
+        const float *P = pref + (pbase + (head < p.H ? head : 0)) * LCLA_SZ + c * LCLA_D + 8 * (j & 3);
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float y0 = head < p.H ? P[2 * m] : 0.f, y1 = head < p.H ? P[2 * m + 1] : 0.f;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+            const float2 hf = __bfloat1622float2(h2);
+            hi[m] = bf2_bits(h2);
+            lo[m] = bf2_bits(__floats2bfloat162_rn(y0 - hf.x, y1 - hf.y));
+        }
+        *reinterpret_cast<uint4 *>(sm + L::B_OFF + n * 128 + ((j ^ (n & 7)) << 4)) =
+            j < 4 ? make_uint4(hi[0], hi[1], hi[2], hi[3]) : make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    fence_async_smem();
+    tc_before();
+    __syncthreads();
+    tc_after();
+    const uint32_t tmem = *tslot;
+
+    const int r = tid & 63, h = (tid >> 6) & 1, f = tid >> 7;   // prologue: token row, head, half
+    const int q4 = w & 3, ch = w >> 2;                            // epilogue: lane quarter, column half
+    const int er = ((q4 & 1) << 5) | lane, eh = q4 >> 1;          // epilogue: token row, head
+    const int ehead = LCLA_HG * hp + eh;
+    float zr[16];
+    {
+        const int head = LCLA_HG * hp + h;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            zr[j] = head < p.H ? pref[(pbase + head) * LCLA_SZ + LCLA_D * LCLA_D + 16 * f + j] : 0.f;
+    }
+    int consumed = 0, issued = 0, drained = 0;
+    bool bad = false;
+
+    // outputs of tile i: this thread's 16 values of (token er, head eh), scaled and
+    // written to the tile's out buffer (full tile, stored by TMA) or to global
     auto epilogue = [&](int i) {
-        const int t = g.t0 + i * T, nt = min(T, g.t1 - t);
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)((w & 3) * 32) << 16) + (i & 1) * 64 + h * 32, v);
+        const int t = g.t0 + i * T, nt = min(T, g.t1 - t), par = i & 1;
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(q4 * 32) << 16) + par * 64 + eh * 32 + ch * 16, v);
+        const float den = dens[((par * 2 + eh) * 2 + 0) * 64 + er] + dens[((par * 2 + eh) * 2 + 1) * 64 + er];
+        const float inv = 1.0f / (den + eps);
         tmem_wait_ld();
-        uint32_t o[16];
+        uint32_t o[8];
 #pragma unroll
-        for (int m = 0; m < 16; ++m)
-            o[m] = bf2_bits(__floats2bfloat162_rn(__uint_as_float(v[2 * m]) * inv_pend,
-                                                  __uint_as_float(v[2 * m + 1]) * inv_pend));
+        for (int m = 0; m < 8; ++m)
+            o[m] = bf2_bits(__floats2bfloat162_rn(__uint_as_float(v[2 * m]) * inv, __uint_as_float(v[2 * m + 1]) * inv));
         if (nt == T) {
-            unsigned char *row = sm + (i % L::STAGES) * L::STAGE + L::Q_OFF + r * 128;
-            const int sw = r & 7;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                *reinterpret_cast<uint4 *>(row + (((4 * h + j) ^ sw) << 4)) =
-                    make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-        } else if (r < nt && head < p.H) {
-            uint4 *dst = reinterpret_cast<uint4 *>(out + (((size_t)b * p.N + (size_t)(t + r)) * p.H + head) * LCLA_D);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            unsigned char *row = sm + L::O_OFF + par * 8192 + er * 128;
+            const int sw = er & 7;
+            *reinterpret_cast<uint4 *>(row + (((4 * eh + 2 * ch) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4 *>(row + (((4 * eh + 2 * ch + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        } else if (er < nt && ehead < p.H) {
+            uint4 *dst = reinterpret_cast<uint4 *>(out + (((size_t)b * p.N + (size_t)(t + er)) * p.H + ehead) * LCLA_D +
+                                                   16 * ch);
+            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
         }
     };
-
-    if (tid == 0)
-        for (; loaded < 2 && loaded < ntile; ++loaded) load(loaded);
+    auto store_tile = [&](int i) {   // thread 0: TMA store of a full tile's outputs
+        const int t = g.t0 + i * T;
+        if (g.t1 - t >= T) tma_store3(&mo, sb + L::O_OFF + (i & 1) * 8192, 64 * hp, t, b);
+        bulk_commit();
+    };
 
     for (int i = 0; i < ntile; ++i) {
-        const int st = i % L::STAGES, ab = i & 1;
+        const int st = i % L::STAGES, par = i & 1;
         unsigned char *stg = sm + st * L::STAGE;
 
         bool ok = bar_wait(full0 + 8 * st, (uint32_t)((i / L::STAGES) & 1));
+        if (i >= 1)   // the single A buffer is free once MMA(i-1) is done
+            ok = bar_wait(done0 + 8 * ((i - 1) & 1), (uint32_t)(((i - 1) >> 1) & 1)) && ok;
+        {   // phi, denominator half, rotary, hi/lo split -> A operand row (head h, token r)
+            uint32_t fw[8], hi[8], lo[8];
+            float cv[8], sv[8];
+            load_half_row(stg + L::Q_OFF, r, h, f, fw);
+            load_half_table(stg + L::C_OFF, r, f, cv);
+            load_half_table(stg + L::S_OFF, r, f, sv);
+            float den = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                fw[j] = relu2(fw[j]);
+                den = fmaf(bf_lo(fw[j]), zr[2 * j], den);
+                den = fmaf(bf_hi(fw[j]), zr[2 * j + 1], den);
+            }
+            dens[((par * 2 + h) * 2 + f) * 64 + r] = den;
+            rope_split8(fw, cv, sv, hi, lo);
+            store_half_hi_lo(sm + L::A_OFF, 64 * h + r, f, hi, lo);
+        }
+        fence_async_smem();
         if (__syncthreads_or(!ok)) { bad = true; break; }
         consumed = i + 1;
 
-        float inv_new;
-        {
-            float f[32], cv[16], sv[16];
-            load_head_row(stg + L::Q_OFF, r, h, f);
-            load_table_row(stg + L::C_OFF, r, cv);
-            load_table_row(stg + L::S_OFF, r, sv);
-            float den = 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                f[j] = relu(f[j]);
-                den = fmaf(f[j], zs[h * 32 + j], den);
-            }
-            inv_new = 1.0f / (den + eps);
-            uint32_t hi[16], lo[16];
-            rope_split(f, cv, sv, hi, lo);
-            store_hi_lo_row(sm + L::A_OFF + ab * L::A_BYTES + h * 16384, r, hi, lo);
-        }
-        fence_async_smem();
-        __syncthreads();
-
         if (tid == 0) {
             tc_after();
+            const uint32_t d = tmem + par * 64;
+            const uint32_t a0 = sb + L::A_OFF, b0 = sb + L::B_OFF;
 #pragma unroll
-            for (int hh = 0; hh < LCLA_HG; ++hh) {
-                const uint32_t d = tmem + ab * 64 + hh * 32;
-                const uint32_t a0 = sb + L::A_OFF + ab * L::A_BYTES + hh * 16384;
-                const uint32_t b1 = sb + L::B_OFF + hh * 8192, b2 = b1 + 4096;
+            for (int j = 0; j < 4; ++j)      // q~hi.P hi + q~lo.P hi
+                mma_bf16(d, desc_sw128(a0 + 32 * j, 16, 1024), desc_sw128(b0 + 32 * (j & 1), 16, 1024), L::IDESC, j > 0);
 #pragma unroll
-                for (int j = 0; j < 4; ++j)      // q~hi.P hi + q~lo.P hi
-                    mma_bf16(d, desc_sw128(a0 + 32 * j, 16, 1024), desc_sw128(b1 + 32 * j, 16, 1024), L::IDESC, j > 0);
-#pragma unroll
-                for (int j = 0; j < 2; ++j)      // + q~hi.P lo
-                    mma_bf16(d, desc_sw128(a0 + 32 * j, 16, 1024), desc_sw128(b2 + 32 * j, 16, 1024), L::IDESC, 1);
-            }
-            mma_commit(done0 + 8 * ab);
+            for (int j = 0; j < 2; ++j)      // + q~hi.P lo
+                mma_bf16(d, desc_sw128(a0 + 32 * j, 16, 1024), desc_sw128(b0 + 64 + 32 * j, 16, 1024), L::IDESC, 1);
+            mma_commit(done0 + 8 * par);
         }
         issued = i + 1;
 
-        if (i >= 1) {
-            ok = bar_wait(done0 + 8 * ((i - 1) & 1), (uint32_t)(((i - 1) >> 1) & 1));
-            if (__syncthreads_or(!ok)) { bad = true; break; }
+        if (i >= 1) {   // MMA(i-1) completion was observed above by every thread
             tc_after();
             epilogue(i - 1);
-            drained = i;
         }
-        inv_pend = inv_new;
         fence_async_smem();
         tc_before();
         __syncthreads();
+        drained = i;
         if (tid == 0) {
             if (i >= 1) {
-                const int tp = g.t0 + (i - 1) * T;
-                if (g.t1 - tp >= T) tma_store3(&mo, sb + ((i - 1) % L::STAGES) * L::STAGE + L::Q_OFF, 64 * hp, tp, b);
-                bulk_commit();
+                store_tile(i - 1);
+                bulk_wait_read1();   // the out buffer written next has been read by its store
             }
-            if (loaded < ntile) {
-                bulk_wait_read1();   // the store that last used this stage has read its source
-                load(loaded);
-                ++loaded;
-            }
+            if (loaded < ntile) { load(loaded); ++loaded; }
         }
     }
     if (!bad) {
         const bool ok = bar_wait(done0 + 8 * ((ntile - 1) & 1), (uint32_t)(((ntile - 1) >> 1) & 1));
+        if (ok) {
+            tc_after();
+            epilogue(ntile - 1);
+        }
+        fence_async_smem();
+        tc_before();
         if (__syncthreads_or(!ok)) {
             bad = true;
         } else {
-            tc_after();
-            epilogue(ntile - 1);
             drained = ntile;
-            fence_async_smem();
-            tc_before();
-            __syncthreads();
-            if (tid == 0) {
-                const int tp = g.t0 + (ntile - 1) * T;
-                if (g.t1 - tp >= T) tma_store3(&mo, sb + ((ntile - 1) % L::STAGES) * L::STAGE + L::Q_OFF, 64 * hp, tp, b);
-                bulk_commit();
-            }
+            if (tid == 0) store_tile(ntile - 1);
         }
     }
     if (tid == 0) {
