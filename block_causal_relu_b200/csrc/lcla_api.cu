@@ -395,6 +395,7 @@ const char *lcla_status_string(int status)
     case LCLA_ERR_MISALIGNED: return "array pointer not 16-byte aligned";
     case LCLA_ERR_WORKSPACE: return "workspace missing or too small";
     case LCLA_ERR_CUDA: return "CUDA launch failed";
+    case LCLA_ERR_TOO_LARGE: return "problem needs more scratch than the built-in array holds";
     default: return "unknown status";
     }
 }

@@ -64,7 +64,8 @@ typedef enum {
     LCLA_ERR_UNSUPPORTED = 2,   /* valid request this build does not serve (d != 32, N > 2^30) */
     LCLA_ERR_MISALIGNED = 3,    /* an array pointer is not 16-byte aligned */
     LCLA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the query says */
-    LCLA_ERR_CUDA = 5           /* a CUDA launch failed; see cudaGetLastError */
+    LCLA_ERR_CUDA = 5,          /* a CUDA launch failed; see cudaGetLastError */
+    LCLA_ERR_TOO_LARGE = 6      /* lcla_forward_noalloc: problem needs more scratch than built in */
 } lcla_status;
 
 typedef enum {
@@ -152,6 +153,37 @@ LCLA_API int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk,
  */
 LCLA_API int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,
                                     int *info);
+
+/*
+ * lcla_forward for callers that cannot allocate device memory.  (The paper
+ * has no counterpart: this is a packaging choice of this library.)
+ *
+ * Some callers have no way to obtain scratch memory: a plugin running inside
+ * a host application whose device memory is owned by that application's own
+ * pool, or a real-time loop that must not enter the driver's allocator
+ * (cudaMalloc and cudaFree can block and synchronise the device).  This entry
+ * point takes the same arguments as lcla_forward minus the workspace, and
+ * uses instead a fixed scratch array of LCLA_NOALLOC_SCRATCH_BYTES compiled
+ * into the library.  Every GPU that loads the library holds that array until
+ * the process exits.  It allocates nothing.
+ *
+ *   - Returns LCLA_ERR_TOO_LARGE, with nothing enqueued, when the problem
+ *     needs more scratch than the array holds, i.e. when
+ *     lcla_forward_workspace_bytes(B, H, N, d, block_len, dtype) >
+ *     LCLA_NOALLOC_SCRATCH_BYTES.  Other errors are those of lcla_forward.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.  `stream` must belong to the current device.
+ *   - All calls on a device share the one array, and it keeps the previous
+ *     call's contents (each call re-initialises what it reads).  Calls whose
+ *     GPU work overlaps -- on different streams, or from different host
+ *     threads -- race on the array and give wrong results: serialise them.
+ */
+#define LCLA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+LCLA_API int lcla_forward_noalloc(const void *q, const void *k, const void *v,
+                 const float *rope_cos, const float *rope_sin,
+                 int B, int H, int N, int d, int block_len, float eps,
+                 void *out, float *state_out, int dtype, void *stream);
 
 /* Static, human-readable name of a status code. */
 LCLA_API const char *lcla_status_string(int status);
