@@ -54,16 +54,23 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
         const long long tpb = ((long long)(L < N ? L : N) + p.T - 1) / p.T;   // tiles per full block
         long long nsb;
         if (p.tc) {
-            // LCLA_TC_RESIDENT CTAs per SM: the smallest split whose CTA count
-            // fills at least one wave and whose last wave is >= 90% full.
+            // Persistent CTAs take units round-robin.  Pick the split that
+            // minimises (1 + partial-state overhead) / balance, where balance
+            // is the busy fraction of the CTAs over the rounds of units and
+            // the overhead is a unit's partial state (written and read back,
+            // 2 heads x 4224 B each way) relative to its k, v bytes.
             const long long base = units * p.nb;
+            const long long Lb = L < N ? L : N;
             long long best = 1;
-            double best_eff = 0.0;
+            double best_cost = 1e30;
             for (nsb = 1; nsb <= tpb && nsb <= 64; ++nsb) {
-                const double waves = (double)(base * nsb) / (LCLA_SMS * LCLA_TC_RESIDENT);
-                const double eff = waves / (double)(long long)(waves + 0.999999);
-                if (eff > best_eff + 1e-9) { best_eff = eff; best = nsb; }
-                if (waves >= 0.9 && eff >= 0.9) { best = nsb; break; }
+                const long long n = base * nsb;
+                const long long ctas = n < LCLA_TC_CTAS ? n : LCLA_TC_CTAS;
+                const long long rounds = (n + ctas - 1) / ctas;
+                const double balance = (double)n / (double)(rounds * LCLA_TC_CTAS);
+                const double overhead = (4.0 * 4224.0 * nsb) / (256.0 * (double)Lb);
+                const double cost = (1.0 + overhead) / balance;
+                if (cost < best_cost - 1e-9) { best_cost = cost; best = nsb; }
             }
             nsb = best;
         } else {
@@ -165,7 +172,21 @@ bool map_tokens(CUtensorMap *m, const void *base, int B, int N, int H)
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [N, d/2] fp32 rotary table; box = 128 tokens, 64-byte swizzle.
+// [B, N, H*d] bf16 output blocks of one head x 32 tokens, 64-byte swizzle (TMA stores).
+bool map_out_blocks(CUtensorMap *m, const void *base, int B, int N, int H)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)H * LCLA_D, (cuuint64_t)N, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)H * LCLA_D * 2, (cuuint64_t)N * H * LCLA_D * 2};
+    cuuint32_t box[3] = {LCLA_D, 32, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [N, d/2] fp32 rotary table; box = one tile of tokens, 64-byte swizzle.
 bool map_table(CUtensorMap *m, const float *base, int N)
 {
     auto fn = encode_fn();
@@ -187,23 +208,25 @@ bool launch_tc(const void *q, const void *k, const void *v, const float *rc, con
 {
     CUtensorMap mq, mk, mv, mo, mc, ms;
     if (!map_tokens(&mq, q, p.B, p.N, p.H) || !map_tokens(&mk, k, p.B, p.N, p.H) ||
-        !map_tokens(&mv, v, p.B, p.N, p.H) || !map_tokens(&mo, out, p.B, p.N, p.H) ||
+        !map_tokens(&mv, v, p.B, p.N, p.H) || !map_out_blocks(&mo, out, p.B, p.N, p.H) ||
         !map_table(&mc, rc, p.N) || !map_table(&ms, rs, p.N))
         return false;
     float *part = reinterpret_cast<float *>(ws + p.part_off);
     float *pref = reinterpret_cast<float *>(ws + p.pref_off);
     int *status = reinterpret_cast<int *>(ws);
-    const dim3 grid(p.nseg * p.ngroups, p.B);
+    const long long units = (long long)p.nseg * p.ngroups * p.B;
+    const dim3 grid((unsigned)(units < LCLA_TC_CTAS ? units : LCLA_TC_CTAS));
     set_smem(lcla::tc::pass_a_tc, lcla::tc::LayA::BYTES);
     set_smem(lcla::tc::pass_c_tc, lcla::tc::LayC::BYTES);
     cudaMemsetAsync(status, 0, sizeof(int), st);
     if (ev) cudaEventRecord(ev[0], st);
-    lcla::tc::pass_a_tc<<<grid, 256, lcla::tc::LayA::BYTES, st>>>(mk, mv, mc, ms, p, part, status);
+    lcla::tc::pass_a_tc<<<grid, lcla::tc::LayA::NTHREADS, lcla::tc::LayA::BYTES, st>>>(mk, mv, mc, ms, p, part,
+                                                                                       status);
     if (ev) cudaEventRecord(ev[1], st);
     launch_pdl(lcla::scan_states, dim3(scan_blocks(p)), dim3(lcla::SCAN_THREADS), 0, st, p, part, pref,
                state_in, state_out);
     if (ev) cudaEventRecord(ev[2], st);
-    launch_pdl(lcla::tc::pass_c_tc, grid, dim3(256), lcla::tc::LayC::BYTES, st, mq, mc, ms, mo, p,
+    launch_pdl(lcla::tc::pass_c_tc, grid, dim3(lcla::tc::LayC::NTHREADS), lcla::tc::LayC::BYTES, st, mq, mc, ms, mo, p,
                (const float *)pref, eps, (__nv_bfloat16 *)out, status);
     if (ev) cudaEventRecord(ev[3], st);
     *rc_out = cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;

@@ -19,7 +19,7 @@
 #define LCLA_HG 2                              // heads per CTA (both paths)
 #define LCLA_T 64                              // tokens per tile (CUDA-core path)
 #define LCLA_TC_T 64                           // tokens per tile (tensor-core path)
-#define LCLA_TC_RESIDENT 2                     // tensor-core CTAs resident per SM
+#define LCLA_TC_CTAS LCLA_SMS                  // persistent tensor-core CTAs (one per SM)
 #define LCLA_SZ ((LCLA_D + 1) * LCLA_D)        // floats per (S, z) state
 #define LCLA_SMS 148                           // B200 streaming multiprocessors
 #define LCLA_TARGET_CTAS (LCLA_SMS * 4)        // CTAs per pass the CUDA-core plan aims for
