@@ -44,6 +44,7 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
     memset(&p, 0, sizeof p);
     p.B = B; p.H = H; p.N = N; p.L = L; p.dtype = dtype;
     p.ngroups = (H + LCLA_HG - 1) / LCLA_HG;
+    p.nquads = (H + LCLA_TC_HQ - 1) / LCLA_TC_HQ;
     if (N == 0) return p;
     p.nb = (int)(((long long)N + L - 1) / L);
     const long long units = (long long)p.ngroups * B;
@@ -54,12 +55,13 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
         const long long tpb = ((long long)(L < N ? L : N) + p.T - 1) / p.T;   // tiles per full block
         long long nsb;
         if (p.tc) {
-            // Persistent CTAs take units round-robin.  Pick the split that
-            // minimises (1 + partial-state overhead) / balance, where balance
-            // is the busy fraction of the CTAs over the rounds of units and
-            // the overhead is a unit's partial state (written and read back,
-            // 2 heads x 4224 B each way) relative to its k, v bytes.
-            const long long base = units * p.nb;
+            // Persistent CTAs take units (segment, head quad, batch entry)
+            // round-robin.  Pick the split that minimises (1 + partial-state
+            // overhead) / balance, where balance is the busy fraction of the
+            // CTAs over the rounds of units and the overhead is a segment's
+            // partial state per head (4224 B, written and read back) relative
+            // to the head's q, k, v, out bytes.
+            const long long base = (long long)p.nquads * B * p.nb;
             const long long Lb = L < N ? L : N;
             long long best = 1;
             double best_cost = 1e30;
@@ -158,31 +160,31 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// [B, N, H*d] bf16 viewed as a 3-D tensor; box = 2 heads x 128 tokens, 128-byte swizzle.
+// [B, N, H*d] bf16 viewed as a 3-D tensor; box = 2 heads x 64 tokens, 128-byte swizzle.
 bool map_tokens(CUtensorMap *m, const void *base, int B, int N, int H)
 {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)H * LCLA_D, (cuuint64_t)N, (cuuint64_t)B};
     cuuint64_t strides[2] = {(cuuint64_t)H * LCLA_D * 2, (cuuint64_t)N * H * LCLA_D * 2};
-    cuuint32_t box[3] = {LCLA_HG * LCLA_D, LCLA_TC_T, 1};
+    cuuint32_t box[3] = {2 * LCLA_D, LCLA_TC_T, 1};   // 128 B of a token row: 2 heads
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [B, N, H*d] bf16 output blocks of one head x 32 tokens, 64-byte swizzle (TMA stores).
+// [B, N, H*d] bf16 output blocks of one head x 64 tokens, no swizzle (TMA stores).
 bool map_out_blocks(CUtensorMap *m, const void *base, int B, int N, int H)
 {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)H * LCLA_D, (cuuint64_t)N, (cuuint64_t)B};
     cuuint64_t strides[2] = {(cuuint64_t)H * LCLA_D * 2, (cuuint64_t)N * H * LCLA_D * 2};
-    cuuint32_t box[3] = {LCLA_D, 32, 1};
+    cuuint32_t box[3] = {LCLA_D, LCLA_TC_T, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -214,7 +216,7 @@ bool launch_tc(const void *q, const void *k, const void *v, const float *rc, con
     float *part = reinterpret_cast<float *>(ws + p.part_off);
     float *pref = reinterpret_cast<float *>(ws + p.pref_off);
     int *status = reinterpret_cast<int *>(ws);
-    const long long units = (long long)p.nseg * p.ngroups * p.B;
+    const long long units = (long long)p.nseg * p.nquads * p.B;
     const dim3 grid((unsigned)(units < LCLA_TC_CTAS ? units : LCLA_TC_CTAS));
     set_smem(lcla::tc::pass_a_tc, lcla::tc::LayA::BYTES);
     set_smem(lcla::tc::pass_c_tc, lcla::tc::LayC::BYTES);

@@ -16,9 +16,10 @@
 #include <stddef.h>
 
 #define LCLA_D 32                              // head dim served
-#define LCLA_HG 2                              // heads per CTA (both paths)
+#define LCLA_HG 2                              // heads per CTA (CUDA-core path)
 #define LCLA_T 64                              // tokens per tile (CUDA-core path)
 #define LCLA_TC_T 64                           // tokens per tile (tensor-core path)
+#define LCLA_TC_HQ 4                           // heads per work unit (tensor-core path)
 #define LCLA_TC_CTAS LCLA_SMS                  // persistent tensor-core CTAs (one per SM)
 #define LCLA_SZ ((LCLA_D + 1) * LCLA_D)        // floats per (S, z) state
 #define LCLA_SMS 148                           // B200 streaming multiprocessors
@@ -34,7 +35,8 @@ struct LclaPlan {
     int tps;       // chunk mode: tiles per segment
     int nseg;      // segments
     int npref;     // prefix entries: block mode nb, chunk mode nseg
-    int ngroups;   // head groups of LCLA_HG heads
+    int ngroups;   // head groups of LCLA_HG heads (CUDA-core grid)
+    int nquads;    // head groups of LCLA_TC_HQ heads (tensor-core work units)
     size_t part_off, pref_off, ws_bytes;   // workspace layout (bytes)
 };
 

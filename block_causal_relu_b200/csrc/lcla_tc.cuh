@@ -7,39 +7,46 @@
 // ReLU features), with the d x d contractions on the 5th-generation tensor
 // cores.
 //
-// Both kernels are persistent (one CTA per SM, looping over work units =
-// (segment, head pair, batch entry), head pair fastest) and warp-specialised:
-//   producer warp   TMA loads of 64-token tiles into a deep ring of stages;
+// A tcgen05.mma of M = 128, K = 16 takes the same time for any N up to 256,
+// so both passes are built around N = 256 products: a work unit is
+// (segment, head quad, batch entry) -- four heads of 32 -- and a tile is 64
+// tokens of those four heads.  Both kernels are persistent (one CTA per SM,
+// units c, c + gridDim.x, ..., quad fastest) and warp-specialised:
+//   producer warp   TMA loads of each tile's q or k, v boxes into a ring of
+//                   stages and of its rotary rows into a smaller table ring;
 //   MMA warp        one thread issues tcgen05.mma and tcgen05.commit;
-//   prologue warps  ReLU, rotary, bf16 hi/lo split into the MMA operand;
-//   drain/epilogue  tensor memory -> registers -> partial states / outputs.
-// Roles talk only through mbarriers, so loads run as far ahead as the ring
-// allows, independently of the compute.
+//   prologue warps  (16) ReLU, rotary, bf16 hi + lo split of q or k, written
+//                   in place over the stage's raw input as the MMA operand;
+//                   thread (token r, quarter f, head pair g) does a quarter
+//                   of one token row of two heads;
+//   drain/epilogue  (warps 0-3; warp q owns head q of the quad and tensor
+//                   memory lanes 32q..32q+31) tensor memory -> registers.
+// Roles talk only through mbarriers.  A stage holds one tile from its TMA
+// load until the tile's MMAs complete; the table slot is released as soon as
+// the prologue has read it.
 //
-// Pass A.  The rotated keys k~ of a head pair are split into bf16 hi + lo
-// (k~ = hi + lo to 2^-16 relative) and stacked as the 128 rows of the A
-// operand, [hi_h0; lo_h0; hi_h1; lo_h1] (MN-major, written by the threads);
-// V of the two heads is the B operand exactly as TMA lands it (MN-major,
-// 128-byte swizzle):  D[part*32 + e][c] = sum_tok part(k~)[tok][e] v[tok][c].
-// The unrotated key sum comes from the tensor cores as well: the prologue
-// writes phi(k) back into the K tile in place and an all-ones A operand sums
-// it over the tile's tokens.  Every tile's result is read back and added into
-// fp32 registers (no long accumulation chain inside the tensor core).
+// Pass A.  A = V^T of the quad exactly as TMA lands it (MN-major, rows
+// (head, c)), B = the rotated keys split into bf16 hi + lo (k~ = hi + lo to
+// 2^-16 relative), MN-major, one 64-column atom [hi 32 | lo 32] per head:
+//     D[(h', c)][(h, part, e)] = sum_tok v[tok][h', c] part(k~)[tok][h, e].
+// Warp q adds the diagonal block h = h' of every tile (hi + lo) into fp32
+// registers; the unrotated key sum z comes from the prologue's registers.
 //
-// Pass C.  The block's prefix state P of both heads is split once per unit
-// into bf16 hi + lo and staged as the B operand (K-major rows (head, c) =
-// [P hi | P lo]); per tile the rotated queries of both heads, split into
-// hi + lo, are the 128 rows (head, token) of the A operand (K-major) and
-//   D[(h,tok)][(h',c)] = q~hi.Phi + q~lo.Phi + q~hi.Plo   (6 MMAs of K = 16)
-// (blocks h = h' used) is scaled by 1 / (z . phi(q) + eps); each epilogue
-// warp stores its 32 x 32 output block through TMA.
+// Pass C.  A = the block's prefix state P of the quad split into hi + lo,
+// rows (h', c), K-major [P hi | P lo]; B = the rotated queries split into
+// hi + lo, rows (head, token), K-major [q~hi | q~lo]:
+//     D[(h', c)][(h, tok)] = Phi.q~hi + Plo.q~hi + Phi.q~lo   (6 MMAs of K = 16).
+// Warp q scales the diagonal block by 1 / (z . phi(q) + eps), computed by the
+// prologue, writes it as bf16 [64 tok][32 c] into shared memory and stores it
+// with one TMA store (ragged tiles: plain stores of the valid rows).
 //
-// Every mbarrier wait is bounded (LCLA_TC_WAIT_NS of globaltimer) and also
-// gives up when another role has set the CTA's abort flag; the multi-warp
-// roles vote after each wait (named-barrier OR), so an abort is uniform within
-// a role and no barrier can deadlock.  An aborting CTA waits (bounded) for
-// its own copies and MMAs in flight, frees its tensor memory, writes NaN
-// partial states (pass A), sets the caller-visible status word and returns.
+// Every mbarrier wait is bounded (LCLA_TC_WAIT_NS of globaltimer) and gives
+// up when another role has set the CTA's abort flag; each warp makes the
+// outcome of a wait uniform across its lanes before acting on it, and no two
+// warps share any other barrier, so an abort cannot deadlock.  An aborting
+// CTA waits (bounded) for its own copies and MMAs in flight, frees its tensor
+// memory, writes NaN partial states (pass A), sets the caller-visible status
+// word and returns.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -53,7 +60,9 @@
 namespace lcla {
 namespace tc {
 
-constexpr int T = LCLA_TC_T;
+constexpr int T = LCLA_TC_T;     // tokens per tile
+constexpr int HQ = LCLA_TC_HQ;   // heads per unit
+constexpr unsigned ALL = 0xffffffffu;
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -88,11 +97,10 @@ __device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete; gives up when
-// the CTA's abort flag is set.  Sets the flag itself on timeout.
-__device__ __noinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+// Slow path of bar_wait: keep trying until the phase completes, the CTA's
+// abort flag is set, or LCLA_TC_WAIT_NS pass (then set the flag).
+__device__ __noinline__ bool bar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag)
 {
-    if (bar_try(bar, parity)) return true;
     const uint64_t t0 = gtimer();
     for (;;) {
         if (bar_try(bar, parity)) return true;
@@ -103,6 +111,23 @@ __device__ __noinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile in
         }
     }
 }
+// Bounded wait for the phase with the given parity to complete; gives up when
+// the CTA's abort flag is set.  Sets the flag itself on timeout.
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    return bar_try(bar, parity) || bar_wait_slow(bar, parity, abort_flag);
+}
+// Bounded wait that ignores the abort flag (used to let in-flight work land).
+__device__ __forceinline__ void bar_wait_quiet(uint32_t bar, uint32_t parity)
+{
+    volatile int never = 0;
+    bar_wait(bar, parity, &never);
+}
+__device__ __forceinline__ void bar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 // Position in a ring of N barrier-guarded slots: index and the parity of the
 // phase to wait for.  Consumers of "filled" slots start at phase 0; producers
 // waiting for "freed" slots start at phase 1 (the first round is free).
@@ -118,22 +143,6 @@ __device__ __forceinline__ void ring_next(Ring &r)
         r.phase ^= 1u;
     }
 }
-__device__ __forceinline__ void bar_arrive(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// OR of x over the `nthreads` threads that use named barrier `id` (also a barrier).
-__device__ __forceinline__ bool vote_any(int id, int nthreads, bool x)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.cta.red.or.pred q, %2, %3, p;\n"
-        " selp.u32 %0, 1, 0, q;\n}\n"
-        : "=r"(r)
-        : "r"((uint32_t)x), "r"(id), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -144,6 +153,7 @@ __device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap *map, 
         ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+
 __device__ __forceinline__ void tma_load2(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y)
 {
     asm volatile(
@@ -188,22 +198,8 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// 32 lanes x 16 columns of 32 bits: thread t of the warp gets lane (quarter*32 + t).
-__device__ __forceinline__ void tmem_ld16(uint32_t ta, uint32_t (&r)[16])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(ta));
-}
-__device__ __forceinline__ void tmem_ld8(uint32_t ta, uint32_t (&r)[8])
-{
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-                 : "r"(ta));
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t ta, uint32_t (&r)[32])
+// 32 lanes x 32 columns of 32 bits: thread t of the warp gets lane (quarter*32 + t).
+__device__ __forceinline__ void tmem_ld32(uint32_t ta, uint32_t *r)
 {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -230,6 +226,7 @@ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major)
 }
 
 __device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t *>(&v); }
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) { return bf2_bits(__floats2bfloat162_rn(a, b)); }
 
 // ReLU on two packed bf16 (NaN passes through).
 __device__ __forceinline__ uint32_t relu2(uint32_t w)
@@ -239,16 +236,11 @@ __device__ __forceinline__ uint32_t relu2(uint32_t w)
     return bf2_bits(x);
 }
 
-// Elements [8f, 8f+8) of head h in row r of a [64][64] bf16 tile (128-byte
-// swizzle), as 4 packed bf16 pairs.
-__device__ __forceinline__ uint4 load_quarter_row(const unsigned char *tile, int r, int h, int f)
+// Elements [8f, 8f+8) of head h (0 or 1) in row r of a [64][64] bf16 box
+// (128-byte swizzle), as 4 packed bf16 pairs.
+__device__ __forceinline__ uint4 load_quarter_row(const unsigned char *box, int r, int h, int f)
 {
-    return *reinterpret_cast<const uint4 *>(tile + r * 128 + (((4 * h + f) ^ (r & 7)) << 4));
-}
-// Pairs [4f, 4f+4) of row r of a [64][16] fp32 table tile (64-byte swizzle).
-__device__ __forceinline__ float4 load_quarter_table(const unsigned char *tile, int r, int f)
-{
-    return *reinterpret_cast<const float4 *>(tile + r * 64 + ((f ^ ((r >> 1) & 3)) << 4));
+    return *reinterpret_cast<const uint4 *>(box + r * 128 + (((4 * h + f) ^ (r & 7)) << 4));
 }
 // Rotate 4 pairs of (packed bf16) ReLU features, split into bf16 hi + lo.
 __device__ __forceinline__ void rope_split4(const uint32_t *fw, const float4 &c4, const float4 &s4, uint32_t *hi,
@@ -263,7 +255,7 @@ __device__ __forceinline__ void rope_split4(const uint32_t *fw, const float4 &c4
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
         const float2 hf = __bfloat1622float2(h2);
         hi[p] = bf2_bits(h2);
-        lo[p] = bf2_bits(__floats2bfloat162_rn(y0 - hf.x, y1 - hf.y));
+        lo[p] = pack_bf2(y0 - hf.x, y1 - hf.y);
     }
 }
 // Quarter f of operand row r (128 B, 128-byte swizzle): hi -> chunk f, lo -> chunk 4+f.
@@ -275,12 +267,25 @@ __device__ __forceinline__ void store_quarter_hi_lo(unsigned char *tile, int r, 
     *reinterpret_cast<uint4 *>(row + (((4 + f) ^ (r & 7)) << 4)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
 }
 
+// Pairs [4f, 4f+4) of row r of a [64][16] fp32 rotary-table box (64-byte swizzle).
+__device__ __forceinline__ float4 load_quarter_table(const unsigned char *box, int r, int f)
+{
+    return *reinterpret_cast<const float4 *>(box + r * 64 + ((f ^ ((r >> 1) & 3)) << 4));
+}
+
+// Heads of a quad are handled by two groups of prologue warps, group g taking
+// heads 2g and 2g+1.  A [64 token][2 heads] input box g lands where operand
+// atom g lives, so each thread overwrites exactly the 16-byte chunks it has
+// read; the operand of head 2g+1 goes to the fresh atom 2+g.  Atom a therefore
+// holds head 2(a & 1) + (a >> 1), and head h sits in atom (h >> 1) + 2(h & 1).
+__device__ __forceinline__ int atom_of(int h) { return (h >> 1) + 2 * (h & 1); }
+
 // ---------------------------------------------------------------------------
-// Work units of a persistent CTA: unit u = (segment, head pair, batch entry),
-// head pair fastest; CTA c takes units c, c + gridDim.x, ...
+// Work units of a persistent CTA: unit u = (segment, head quad, batch entry),
+// quad fastest; CTA c takes units c, c + gridDim.x, ...
 // ---------------------------------------------------------------------------
 struct Unit {
-    int s, hp, b;       // segment, head pair, batch entry
+    int s, hq, b;       // segment, head quad, batch entry
     int t0, t1, blk;    // token range [t0, t1) and its block
     int ntile;          // 64-token tiles
 };
@@ -288,8 +293,8 @@ struct Unit {
 __device__ __forceinline__ Unit unit_at(const LclaPlan &p, long long u)
 {
     Unit x;
-    x.hp = (int)(u % p.ngroups);
-    const long long rest = u / p.ngroups;
+    x.hq = (int)(u % p.nquads);
+    const long long rest = u / p.nquads;
     x.s = (int)(rest % p.nseg);
     x.b = (int)(rest / p.nseg);
     const LclaSeg g = lcla_segment(p, x.s);
@@ -300,70 +305,118 @@ __device__ __forceinline__ Unit unit_at(const LclaPlan &p, long long u)
     return x;
 }
 
-// Bounded wait that ignores the abort flag (used to let in-flight work land).
-__device__ __forceinline__ void bar_wait_quiet(uint32_t bar, uint32_t parity)
+constexpr int NT = 3;             // rotary-table ring slots ([cos 4 KB | sin 4 KB] per tile)
+constexpr int TAB_BYTES = 8192;
+constexpr int NPRO = 16;          // prologue warps
+
+// Producer: per tile, TMA loads of the quad's input boxes into the stage ring
+// (two [64 token][2 heads] boxes per tensor map, heads past H read as zeros)
+// and of the tile's rotary rows into the table ring.  On abort, waits
+// (bounded) for the loads already issued before returning.
+template <int S, int STAGE, int NMAP>
+__device__ __forceinline__ void produce(const LclaPlan &p, long long nunits, uint32_t sb, uint32_t tab0,
+                                        uint32_t FULL, uint32_t EMPTY, uint32_t CFULL, uint32_t CEMPTY,
+                                        const CUtensorMap *const (&maps)[NMAP], const int (&offs)[NMAP],
+                                        const CUtensorMap *mc, const CUtensorMap *ms, volatile int *abort_flag)
 {
-    volatile int never = 0;
-    bar_wait(bar, parity, &never);
+    Ring er = {0, 1u}, cr = {0, 1u};
+    int issued = 0, tissued = 0;
+    bool ok = true;
+    for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+        const Unit x = unit_at(p, u);
+        const int x0 = HQ * LCLA_D * x.hq;
+        for (int i = 0; i < x.ntile; ++i) {
+            const int t = x.t0 + i * T;
+            if (!bar_wait(EMPTY + 8 * er.idx, er.phase, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const uint32_t base = sb + er.idx * STAGE, fb = FULL + 8 * er.idx;
+            bar_expect_tx(fb, (uint32_t)(NMAP * 2 * 8192));
+#pragma unroll
+            for (int m = 0; m < NMAP; ++m) {
+                tma_load3(base + offs[m], maps[m], fb, x0, t, x.b);
+                tma_load3(base + offs[m] + 8192, maps[m], fb, x0 + 2 * LCLA_D, t, x.b);
+            }
+            ring_next<S>(er);
+            ++issued;
+            if (!bar_wait(CEMPTY + 8 * cr.idx, cr.phase, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const uint32_t tb = tab0 + cr.idx * TAB_BYTES, cb = CFULL + 8 * cr.idx;
+            bar_expect_tx(cb, (uint32_t)TAB_BYTES);
+            tma_load2(tb, mc, cb, 0, t);
+            tma_load2(tb + TAB_BYTES / 2, ms, cb, 0, t);
+            ring_next<NT>(cr);
+            ++tissued;
+        }
+    }
+    if (!ok) {   // let the copies already issued land before the CTA releases its memory
+        for (int j = issued > S ? issued - S : 0; j < issued; ++j)
+            bar_wait_quiet(FULL + 8 * (j % S), (uint32_t)((j / S) & 1));
+        for (int j = tissued > NT ? tissued - NT : 0; j < tissued; ++j)
+            bar_wait_quiet(CFULL + 8 * (j % NT), (uint32_t)((j / NT) & 1));
+    }
 }
 
 // ---------------------------------------------------------------------------
 // Pass A
 // ---------------------------------------------------------------------------
 struct LayA {
-    static constexpr int STAGES = 6;                                // TMA ring
-    static constexpr int NA = 3;                                    // A-operand ring
-    static constexpr int NTM = 4;                                   // tensor-memory ring
-    static constexpr int K_OFF = 0, V_OFF = 8192, C_OFF = 16384, S_OFF = 20480, STAGE = 24576;
-    static constexpr int A_OFF = STAGES * STAGE, A_BYTES = 16384;   // [64 tok][128 B] head 0 | head 1
-    static constexpr int RED_OFF = A_OFF + NA * A_BYTES;            // [4 quarters][32 e][33] fp32
-    static constexpr int Z_OFF = RED_OFF + 4 * 32 * 33 * 4;         // key-sum parts [2 unit parity][16 warps][8]
-    static constexpr int CTRL = Z_OFF + 2 * 16 * 8 * 4;
-    static constexpr int BYTES = CTRL + 512 + 1024;
+    static constexpr int STAGES = 4;
+    // stage: [k~ operand, 4 atoms of [64 tok][hi 32 | lo 32] (raw k lands in atoms 0-1) | v, 2 boxes]
+    static constexpr int K_OFF = 0, V_OFF = 32768, STAGE = 49152;
+    static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
+    static constexpr int Z_OFF = C_OFF + NT * TAB_BYTES;            // key-sum parts [2][16 warps][4 f][2 heads][8]
+    static constexpr int CTRL = Z_OFF + 2 * NPRO * 4 * 2 * 8 * 4;
+    static constexpr int BYTES = CTRL + 256 + 1024;
+    static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
     static constexpr int NTHREADS = 704;                            // drain 0-3, producer 4, MMA 5, prologue 6-21
-    static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6, NPRO = 512;
-    static constexpr uint32_t TX = STAGE;
-    static constexpr uint32_t IDESC = idesc_bf16(128, 64, 1, 1);
-    static constexpr int TMEM_COLS = NTM * 64;
+    static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6;
+    static constexpr uint32_t IDESC = idesc_bf16(128, 256, 1, 1);
+    static constexpr int TMEM_COLS = NTM * 256;
 };
 
 __global__ void __launch_bounds__(LayA::NTHREADS, 1)
 pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
-          const __grid_constant__ CUtensorMap mc, const __grid_constant__ CUtensorMap ms,
-          const LclaPlan p, float *__restrict__ part, int *__restrict__ status)
+          const __grid_constant__ CUtensorMap mc, const __grid_constant__ CUtensorMap ms, const LclaPlan p,
+          float *__restrict__ part, int *__restrict__ status)
 {
     using L = LayA;
-    constexpr int S = L::STAGES, NA = L::NA, NTM = L::NTM;
+    constexpr int S = L::STAGES, NTM = L::NTM;
     extern __shared__ __align__(1024) unsigned char smraw[];
     const uint32_t raw = s32(smraw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     unsigned char *sm = smraw + pad;
     const uint32_t sb = raw + pad;
-    const uint32_t FULL = sb + L::CTRL, EMPTY = FULL + 8 * S, AREADY = EMPTY + 8 * S, AFREE = AREADY + 8 * NA,
-                   TFULL = AFREE + 8 * NA, TFREE = TFULL + 8 * NTM, ZREADY = TFREE + 8 * NTM, ZFREE = ZREADY + 16;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * (2 * S + 2 * NA + 2 * NTM + 4));
+    const uint32_t FULL = sb + L::CTRL, EMPTY = FULL + 8 * S, KREADY = EMPTY + 8 * S, CFULL = KREADY + 8 * S,
+                   CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
+                   ZREADY = TFREE + 8 * NTM, ZFREE = ZREADY + 16;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * (3 * S + 2 * NT + 2 * NTM + 4));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     float *zbuf = reinterpret_cast<float *>(sm + L::Z_OFF);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const long long nunits = (long long)p.nseg * p.ngroups * p.B;
+    const long long nunits = (long long)p.nseg * p.nquads * p.B;
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
             bar_init(FULL + 8 * i, 1);
             bar_init(EMPTY + 8 * i, 1);
+            bar_init(KREADY + 8 * i, NPRO);
         }
-        for (int i = 0; i < NA; ++i) {
-            bar_init(AREADY + 8 * i, L::NPRO / 32);
-            bar_init(AFREE + 8 * i, 1);
+        for (int i = 0; i < NT; ++i) {
+            bar_init(CFULL + 8 * i, 1);
+            bar_init(CEMPTY + 8 * i, NPRO);
         }
         for (int i = 0; i < NTM; ++i) {
             bar_init(TFULL + 8 * i, 1);
             bar_init(TFREE + 8 * i, 4);
         }
         for (int i = 0; i < 2; ++i) {
-            bar_init(ZREADY + 8 * i, L::NPRO / 32);
-            bar_init(ZFREE + 8 * i, 1);
+            bar_init(ZREADY + 8 * i, NPRO);
+            bar_init(ZFREE + 8 * i, 4);
         }
         *abort_flag = 0;
         bar_fence_init();
@@ -378,65 +431,42 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
     const uint32_t tmem = *tslot;
 
     if (w == L::W_PROD) {
-        // ---------------- producer: TMA loads into the ring ----------------
+        // ---------------- producer: k, v and rotary rows of each tile ----------------
         if (lane == 0) {
-            Ring er = {0, 1u};
-            int issued = 0;
-            bool ok = true;
-            for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
-                const Unit x = unit_at(p, u);
-                for (int i = 0; i < x.ntile; ++i) {
-                    if (!bar_wait(EMPTY + 8 * er.idx, er.phase, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t base = sb + er.idx * L::STAGE, fb = FULL + 8 * er.idx;
-                    const int t = x.t0 + i * T;
-                    bar_expect_tx(fb, L::TX);
-                    tma_load3(base + L::K_OFF, &mk, fb, 64 * x.hp, t, x.b);
-                    tma_load3(base + L::V_OFF, &mv, fb, 64 * x.hp, t, x.b);
-                    tma_load2(base + L::C_OFF, &mc, fb, 0, t);
-                    tma_load2(base + L::S_OFF, &ms, fb, 0, t);
-                    ring_next<S>(er);
-                    ++issued;
-                }
-            }
-            if (!ok)   // let the copies already issued land before the CTA releases its memory
-                for (int j = issued > S ? issued - S : 0; j < issued; ++j)
-                    bar_wait_quiet(FULL + 8 * (j % S), (uint32_t)((j / S) & 1));
+            const CUtensorMap *const maps[2] = {&mk, &mv};
+            const int offs[2] = {L::K_OFF, L::V_OFF};
+            produce<S, L::STAGE, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc, &ms,
+                                    abort_flag);
         }
     } else if (w == L::W_MMA) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            Ring sr = {0, 0u}, ar = {0, 0u}, tr = {0, 1u};   // stage, A-ready, TMEM-free
-            const uint64_t adesc0 = desc_sw128(sb + L::A_OFF, 8192, 1024);
+            Ring sr = {0, 0u}, tr = {0, 1u};   // stage (k~ ready), TMEM free
             const uint64_t vdesc0 = desc_sw128(sb + L::V_OFF, 8192, 1024);
+            const uint64_t kdesc0 = desc_sw128(sb + L::K_OFF, 8192, 1024);
             int issued = 0, last_tb = 0;
             uint32_t last_phase = 0;
             bool ok = true;
             for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const Unit x = unit_at(p, u);
                 for (int i = 0; i < x.ntile; ++i) {
-                    if (!bar_wait(AREADY + 8 * ar.idx, ar.phase, abort_flag) ||
+                    if (!bar_wait(KREADY + 8 * sr.idx, sr.phase, abort_flag) ||
                         !bar_wait(TFREE + 8 * tr.idx, tr.phase, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_after();
-                    const uint32_t d = tmem + tr.idx * 64;
-                    // descriptor start addresses advance in 16-byte units
-                    const uint64_t ad = adesc0 + (uint64_t)((ar.idx * L::A_BYTES) >> 4);
-                    const uint64_t vd = vdesc0 + (uint64_t)((sr.idx * L::STAGE) >> 4);
+                    const uint32_t d = tmem + tr.idx * 256;
+                    // descriptor start addresses advance in 16-byte units; 16 tokens = 2048 B
+                    const uint64_t so = (uint64_t)((sr.idx * L::STAGE) >> 4);
 #pragma unroll
-                    for (int j = 0; j < T / 16; ++j)   // [hi; lo] k~ (x) v
-                        mma_bf16(d, ad + (uint64_t)(128 * j), vd + (uint64_t)(128 * j), L::IDESC, j > 0);
+                    for (int j = 0; j < T / 16; ++j)   // v^T (x) [k~hi | k~lo]
+                        mma_bf16(d, vdesc0 + so + 128 * j, kdesc0 + so + 128 * j, L::IDESC, j > 0);
                     mma_commit(TFULL + 8 * tr.idx);
-                    mma_commit(AFREE + 8 * ar.idx);
                     mma_commit(EMPTY + 8 * sr.idx);
                     last_tb = tr.idx;
                     last_phase = tr.phase ^ 1u;   // TFULL runs one phase behind TFREE's producer-side parity
                     ring_next<S>(sr);
-                    ring_next<NA>(ar);
                     ring_next<NTM>(tr);
                     ++issued;
                 }
@@ -445,124 +475,143 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
         }
     } else if (w >= L::W_PRO0) {
         // ---------------- prologue: phi, key sum, rotary, hi/lo split ----------------
-        const int pt = tid - 32 * L::W_PRO0, pw = pt >> 5;
-        const int r = pt & 63, h = (pt >> 6) & 1, f = pt >> 7;   // token row, head, quarter of the row
-        Ring fr = {0, 0u}, ar = {0, 1u}, zr2 = {0, 1u};   // stage-full, A-free, key-sum buffer free
+        const int pw = w - L::W_PRO0, g = pw >> 3;                   // heads 2g, 2g+1 of the quad
+        const int r = 8 * (pw & 7) + (lane >> 2), f = lane & 3;      // token row, quarter of the row
+        Ring fr = {0, 0u}, cr = {0, 0u}, zr = {0, 1u};   // stage full, table full, key-sum buffer free
         bool ok = true;
         for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
-            float zacc[8];
+            float zacc[2][8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) zacc[j] = 0.f;
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) zacc[hh][j] = 0.f;
             for (int i = 0; i < x.ntile; ++i) {
-                const int st = fr.idx, ab = ar.idx;
+                const int st = fr.idx, ct = cr.idx;
                 bool fine = bar_wait(FULL + 8 * fr.idx, fr.phase, abort_flag);
-                fine = bar_wait(AFREE + 8 * ar.idx, ar.phase, abort_flag) && fine;
-                if (vote_any(1, L::NPRO, !fine)) {
+                fine = bar_wait(CFULL + 8 * cr.idx, cr.phase, abort_flag) && fine;
+                if (!__all_sync(ALL, fine)) {
                     ok = false;
                     break;
                 }
                 ring_next<S>(fr);
-                ring_next<NA>(ar);
+                ring_next<NT>(cr);
                 unsigned char *stg = sm + st * L::STAGE;
+                const unsigned char *tab = sm + L::C_OFF + ct * TAB_BYTES;
+                const float4 c4 = load_quarter_table(tab, r, f);
+                const float4 s4 = load_quarter_table(tab + TAB_BYTES / 2, r, f);
+                const uint4 k0 = load_quarter_row(stg + L::K_OFF + g * 8192, r, 0, f);   // head 2g
+                const uint4 k1 = load_quarter_row(stg + L::K_OFF + g * 8192, r, 1, f);   // head 2g+1
+                __syncwarp();
+                if (lane == 0) bar_arrive(CEMPTY + 8 * ct);   // table rows consumed
                 const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
                 const bool valid = r < nt;
-                const uint4 kq = load_quarter_row(stg + L::K_OFF, r, h, f);
-                const float4 c4 = load_quarter_table(stg + L::C_OFF, r, f);
-                const float4 s4 = load_quarter_table(stg + L::S_OFF, r, f);
-                uint32_t fw[4] = {kq.x, kq.y, kq.z, kq.w}, hi[4], lo[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    fw[j] = valid ? relu2(fw[j]) : 0u;
-                    zacc[2 * j] += bf_lo(fw[j]);
-                    zacc[2 * j + 1] += bf_hi(fw[j]);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint4 kq = hh ? k1 : k0;
+                    uint32_t fw[4] = {kq.x, kq.y, kq.z, kq.w}, hi[4], lo[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        fw[j] = valid ? relu2(fw[j]) : 0u;
+                        zacc[hh][2 * j] += bf_lo(fw[j]);
+                        zacc[hh][2 * j + 1] += bf_hi(fw[j]);
+                    }
+                    rope_split4(fw, c4, s4, hi, lo);
+                    store_quarter_hi_lo(stg + L::K_OFF + atom_of(2 * g + hh) * 8192, r, f, hi, lo);
+                    if (!valid)   // rows past the segment belong to another unit: zero this quarter of v
+                        *reinterpret_cast<uint4 *>(stg + L::V_OFF + g * 8192 + r * 128 +
+                                                   (((4 * hh + f) ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
                 }
-                rope_split4(fw, c4, s4, hi, lo);
-                store_quarter_hi_lo(sm + L::A_OFF + ab * L::A_BYTES + h * 8192, r, f, hi, lo);
-                if (!valid)   // rows past the segment belong to another unit: zero this quarter of V
-                    *reinterpret_cast<uint4 *>(stg + L::V_OFF + r * 128 + (((4 * h + f) ^ (r & 7)) << 4)) =
-                        make_uint4(0u, 0u, 0u, 0u);
                 fence_async_smem();
                 __syncwarp();
-                if (lane == 0) bar_arrive(AREADY + 8 * ab);
+                if (lane == 0) bar_arrive(KREADY + 8 * st);
             }
             if (!ok) break;
-            // unit done: key-sum parts of this warp (32 rows of one (head, quarter)) for the drain
+            // unit done: this warp's key-sum parts (8 tokens per quarter) for the drain
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-                for (int m = 16; m >= 1; m >>= 1) zacc[j] += __shfl_xor_sync(0xffffffffu, zacc[j], m);
-            }
-            const int zb = zr2.idx;
-            if (!bar_wait(ZFREE + 8 * zr2.idx, zr2.phase, abort_flag)) {
+                for (int j = 0; j < 8; ++j)
+#pragma unroll
+                    for (int m = 4; m <= 16; m <<= 1) zacc[hh][j] += __shfl_xor_sync(ALL, zacc[hh][j], m);
+            const int zb = zr.idx;
+            if (!__all_sync(ALL, bar_wait(ZFREE + 8 * zr.idx, zr.phase, abort_flag))) {
                 ok = false;
                 break;
             }
-            ring_next<2>(zr2);
-            if (lane == 0) {
+            ring_next<2>(zr);
+            if (lane < 4) {   // lane = quarter f
+                float4 *dst = reinterpret_cast<float4 *>(zbuf + ((zb * NPRO + pw) * 4 + f) * 16);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) zbuf[(zb * 16 + pw) * 8 + j] = zacc[j];
-                bar_arrive(ZREADY + 8 * zb);
+                for (int hh = 0; hh < 2; ++hh) {
+                    dst[2 * hh] = make_float4(zacc[hh][0], zacc[hh][1], zacc[hh][2], zacc[hh][3]);
+                    dst[2 * hh + 1] = make_float4(zacc[hh][4], zacc[hh][5], zacc[hh][6], zacc[hh][7]);
+                }
             }
+            __syncwarp();
+            if (lane == 0) bar_arrive(ZREADY + 8 * zb);
         }
     } else {
         // ---------------- drain: tensor memory -> registers -> partial states ----------------
-        const int q4 = w;   // lane quarter: hi_h0, lo_h0, hi_h1, lo_h1
-        float *red = reinterpret_cast<float *>(sm + L::RED_OFF);
+        const int q = w;   // head of the quad; tensor-memory lanes 32q + c
         const float nanv = __int_as_float(0x7fc00000);
-        Ring tr = {0, 0u}, zr2 = {0, 0u};   // TMEM-full, key-sum ready
+        Ring tr = {0, 0u}, zr = {0, 0u};   // TMEM full, key sum ready
         bool ok = true;
         for (long long u = blockIdx.x; u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
-            float sacc[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) sacc[j] = 0.f;
-            for (int i = 0; ok && i < x.ntile; ++i) {
-                const int tb = tr.idx;
-                const bool fine = bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag);
-                ring_next<NTM>(tr);
-                if (vote_any(2, 128, !fine)) {
-                    ok = false;
-                    break;
-                }
-                tc_after();
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + tb * 64 + (q4 >> 1) * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) sacc[j] += __uint_as_float(v[j]);
-                tc_before();
-                __syncwarp();
-                if (lane == 0) bar_arrive(TFREE + 8 * tb);
-            }
-            // unit done: S = hi quarter + lo quarter (fixed order); z from the prologue's parts
-            const size_t pbase = ((size_t)x.s * p.B + x.b) * p.H;
-            const int zb = zr2.idx;
-            bool zok = ok && bar_wait(ZREADY + 8 * zr2.idx, zr2.phase, abort_flag);
-            ring_next<2>(zr2);
+            const int head = HQ * x.hq + q;
+            float *dst = part + (((size_t)x.s * p.B + x.b) * p.H + (head < p.H ? head : 0)) * LCLA_SZ;
             if (ok) {
+                float sacc[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) red[(q4 * 32 + lane) * 33 + j] = sacc[j];
-            }
-            if (vote_any(2, 128, !zok)) ok = false;
-            for (int xx = tid; xx < LCLA_HG * LCLA_SZ; xx += 128) {
-                const int hh = xx / LCLA_SZ, e = xx - hh * LCLA_SZ;
-                const int head = LCLA_HG * x.hp + hh;
-                float val = nanv;
+                for (int j = 0; j < 32; ++j) sacc[j] = 0.f;
+                for (int i = 0; i < x.ntile; ++i) {
+                    const int tb = tr.idx;
+                    if (!__all_sync(ALL, bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    ring_next<NTM>(tr);
+                    tc_after();
+                    const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q);
+#pragma unroll
+                    for (int part_ = 0; part_ < 2; ++part_) {   // hi columns, then lo columns
+                        uint32_t v[32];
+                        tmem_ld32(ta + 32 * part_, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) sacc[j] += __uint_as_float(v[j]);
+                    }
+                    tc_before();
+                    __syncwarp();
+                    if (lane == 0) bar_arrive(TFREE + 8 * tb);
+                }
                 if (ok) {
-                    if (e < LCLA_D * LCLA_D) {
-                        const int c = e >> 5, ee = e & 31;
-                        val = red[((2 * hh) * 32 + ee) * 33 + c] + red[((2 * hh + 1) * 32 + ee) * 33 + c];
-                    } else {   // z[hh][8f + j]: warps 2*(2f + hh) and +1 of the prologue
-                        const int ez = e - LCLA_D * LCLA_D, ff = ez >> 3, j = ez & 7;
-                        const int w0 = 2 * (2 * ff + hh);
-                        val = zbuf[(zb * 16 + w0) * 8 + j] + zbuf[(zb * 16 + w0 + 1) * 8 + j];
+                    const int zb = zr.idx;
+                    if (!__all_sync(ALL, bar_wait(ZREADY + 8 * zr.idx, zr.phase, abort_flag))) {
+                        ok = false;
+                    } else {
+                        ring_next<2>(zr);
+                        // z[e], e = lane: quarter e >> 3, element e & 7, summed over group (q >> 1)'s warps
+                        const float *zp = zbuf + ((zb * NPRO + 8 * (q >> 1)) * 4 + (lane >> 3)) * 16 + (q & 1) * 8 +
+                                          (lane & 7);
+                        float zs = 0.f;
+#pragma unroll
+                        for (int pw = 0; pw < 8; ++pw) zs += zp[pw * 4 * 16];
+                        __syncwarp();
+                        if (lane == 0) bar_arrive(ZFREE + 8 * zb);
+                        if (head < p.H) {   // row c = lane of S, then z
+                            float4 *row = reinterpret_cast<float4 *>(dst + lane * LCLA_D);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                row[j] = make_float4(sacc[4 * j], sacc[4 * j + 1], sacc[4 * j + 2], sacc[4 * j + 3]);
+                            dst[LCLA_D * LCLA_D + lane] = zs;
+                        }
                     }
                 }
-                if (head < p.H) part[(pbase + head) * LCLA_SZ + e] = val;
             }
-            vote_any(2, 128, false);
-            if (tid == 0 && zok) bar_arrive(ZFREE + 8 * zb);
+            if (!ok && head < p.H)   // aborted: this and every later partial of the head reads NaN
+                for (int e = lane; e < LCLA_SZ; e += 32) dst[e] = nanv;
         }
     }
 
@@ -580,61 +629,64 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
 // Pass C
 // ---------------------------------------------------------------------------
 struct LayC {
-    static constexpr int STAGES = 6;                                // TMA ring
-    static constexpr int NA = 3;                                    // A-operand ring
-    static constexpr int NTM = 4;                                   // tensor-memory / denominator ring
-    static constexpr int Q_OFF = 0, C_OFF = 8192, S_OFF = 12288, STAGE = 16384;
-    static constexpr int A_OFF = STAGES * STAGE, A_BYTES = 16384;   // [128 rows (head, token)][q~hi | q~lo]
-    static constexpr int B_OFF = A_OFF + NA * A_BYTES;              // 2 (unit parity) x [64 rows (head, c)][P hi | P lo]
-    static constexpr int O_OFF = B_OFF + 2 * 8192;                  // 4 warps x 2 x [32 tok][64 B] output blocks
-    static constexpr int D_OFF = O_OFF + 4 * 2 * 2048;              // denominator parts [NTM][2 h][4 f][64 r]
-    static constexpr int CTRL = D_OFF + NTM * 2048;
-    static constexpr int BYTES = CTRL + 512 + 1024;
+    static constexpr int STAGES = 4;
+    // stage: q~ operand, 4 blocks of [64 rows (tok)][q~hi 32 | q~lo 32] (raw q lands in blocks 0-1)
+    static constexpr int STAGE = 32768;
+    static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
+    static constexpr int P_OFF = C_OFF + NT * TAB_BYTES, P_BYTES = 16384;   // 2 x [128 rows (head, c)][P hi | P lo]
+    static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 4 warps x 2 x [64 tok][32 c] bf16
+    static constexpr int D_OFF = O_OFF + 4 * 2 * 4096;              // 1/den ring [ND][4 heads][64 tok]
+    static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
+    static constexpr int ND = 4;                                    // 1/den ring
+    static constexpr int CTRL = D_OFF + ND * HQ * T * 4;
+    static constexpr int BYTES = CTRL + 256 + 1024;
     static constexpr int NTHREADS = 704;                            // epilogue 0-3, producer 4, MMA 5, prologue 6-21
-    static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6, NPRO = 512;
-    static constexpr uint32_t TX = STAGE;
-    static constexpr uint32_t IDESC = idesc_bf16(128, 64, 0, 0);
-    static constexpr int TMEM_COLS = NTM * 64;
+    static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6;
+    static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
+    static constexpr int TMEM_COLS = NTM * 256;
 };
 
 __global__ void __launch_bounds__(LayC::NTHREADS, 1)
 pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mc,
-          const __grid_constant__ CUtensorMap ms, const __grid_constant__ CUtensorMap mo,
-          const LclaPlan p, const float *__restrict__ pref, const float eps,
-          __nv_bfloat16 *__restrict__ out, int *__restrict__ status)
+          const __grid_constant__ CUtensorMap ms, const __grid_constant__ CUtensorMap mo, const LclaPlan p,
+          const float *__restrict__ pref, const float eps, __nv_bfloat16 *__restrict__ out, int *__restrict__ status)
 {
     using L = LayC;
-    constexpr int S = L::STAGES, NA = L::NA, NTM = L::NTM;
+    constexpr int S = L::STAGES, NTM = L::NTM, ND = L::ND;
     extern __shared__ __align__(1024) unsigned char smraw[];
     const uint32_t raw = s32(smraw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     unsigned char *sm = smraw + pad;
     const uint32_t sb = raw + pad;
-    const uint32_t FULL = sb + L::CTRL, EMPTY = FULL + 8 * S, AREADY = EMPTY + 8 * S, AFREE = AREADY + 8 * NA,
-                   TFULL = AFREE + 8 * NA, TFREE = TFULL + 8 * NTM, DREADY = TFREE + 8 * NTM,
-                   BFREE = DREADY + 8 * NTM;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * (2 * S + 2 * NA + 3 * NTM + 2));
+    const uint32_t FULL = sb + L::CTRL, EMPTY = FULL + 8 * S, KREADY = EMPTY + 8 * S, CFULL = KREADY + 8 * S,
+                   CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
+                   DREADY = TFREE + 8 * NTM, DFREE = DREADY + 8 * ND, PFREE = DFREE + 8 * ND;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * (3 * S + 2 * NT + 2 * NTM + 2 * ND + 2));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     float *dens = reinterpret_cast<float *>(sm + L::D_OFF);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const long long nunits = (long long)p.nseg * p.ngroups * p.B;
+    const long long nunits = (long long)p.nseg * p.nquads * p.B;
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
             bar_init(FULL + 8 * i, 1);
-            bar_init(EMPTY + 8 * i, L::NPRO / 32);
+            bar_init(EMPTY + 8 * i, 1);
+            bar_init(KREADY + 8 * i, NPRO);
         }
-        for (int i = 0; i < NA; ++i) {
-            bar_init(AREADY + 8 * i, L::NPRO / 32);
-            bar_init(AFREE + 8 * i, 1);
+        for (int i = 0; i < NT; ++i) {
+            bar_init(CFULL + 8 * i, 1);
+            bar_init(CEMPTY + 8 * i, NPRO);
         }
         for (int i = 0; i < NTM; ++i) {
             bar_init(TFULL + 8 * i, 1);
             bar_init(TFREE + 8 * i, 4);
-            bar_init(DREADY + 8 * i, L::NPRO / 32);
         }
-        for (int i = 0; i < 2; ++i) bar_init(BFREE + 8 * i, 1);
+        for (int i = 0; i < ND; ++i) {
+            bar_init(DREADY + 8 * i, NPRO);
+            bar_init(DFREE + 8 * i, 4);
+        }
+        for (int i = 0; i < 2; ++i) bar_init(PFREE + 8 * i, 1);
         *abort_flag = 0;
         bar_fence_init();
     }
@@ -650,63 +702,46 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
     if (w == L::W_PROD) {
         // ---------------- producer (q and the tables are inputs: no wait on earlier kernels) ----------------
         if (lane == 0) {
-            Ring er = {0, 1u};
-            int issued = 0;
-            bool ok = true;
-            for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
-                const Unit x = unit_at(p, u);
-                for (int i = 0; i < x.ntile; ++i) {
-                    if (!bar_wait(EMPTY + 8 * er.idx, er.phase, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t base = sb + er.idx * L::STAGE, fb = FULL + 8 * er.idx;
-                    const int t = x.t0 + i * T;
-                    bar_expect_tx(fb, L::TX);
-                    tma_load3(base + L::Q_OFF, &mq, fb, 64 * x.hp, t, x.b);
-                    tma_load2(base + L::C_OFF, &mc, fb, 0, t);
-                    tma_load2(base + L::S_OFF, &ms, fb, 0, t);
-                    ring_next<S>(er);
-                    ++issued;
-                }
-            }
-            if (!ok)
-                for (int j = issued > S ? issued - S : 0; j < issued; ++j)
-                    bar_wait_quiet(FULL + 8 * (j % S), (uint32_t)((j / S) & 1));
+            const CUtensorMap *const maps[1] = {&mq};
+            const int offs[1] = {0};
+            produce<S, L::STAGE, 1>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc, &ms,
+                                    abort_flag);
         }
     } else if (w == L::W_MMA) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            Ring ar = {0, 0u}, tr = {0, 0u};   // A-ready; TMEM slot (freed through the prologue's wait)
-            const uint64_t adesc0 = desc_sw128(sb + L::A_OFF, 16, 1024);
-            const uint64_t bdesc0 = desc_sw128(sb + L::B_OFF, 16, 1024);
+            Ring sr = {0, 0u}, tr = {0, 1u};   // stage (q~ ready), TMEM free
+            const uint64_t pdesc0 = desc_sw128(sb + L::P_OFF, 16, 1024);
+            const uint64_t qdesc0 = desc_sw128(sb, 16, 1024);
             int ub = 0, issued = 0, last_tb = 0;
             uint32_t last_phase = 0;
             bool ok = true;
             for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const Unit x = unit_at(p, u);
                 if (x.ntile == 0) continue;
-                const uint64_t bd = bdesc0 + (uint64_t)((ub * 8192) >> 4);
+                const uint64_t pd = pdesc0 + (uint64_t)((ub * L::P_BYTES) >> 4);
                 for (int i = 0; i < x.ntile; ++i) {
-                    if (!bar_wait(AREADY + 8 * ar.idx, ar.phase, abort_flag)) {
+                    if (!bar_wait(KREADY + 8 * sr.idx, sr.phase, abort_flag) ||
+                        !bar_wait(TFREE + 8 * tr.idx, tr.phase, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_after();
-                    const uint32_t d = tmem + tr.idx * 64;
-                    const uint64_t ad = adesc0 + (uint64_t)((ar.idx * L::A_BYTES) >> 4);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)   // q~hi.P hi + q~lo.P hi  (32 B = 2 descriptor units per K step)
-                        mma_bf16(d, ad + (uint64_t)(2 * j), bd + (uint64_t)(2 * (j & 1)), L::IDESC, j > 0);
-#pragma unroll
-                    for (int j = 0; j < 2; ++j)   // + q~hi.P lo
-                        mma_bf16(d, ad + (uint64_t)(2 * j), bd + (uint64_t)(4 + 2 * j), L::IDESC, 1);
+                    const uint32_t d = tmem + tr.idx * 256;
+                    const uint64_t bd = qdesc0 + (uint64_t)((sr.idx * L::STAGE) >> 4);
+                    // K steps of 16 elements = 32 B = 2 descriptor units; hi at +0, lo at +64 B
+                    mma_bf16(d, pd + 0, bd + 0, L::IDESC, 0);   // P hi . q~hi
+                    mma_bf16(d, pd + 2, bd + 2, L::IDESC, 1);
+                    mma_bf16(d, pd + 4, bd + 0, L::IDESC, 1);   // P lo . q~hi
+                    mma_bf16(d, pd + 6, bd + 2, L::IDESC, 1);
+                    mma_bf16(d, pd + 0, bd + 4, L::IDESC, 1);   // P hi . q~lo
+                    mma_bf16(d, pd + 2, bd + 6, L::IDESC, 1);
                     mma_commit(TFULL + 8 * tr.idx);
-                    mma_commit(AFREE + 8 * ar.idx);
-                    if (i == x.ntile - 1) mma_commit(BFREE + 8 * ub);
+                    mma_commit(EMPTY + 8 * sr.idx);
+                    if (i == x.ntile - 1) mma_commit(PFREE + 8 * ub);
                     last_tb = tr.idx;
-                    last_phase = tr.phase;
-                    ring_next<NA>(ar);
+                    last_phase = tr.phase ^ 1u;   // TFULL runs one phase behind TFREE's producer-side parity
+                    ring_next<S>(sr);
                     ring_next<NTM>(tr);
                     ++issued;
                 }
@@ -715,141 +750,185 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             if (!ok && issued > 0) bar_wait_quiet(TFULL + 8 * last_tb, last_phase);
         }
     } else if (w >= L::W_PRO0) {
-        // ---------------- prologue: prefix state staging, phi, denominator, rotary, hi/lo split ----------------
-        const int pt = tid - 32 * L::W_PRO0;
-        const int r = pt & 63, h = (pt >> 6) & 1, f = pt >> 7;   // token row, head, quarter of the row
+        // ---------------- prologue: prefix staging, phi, 1/den, rotary, hi/lo split ----------------
+        const int pw = w - L::W_PRO0, pt = tid - 32 * L::W_PRO0, g = pw >> 3;   // heads 2g, 2g+1
+        const int r = 8 * (pw & 7) + (lane >> 2), f = lane & 3;                  // token row, quarter
         pdl_wait();   // the prefix states come from the previous kernel
-        Ring fr = {0, 0u}, ar = {0, 1u}, tr = {0, 1u}, br = {0, 1u};   // stage-full, A-free, TMEM-free, B-free
+        Ring fr = {0, 0u}, cr = {0, 0u}, dr = {0, 1u}, br = {0, 1u};   // stage full, table full, 1/den free, P free
         bool ok = true;
         for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
             if (x.ntile == 0) continue;
             const int ub = br.idx;
-            unsigned char *bop = sm + L::B_OFF + ub * 8192;
             const size_t pbase = ((size_t)x.blk * p.B + x.b) * p.H;
-            // this unit's prefix state -> B operand rows (head, c) = [P hi | P lo], once its buffer is free
-            bool fine = bar_wait(BFREE + 8 * br.idx, br.phase, abort_flag);
-            ring_next<2>(br);
-            if (vote_any(1, L::NPRO, !fine)) {
+            if (!__all_sync(ALL, bar_wait(PFREE + 8 * br.idx, br.phase, abort_flag))) {
                 ok = false;
                 break;
             }
-            {
-                const int n = pt >> 3, j = pt & 7, hh = n >> 5, c = n & 31;   // 512 chunks, one per thread
-                const int head = LCLA_HG * x.hp + hh;
-                const float *P = pref + (pbase + (head < p.H ? head : 0)) * LCLA_SZ + c * LCLA_D + 8 * (j & 3);
-                uint32_t hq[4], lq[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const float y0 = head < p.H ? P[2 * m] : 0.f, y1 = head < p.H ? P[2 * m + 1] : 0.f;
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
-                    const float2 hf = __bfloat1622float2(h2);
-                    hq[m] = bf2_bits(h2);
-                    lq[m] = bf2_bits(__floats2bfloat162_rn(y0 - hf.x, y1 - hf.y));
+            ring_next<2>(br);
+            {   // the quad's prefix state -> A operand rows m = (head, c): [P hi | P lo]; thread = (m, quarter of e)
+                const int m = pt >> 2, qq = pt & 3, head = HQ * x.hq + (m >> 5);
+                float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+                if (head < p.H) {
+                    const float4 *src =
+                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + (m & 31) * LCLA_D + 8 * qq);
+                    a = src[0];
+                    b = src[1];
                 }
-                *reinterpret_cast<uint4 *>(bop + n * 128 + ((j ^ (n & 7)) << 4)) =
-                    j < 4 ? make_uint4(hq[0], hq[1], hq[2], hq[3]) : make_uint4(lq[0], lq[1], lq[2], lq[3]);
-            }
-            float zr[8];
-            {
-                const int head = LCLA_HG * x.hp + h;
+                const float y[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                uint32_t hw[4], lw[4];
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    zr[j] = head < p.H ? pref[(pbase + head) * LCLA_SZ + LCLA_D * LCLA_D + 8 * f + j] : 0.f;
+                for (int j = 0; j < 4; ++j) {
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
+                    const float2 hf = __bfloat1622float2(h2);
+                    hw[j] = bf2_bits(h2);
+                    lw[j] = pack_bf2(y[2 * j] - hf.x, y[2 * j + 1] - hf.y);
+                }
+                store_quarter_hi_lo(sm + L::P_OFF + ub * L::P_BYTES, m, qq, hw, lw);
+            }
+            float zq[2][8];   // z[8f, 8f+8) of heads 2g, 2g+1
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int head = HQ * x.hq + 2 * g + hh;
+                float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+                if (head < p.H) {
+                    const float4 *src =
+                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + LCLA_D * LCLA_D + 8 * f);
+                    a = src[0];
+                    b = src[1];
+                }
+                zq[hh][0] = a.x; zq[hh][1] = a.y; zq[hh][2] = a.z; zq[hh][3] = a.w;
+                zq[hh][4] = b.x; zq[hh][5] = b.y; zq[hh][6] = b.z; zq[hh][7] = b.w;
             }
             for (int i = 0; i < x.ntile; ++i) {
-                const int st = fr.idx, ab = ar.idx, tb = tr.idx;
-                fine = bar_wait(FULL + 8 * fr.idx, fr.phase, abort_flag);
-                fine = bar_wait(AFREE + 8 * ar.idx, ar.phase, abort_flag) && fine;
-                fine = bar_wait(TFREE + 8 * tr.idx, tr.phase, abort_flag) && fine;
-                if (vote_any(1, L::NPRO, !fine)) {
+                const int st = fr.idx, ct = cr.idx, db = dr.idx;
+                bool fine = bar_wait(FULL + 8 * fr.idx, fr.phase, abort_flag);
+                fine = bar_wait(CFULL + 8 * cr.idx, cr.phase, abort_flag) && fine;
+                fine = bar_wait(DFREE + 8 * dr.idx, dr.phase, abort_flag) && fine;
+                if (!__all_sync(ALL, fine)) {
                     ok = false;
                     break;
                 }
                 ring_next<S>(fr);
-                ring_next<NA>(ar);
-                ring_next<NTM>(tr);
+                ring_next<NT>(cr);
+                ring_next<ND>(dr);
                 unsigned char *stg = sm + st * L::STAGE;
-                const uint4 qq = load_quarter_row(stg + L::Q_OFF, r, h, f);
-                const float4 c4 = load_quarter_table(stg + L::C_OFF, r, f);
-                const float4 s4 = load_quarter_table(stg + L::S_OFF, r, f);
-                uint32_t fw[4] = {qq.x, qq.y, qq.z, qq.w}, hi[4], lo[4];
-                float den = 0.f;
+                const unsigned char *tab = sm + L::C_OFF + ct * TAB_BYTES;
+                const float4 c4 = load_quarter_table(tab, r, f);
+                const float4 s4 = load_quarter_table(tab + TAB_BYTES / 2, r, f);
+                const uint4 q0 = load_quarter_row(stg + g * 8192, r, 0, f);   // head 2g
+                const uint4 q1 = load_quarter_row(stg + g * 8192, r, 1, f);   // head 2g+1
+                __syncwarp();
+                if (lane == 0) bar_arrive(CEMPTY + 8 * ct);   // table rows consumed
+                float den[2];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    fw[j] = relu2(fw[j]);
-                    den = fmaf(bf_lo(fw[j]), zr[2 * j], den);
-                    den = fmaf(bf_hi(fw[j]), zr[2 * j + 1], den);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint4 qv = hh ? q1 : q0;
+                    uint32_t fw[4] = {qv.x, qv.y, qv.z, qv.w}, hi[4], lo[4];
+                    float dd = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        fw[j] = relu2(fw[j]);
+                        dd = fmaf(bf_lo(fw[j]), zq[hh][2 * j], dd);
+                        dd = fmaf(bf_hi(fw[j]), zq[hh][2 * j + 1], dd);
+                    }
+                    den[hh] = dd;
+                    rope_split4(fw, c4, s4, hi, lo);
+                    store_quarter_hi_lo(stg + atom_of(2 * g + hh) * 8192, r, f, hi, lo);
                 }
-                dens[((tb * 2 + h) * 4 + f) * 64 + r] = den;
-                rope_split4(fw, c4, s4, hi, lo);
-                store_quarter_hi_lo(sm + L::A_OFF + ab * L::A_BYTES, 64 * h + r, f, hi, lo);
+                // z . phi(q) of each head over the token's four quarters (lanes 4(r & 7) .. +3)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    den[hh] += __shfl_xor_sync(ALL, den[hh], 1);
+                    den[hh] += __shfl_xor_sync(ALL, den[hh], 2);
+                }
+                if (f < 2) dens[(db * HQ + 2 * g + f) * T + r] = 1.0f / ((f ? den[1] : den[0]) + eps);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    bar_arrive(AREADY + 8 * ab);
-                    bar_arrive(DREADY + 8 * tb);
-                    bar_arrive(EMPTY + 8 * st);
+                    bar_arrive(KREADY + 8 * st);
+                    bar_arrive(DREADY + 8 * db);
                 }
             }
         }
     } else {
         // ---------------- epilogue: tensor memory -> scaled bf16 -> TMA store ----------------
-        const int q4 = w, er = ((q4 & 1) << 5) | lane, eh = q4 >> 1;
-        Ring tr = {0, 0u};   // TMEM-full and denominators-ready share the ring
+        const int q = w;   // head of the quad; tensor-memory lanes 32q + c, c = lane
+        const int odd = lane & 1;
+        const size_t tstride = (size_t)p.H * LCLA_D;   // elements per token
+        unsigned char *ob0 = sm + L::O_OFF + q * 2 * 4096;
         int ob = 0;
+        Ring tr = {0, 0u}, dr = {0, 0u};   // TMEM full, 1/den ready
         bool ok = true;
         for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
-            const int ehead = LCLA_HG * x.hp + eh;
+            const int head = HQ * x.hq + q;
             for (int i = 0; i < x.ntile; ++i) {
-                const int tb = tr.idx;
+                const int tb = tr.idx, db = dr.idx;
                 bool fine = bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag);
-                fine = bar_wait(DREADY + 8 * tr.idx, tr.phase, abort_flag) && fine;
-                if (vote_any(2, 128, !fine)) {
+                fine = bar_wait(DREADY + 8 * dr.idx, dr.phase, abort_flag) && fine;
+                if (!__all_sync(ALL, fine)) {
                     ok = false;
                     break;
                 }
                 ring_next<NTM>(tr);
+                ring_next<ND>(dr);
                 tc_after();
                 const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + tb * 64 + eh * 32, v);
-                const float *dp = dens + (tb * 2 + eh) * 4 * 64 + er;
-                const float inv = 1.0f / (((dp[0] + dp[64]) + dp[128]) + dp[192] + eps);
-                tmem_wait_ld();
-                uint32_t o[16];
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    o[m] = bf2_bits(__floats2bfloat162_rn(__uint_as_float(v[2 * m]) * inv,
-                                                          __uint_as_float(v[2 * m + 1]) * inv));
-                tc_before();
-                __syncwarp();
-                if (lane == 0) bar_arrive(TFREE + 8 * tb);
-                if (nt == T) {
-                    unsigned char *obuf = sm + L::O_OFF + (q4 * 2 + ob) * 2048;
-                    ob ^= 1;
+                const bool whole = nt == T;
+                uint32_t *obuf = reinterpret_cast<uint32_t *>(ob0 + ob * 4096);
+                if (whole) {
                     if (lane == 0) bulk_wait_read1();   // this buffer's previous store has read it
                     __syncwarp();
-                    const int sw = (lane >> 1) & 3;
+                }
+                const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q);
+                const float4 *iv = reinterpret_cast<const float4 *>(dens + (db * HQ + q) * T);
+                uint32_t *gout = reinterpret_cast<uint32_t *>(out + ((size_t)x.b * p.N + t) * tstride +
+                                                              (size_t)head * LCLA_D + (lane & ~1));
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4 *>(obuf + lane * 64 + ((j ^ sw) << 4)) =
-                            make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                for (int half = 0; half < 2; ++half) {   // tokens [32 half, 32 half + 32)
+                    uint32_t v[32], word[16];
+                    tmem_ld32(ta + 32 * half, v);
+                    tmem_wait_ld();
+                    // own column c for tokens (2m, 2m+1) packed; lane pairs (2i, 2i+1) trade them so that
+                    // the even lane holds row 2m's (c, c+1) and the odd lane row 2m+1's
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 s = iv[8 * half + j4];
+#pragma unroll
+                        for (int k = 0; k < 2; ++k) {
+                            const uint32_t mine = pack_bf2(__uint_as_float(v[4 * j4 + 2 * k]) * (k ? s.z : s.x),
+                                                           __uint_as_float(v[4 * j4 + 2 * k + 1]) * (k ? s.w : s.y));
+                            const uint32_t other = __shfl_xor_sync(ALL, mine, 1);
+                            word[2 * j4 + k] = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
+                        }
+                    }
+                    // word[j] is row 2(16 half + j) + odd; branch once per half, outside the arithmetic
+                    if (whole) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) obuf[(32 * half + 2 * j + odd) * 16 + (lane >> 1)] = word[j];
+                    } else if (head < p.H) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int tok = 32 * half + 2 * j + odd;
+                            if (tok < nt) gout[(size_t)tok * (tstride / 2)] = word[j];
+                        }
+                    }
+                }
+                tc_before();
+                __syncwarp();
+                if (lane == 0) {
+                    bar_arrive(TFREE + 8 * tb);
+                    bar_arrive(DFREE + 8 * db);
+                }
+                if (whole) {
                     fence_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store3(&mo, s32(obuf), 64 * x.hp + 32 * eh, t + 32 * (q4 & 1), x.b);
-                        bulk_commit();
+                        if (head < p.H) tma_store3(&mo, s32(obuf), LCLA_D * head, t, x.b);
+                        bulk_commit();   // one group per buffer use keeps the read-wait accounting exact
                     }
-                } else {
-                    if (er < nt && ehead < p.H) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(
-                            out + (((size_t)x.b * p.N + (size_t)(t + er)) * p.H + ehead) * LCLA_D);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-                    }
-                    if (lane == 0) bulk_commit();   // empty group: one group per tile keeps the ring accounting exact
+                    ob ^= 1;
                 }
             }
         }
