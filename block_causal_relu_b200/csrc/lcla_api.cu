@@ -83,6 +83,8 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
         p.nsb = (int)nsb;
         p.nseg = p.nb * p.nsb;
         p.npref = p.nb;
+        // the tensor-core kernels index work units with 32-bit integers
+        if ((long long)p.nseg * p.nquads * B > 0x7fffffffLL) p.tc = 0;
     } else {
         p.chunk = 1;
         p.T = (LCLA_T / L) * L;
@@ -134,7 +136,7 @@ void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
 
 unsigned scan_blocks(const LclaPlan &p)
 {
-    const size_t n = (size_t)p.B * p.H * LCLA_SZ;
+    const size_t n = (size_t)p.B * p.H * (LCLA_SZ / lcla::SCAN_VEC);
     return (unsigned)((n + lcla::SCAN_THREADS - 1) / lcla::SCAN_THREADS);
 }
 

@@ -630,42 +630,53 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
 }
 
 // ---------------------------------------------------------------------------
-// Scan: partials -> prefixes, one thread per state element (b, h, x) with
-// x < (D+1)*D; the segment partials are loaded in batches of independent
-// loads and summed in segment order.
+// Scan: partials -> prefixes, one thread per 4 consecutive state elements
+// (b, h, x..x+3) with x < (D+1)*D; the segment partials are loaded as float4
+// in batches of independent loads and summed in segment order.
 // Block mode: pref[blk] = state_in + sum of all segments of blocks <= blk.
 // Chunk mode: pref[s]   = state_in + sum of segments < s.
 // state_out (may equal state_in) receives the total.
 // ---------------------------------------------------------------------------
-constexpr int SCAN_THREADS = 256;
+constexpr int SCAN_THREADS = 128;
+constexpr int SCAN_VEC = 4;   // elements per thread (LCLA_SZ is a multiple of 4)
+
+__device__ __forceinline__ void add4(float4 &a, const float4 &b)
+{
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+}
 
 __global__ void __launch_bounds__(SCAN_THREADS)
 scan_states(const LclaPlan p, const float *__restrict__ part, float *__restrict__ pref,
             const float *state_in, float *state_out)
 {
     constexpr int BATCH = 16;
-    const size_t n = (size_t)p.B * p.H * LCLA_SZ;                // elements of one slice
+    const size_t n4 = (size_t)p.B * p.H * (LCLA_SZ / SCAN_VEC);   // float4 of one slice
     const size_t x = (size_t)blockIdx.x * SCAN_THREADS + threadIdx.x;
     pdl_wait();
     pdl_trigger();
-    if (x >= n) return;
-    float acc = state_in ? state_in[x] : 0.f;
+    if (x >= n4) return;
+    const float4 *part4 = reinterpret_cast<const float4 *>(part);
+    float4 *pref4 = reinterpret_cast<float4 *>(pref);
+    float4 acc = state_in ? reinterpret_cast<const float4 *>(state_in)[x] : make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = 0; s0 < p.nseg; s0 += BATCH) {
-        float v[BATCH];
+        float4 v[BATCH];
 #pragma unroll
         for (int j = 0; j < BATCH; ++j)
-            if (s0 + j < p.nseg) v[j] = __ldcg(part + (size_t)(s0 + j) * n + x);
+            if (s0 + j < p.nseg) v[j] = __ldcg(part4 + (size_t)(s0 + j) * n4 + x);
 #pragma unroll
         for (int j = 0; j < BATCH; ++j) {
             const int s = s0 + j;
             if (s < p.nseg) {
-                if (p.chunk) pref[(size_t)s * n + x] = acc;
-                acc += v[j];
-                if (!p.chunk && (s + 1) % p.nsb == 0) pref[(size_t)(s / p.nsb) * n + x] = acc;
+                if (p.chunk) pref4[(size_t)s * n4 + x] = acc;
+                add4(acc, v[j]);
+                if (!p.chunk && (s + 1) % p.nsb == 0) pref4[(size_t)(s / p.nsb) * n4 + x] = acc;
             }
         }
     }
-    if (state_out) state_out[x] = acc;
+    if (state_out) reinterpret_cast<float4 *>(state_out)[x] = acc;
 }
 
 }  // namespace lcla

@@ -51,25 +51,28 @@ struct LclaSeg {
 #define LCLA_HD inline
 #endif
 
-LCLA_HD long long lcla_min_ll(long long a, long long b) { return a < b ? a : b; }
+LCLA_HD int lcla_min_i(int a, int b) { return a < b ? a : b; }
 
-// Token range of segment s.
+// Token range of segment s.  All arithmetic fits in 32 bits: N <= 2^30 (the
+// API rejects larger N), so block starts, token counts and j * per stay below
+// 2^30 before the final multiply by the tile length, which is bounded by the
+// block length.
 LCLA_HD LclaSeg lcla_segment(const LclaPlan &p, int s)
 {
     LclaSeg g;
     if (!p.chunk) {
         g.blk = s / p.nsb;
-        const long long j = s - (long long)g.blk * p.nsb;
-        const long long b0 = (long long)g.blk * p.L;
-        const long long bl = lcla_min_ll(p.L, p.N - b0);
-        const long long nt = (bl + p.T - 1) / p.T;               // tiles in this block
-        const long long per = (nt + p.nsb - 1) / p.nsb;          // tiles per segment
-        g.t0 = (int)(b0 + lcla_min_ll(j * per * p.T, bl));
-        g.t1 = (int)(b0 + lcla_min_ll((j + 1) * per * p.T, bl));
+        const int j = s - g.blk * p.nsb;
+        const int b0 = g.blk * p.L;
+        const int bl = lcla_min_i(p.L, p.N - b0);
+        const int nt = (bl + p.T - 1) / p.T;               // tiles in this block
+        const int per = (nt + p.nsb - 1) / p.nsb;          // tiles per segment
+        g.t0 = b0 + lcla_min_i(lcla_min_i(j * per, nt) * p.T, bl);
+        g.t1 = b0 + lcla_min_i(lcla_min_i((j + 1) * per, nt) * p.T, bl);
     } else {
-        const long long span = (long long)p.tps * p.T;
-        g.t0 = (int)lcla_min_ll((long long)s * span, p.N);
-        g.t1 = (int)lcla_min_ll((long long)g.t0 + span, p.N);
+        const int span = p.tps * p.T;
+        g.t0 = s < p.nseg ? lcla_min_i(s * span, p.N) : p.N;   // (nseg - 1) * span < N + T
+        g.t1 = lcla_min_i(g.t0 + span, p.N);
         g.blk = -1;
     }
     return g;

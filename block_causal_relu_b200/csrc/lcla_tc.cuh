@@ -15,10 +15,12 @@
 //   producer warp   TMA loads of each tile's q or k, v boxes into a ring of
 //                   stages and of its rotary rows into a smaller table ring;
 //   MMA warp        one thread issues tcgen05.mma and tcgen05.commit;
-//   prologue warps  (16) ReLU, rotary, bf16 hi + lo split of q or k, written
+//   prologue warps  (8) ReLU, rotary, bf16 hi + lo split of q or k, written
 //                   in place over the stage's raw input as the MMA operand;
-//                   thread (token r, quarter f, head pair g) does a quarter
-//                   of one token row of two heads;
+//                   thread (token r, quarter f) does a quarter of one token
+//                   row of all four heads, so each rotary entry is read once
+//                   and the fixed per-tile work (waits, fences, arrivals) is
+//                   spread over 32 elements per thread;
 //   drain/epilogue  (warps 0-3; warp q owns head q of the quad and tensor
 //                   memory lanes 32q..32q+31) tensor memory -> registers.
 // Roles talk only through mbarriers.  A stage holds one tile from its TMA
@@ -127,6 +129,10 @@ __device__ __forceinline__ void bar_arrive(uint32_t bar)
 {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// release_after_use: a warp releases a shared buffer that a TMA load will
+// refill only after instructions have consumed every value it loaded from it.
+// An arrive issued right after the loads themselves was observed to let the
+// refill overtake them (pass A read the next tile's rotary rows, intermittently).
 
 // Position in a ring of N barrier-guarded slots: index and the parity of the
 // phase to wait for.  Consumers of "filled" slots start at phase 0; producers
@@ -199,18 +205,22 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
 }
 
 // 32 lanes x 32 columns of 32 bits: thread t of the warp gets lane (quarter*32 + t).
+// tcgen05.ld fills its destination registers asynchronously; only
+// tcgen05.wait::ld makes them valid.  Both sit in one asm statement, so that
+// the compiler cannot schedule any use of the outputs before the wait.
 __device__ __forceinline__ void tmem_ld32(uint32_t ta, uint32_t *r)
 {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(ta));
+        : "r"(ta)
+        : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout, version 1).
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo)
@@ -236,12 +246,6 @@ __device__ __forceinline__ uint32_t relu2(uint32_t w)
     return bf2_bits(x);
 }
 
-// Elements [8f, 8f+8) of head h (0 or 1) in row r of a [64][64] bf16 box
-// (128-byte swizzle), as 4 packed bf16 pairs.
-__device__ __forceinline__ uint4 load_quarter_row(const unsigned char *box, int r, int h, int f)
-{
-    return *reinterpret_cast<const uint4 *>(box + r * 128 + (((4 * h + f) ^ (r & 7)) << 4));
-}
 // Rotate 4 pairs of (packed bf16) ReLU features, split into bf16 hi + lo.
 __device__ __forceinline__ void rope_split4(const uint32_t *fw, const float4 &c4, const float4 &s4, uint32_t *hi,
                                             uint32_t *lo)
@@ -267,18 +271,41 @@ __device__ __forceinline__ void store_quarter_hi_lo(unsigned char *tile, int r, 
     *reinterpret_cast<uint4 *>(row + (((4 + f) ^ (r & 7)) << 4)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
 }
 
-// Pairs [4f, 4f+4) of row r of a [64][16] fp32 rotary-table box (64-byte swizzle).
-__device__ __forceinline__ float4 load_quarter_table(const unsigned char *box, int r, int f)
-{
-    return *reinterpret_cast<const float4 *>(box + r * 64 + ((f ^ ((r >> 1) & 3)) << 4));
-}
 
-// Heads of a quad are handled by two groups of prologue warps, group g taking
-// heads 2g and 2g+1.  A [64 token][2 heads] input box g lands where operand
-// atom g lives, so each thread overwrites exactly the 16-byte chunks it has
-// read; the operand of head 2g+1 goes to the fresh atom 2+g.  Atom a therefore
-// holds head 2(a & 1) + (a >> 1), and head h sits in atom (h >> 1) + 2(h & 1).
+// Operand atom a (8 KB: [64 rows][hi 32 | lo 32] of one head) holds head
+// 2(a & 1) + (a >> 1): the [64 token][heads 2b, 2b+1] input box b lands where
+// atom b lives, and the prologue thread that reads a row's quarter f of heads
+// 2b and 2b+1 writes head 2b's hi and lo there -- exactly the two 16-byte
+// chunks it has read -- and head 2b+1's into the fresh atom 2+b.
 __device__ __forceinline__ int atom_of(int h) { return (h >> 1) + 2 * (h & 1); }
+
+// Prologue thread (warp pw in 0..7, lane): token row r = 8 pw + (lane >> 2),
+// quarter f = lane & 3.  Inside a 128-byte-swizzled [64][128 B] box, chunk f
+// of row r is at `a`, chunk 4 + f at `b`; eight consecutive rows per warp keep
+// every 128-bit shared access free of bank conflicts.  `tab` is the row's
+// quarter f inside a [64][16] fp32 rotary box (64-byte swizzle).
+struct ProOffs {
+    int r, f, a, b, tab;
+};
+__device__ __forceinline__ ProOffs pro_offsets(int pw, int lane)
+{
+    ProOffs o;
+    o.f = lane & 3;
+    o.r = 8 * pw + (lane >> 2);
+    const int sw = o.r & 7;
+    o.a = o.r * 128 + ((o.f ^ sw) << 4);
+    o.b = o.r * 128 + (((4 + o.f) ^ sw) << 4);
+    o.tab = o.r * 64 + ((o.f ^ ((o.r >> 1) & 3)) << 4);
+    return o;
+}
+// Raw input quarter of head h in a stage (box h >> 1, chunk f or 4 + f).
+__device__ __forceinline__ int raw_off(const ProOffs &o, int h) { return (h >> 1) * 8192 + ((h & 1) ? o.b : o.a); }
+__device__ __forceinline__ uint4 lds128(const unsigned char *p) { return *reinterpret_cast<const uint4 *>(p); }
+__device__ __forceinline__ float4 ldsf4(const unsigned char *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ void sts128(unsigned char *p, const uint32_t *w)
+{
+    *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 // ---------------------------------------------------------------------------
 // Work units of a persistent CTA: unit u = (segment, head quad, batch entry),
@@ -290,13 +317,14 @@ struct Unit {
     int ntile;          // 64-token tiles
 };
 
-__device__ __forceinline__ Unit unit_at(const LclaPlan &p, long long u)
+// (The host keeps nseg * nquads * B below 2^31 on this path.)
+__device__ __forceinline__ Unit unit_at(const LclaPlan &p, int u)
 {
     Unit x;
-    x.hq = (int)(u % p.nquads);
-    const long long rest = u / p.nquads;
-    x.s = (int)(rest % p.nseg);
-    x.b = (int)(rest / p.nseg);
+    x.hq = u % p.nquads;
+    const int rest = u / p.nquads;
+    x.s = rest % p.nseg;
+    x.b = rest / p.nseg;
     const LclaSeg g = lcla_segment(p, x.s);
     x.t0 = g.t0;
     x.t1 = g.t1;
@@ -306,15 +334,17 @@ __device__ __forceinline__ Unit unit_at(const LclaPlan &p, long long u)
 }
 
 constexpr int NT = 3;             // rotary-table ring slots ([cos 4 KB | sin 4 KB] per tile)
+constexpr int CTRL_BYTES = 512;   // control block: mbarriers (8 B each), tensor-memory slot, abort flag
+constexpr int SMEM_MAX = 232448;  // dynamic shared memory a CTA may opt in to
 constexpr int TAB_BYTES = 8192;
-constexpr int NPRO = 16;          // prologue warps
+constexpr int NPRO = 8;           // prologue warps
 
 // Producer: per tile, TMA loads of the quad's input boxes into the stage ring
 // (two [64 token][2 heads] boxes per tensor map, heads past H read as zeros)
 // and of the tile's rotary rows into the table ring.  On abort, waits
 // (bounded) for the loads already issued before returning.
 template <int S, int STAGE, int NMAP>
-__device__ __forceinline__ void produce(const LclaPlan &p, long long nunits, uint32_t sb, uint32_t tab0,
+__device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t sb, uint32_t tab0,
                                         uint32_t FULL, uint32_t EMPTY, uint32_t CFULL, uint32_t CEMPTY,
                                         const CUtensorMap *const (&maps)[NMAP], const int (&offs)[NMAP],
                                         const CUtensorMap *mc, const CUtensorMap *ms, volatile int *abort_flag)
@@ -322,7 +352,7 @@ __device__ __forceinline__ void produce(const LclaPlan &p, long long nunits, uin
     Ring er = {0, 1u}, cr = {0, 1u};
     int issued = 0, tissued = 0;
     bool ok = true;
-    for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+    for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
         const Unit x = unit_at(p, u);
         const int x0 = HQ * LCLA_D * x.hq;
         for (int i = 0; i < x.ntile; ++i) {
@@ -368,15 +398,19 @@ struct LayA {
     // stage: [k~ operand, 4 atoms of [64 tok][hi 32 | lo 32] (raw k lands in atoms 0-1) | v, 2 boxes]
     static constexpr int K_OFF = 0, V_OFF = 32768, STAGE = 49152;
     static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
-    static constexpr int Z_OFF = C_OFF + NT * TAB_BYTES;            // key-sum parts [2][16 warps][4 f][2 heads][8]
-    static constexpr int CTRL = Z_OFF + 2 * NPRO * 4 * 2 * 8 * 4;
-    static constexpr int BYTES = CTRL + 256 + 1024;
+    static constexpr int Z_OFF = C_OFF + NT * TAB_BYTES;            // key-sum parts [8 warps][4 f][4 heads][8]
+    static constexpr int Z_BYTES = NPRO * 4 * HQ * 8 * 4;
+    static constexpr int CTRL = Z_OFF + Z_BYTES;                    // mbarriers, tensor-memory slot, abort flag
+    static constexpr int BYTES = CTRL + CTRL_BYTES + 1024;          // + worst-case 1024-byte alignment pad
     static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
-    static constexpr int NTHREADS = 704;                            // drain 0-3, producer 4, MMA 5, prologue 6-21
+    static constexpr int NTHREADS = 448;                            // drain 0-3, producer 4, MMA 5, prologue 6-13
     static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6;
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 1, 1);
     static constexpr int TMEM_COLS = NTM * 256;
+    static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 2;
 };
+static_assert(LayA::BYTES <= SMEM_MAX, "pass A shared memory");
+static_assert(8 * LayA::NBARS + 8 <= CTRL_BYTES, "pass A control block");
 
 __global__ void __launch_bounds__(LayA::NTHREADS, 1)
 pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
@@ -392,13 +426,13 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
     const uint32_t sb = raw + pad;
     const uint32_t FULL = sb + L::CTRL, EMPTY = FULL + 8 * S, KREADY = EMPTY + 8 * S, CFULL = KREADY + 8 * S,
                    CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
-                   ZREADY = TFREE + 8 * NTM, ZFREE = ZREADY + 16;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * (3 * S + 2 * NT + 2 * NTM + 4));
+                   ZREADY = TFREE + 8 * NTM, ZFREE = ZREADY + 8;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * L::NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     float *zbuf = reinterpret_cast<float *>(sm + L::Z_OFF);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const long long nunits = (long long)p.nseg * p.nquads * p.B;
+    const int nunits = p.nseg * p.nquads * p.B;
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
@@ -414,10 +448,8 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
             bar_init(TFULL + 8 * i, 1);
             bar_init(TFREE + 8 * i, 4);
         }
-        for (int i = 0; i < 2; ++i) {
-            bar_init(ZREADY + 8 * i, NPRO);
-            bar_init(ZFREE + 8 * i, 4);
-        }
+        bar_init(ZREADY, NPRO);
+        bar_init(ZFREE, 4);
         *abort_flag = 0;
         bar_fence_init();
     }
@@ -447,7 +479,7 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
             int issued = 0, last_tb = 0;
             uint32_t last_phase = 0;
             bool ok = true;
-            for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const Unit x = unit_at(p, u);
                 for (int i = 0; i < x.ntile; ++i) {
                     if (!bar_wait(KREADY + 8 * sr.idx, sr.phase, abort_flag) ||
@@ -475,17 +507,17 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
         }
     } else if (w >= L::W_PRO0) {
         // ---------------- prologue: phi, key sum, rotary, hi/lo split ----------------
-        const int pw = w - L::W_PRO0, g = pw >> 3;                   // heads 2g, 2g+1 of the quad
-        const int r = 8 * (pw & 7) + (lane >> 2), f = lane & 3;      // token row, quarter of the row
-        Ring fr = {0, 0u}, cr = {0, 0u}, zr = {0, 1u};   // stage full, table full, key-sum buffer free
+        const int pw = w - L::W_PRO0;
+        const ProOffs o = pro_offsets(pw, lane);
+        Ring fr = {0, 0u}, cr = {0, 0u}, zr = {0, 1u};   // stage full, table full, key-sum buffer free (1 slot)
         bool ok = true;
-        for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+        for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
-            float zacc[2][8];
+            float zacc[HQ][8];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
+            for (int h = 0; h < HQ; ++h)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) zacc[hh][j] = 0.f;
+                for (int j = 0; j < 8; ++j) zacc[h][j] = 0.f;
             for (int i = 0; i < x.ntile; ++i) {
                 const int st = fr.idx, ct = cr.idx;
                 bool fine = bar_wait(FULL + 8 * fr.idx, fr.phase, abort_flag);
@@ -498,66 +530,67 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                 ring_next<NT>(cr);
                 unsigned char *stg = sm + st * L::STAGE;
                 const unsigned char *tab = sm + L::C_OFF + ct * TAB_BYTES;
-                const float4 c4 = load_quarter_table(tab, r, f);
-                const float4 s4 = load_quarter_table(tab + TAB_BYTES / 2, r, f);
-                const uint4 k0 = load_quarter_row(stg + L::K_OFF + g * 8192, r, 0, f);   // head 2g
-                const uint4 k1 = load_quarter_row(stg + L::K_OFF + g * 8192, r, 1, f);   // head 2g+1
-                __syncwarp();
-                if (lane == 0) bar_arrive(CEMPTY + 8 * ct);   // table rows consumed
-                const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
-                const bool valid = r < nt;
+                const float4 c4 = ldsf4(tab + o.tab);
+                const float4 s4 = ldsf4(tab + TAB_BYTES / 2 + o.tab);
+                uint4 kr[HQ];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const uint4 kq = hh ? k1 : k0;
-                    uint32_t fw[4] = {kq.x, kq.y, kq.z, kq.w}, hi[4], lo[4];
+                for (int h = 0; h < HQ; ++h) kr[h] = lds128(stg + L::K_OFF + raw_off(o, h));
+                const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
+                const bool valid = o.r < nt;
+#pragma unroll
+                for (int h = 0; h < HQ; ++h) {
+                    uint32_t fw[4] = {kr[h].x, kr[h].y, kr[h].z, kr[h].w}, hi[4], lo[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         fw[j] = valid ? relu2(fw[j]) : 0u;
-                        zacc[hh][2 * j] += bf_lo(fw[j]);
-                        zacc[hh][2 * j + 1] += bf_hi(fw[j]);
+                        zacc[h][2 * j] += bf_lo(fw[j]);
+                        zacc[h][2 * j + 1] += bf_hi(fw[j]);
                     }
                     rope_split4(fw, c4, s4, hi, lo);
-                    store_quarter_hi_lo(stg + L::K_OFF + atom_of(2 * g + hh) * 8192, r, f, hi, lo);
+                    unsigned char *atom = stg + L::K_OFF + atom_of(h) * 8192;
+                    sts128(atom + o.a, hi);
+                    sts128(atom + o.b, lo);
                     if (!valid)   // rows past the segment belong to another unit: zero this quarter of v
-                        *reinterpret_cast<uint4 *>(stg + L::V_OFF + g * 8192 + r * 128 +
-                                                   (((4 * hh + f) ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4 *>(stg + L::V_OFF + raw_off(o, h)) = make_uint4(0u, 0u, 0u, 0u);
                 }
                 fence_async_smem();
                 __syncwarp();
-                if (lane == 0) bar_arrive(KREADY + 8 * st);
+                if (lane == 0) {
+                    bar_arrive(KREADY + 8 * st);
+                    bar_arrive(CEMPTY + 8 * ct);   // after the rows have been used: see release_after_use
+                }
             }
             if (!ok) break;
-            // unit done: this warp's key-sum parts (8 tokens per quarter) for the drain
+            // unit done: this warp's key-sum parts (its 8 token rows) for the drain
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
+            for (int h = 0; h < HQ; ++h)
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
 #pragma unroll
-                    for (int m = 4; m <= 16; m <<= 1) zacc[hh][j] += __shfl_xor_sync(ALL, zacc[hh][j], m);
-            const int zb = zr.idx;
-            if (!__all_sync(ALL, bar_wait(ZFREE + 8 * zr.idx, zr.phase, abort_flag))) {
+                    for (int m = 4; m <= 16; m <<= 1) zacc[h][j] += __shfl_xor_sync(ALL, zacc[h][j], m);
+            if (!__all_sync(ALL, bar_wait(ZFREE, zr.phase, abort_flag))) {
                 ok = false;
                 break;
             }
-            ring_next<2>(zr);
+            ring_next<1>(zr);
             if (lane < 4) {   // lane = quarter f
-                float4 *dst = reinterpret_cast<float4 *>(zbuf + ((zb * NPRO + pw) * 4 + f) * 16);
+                float4 *dst = reinterpret_cast<float4 *>(zbuf + (pw * 4 + o.f) * (HQ * 8));
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    dst[2 * hh] = make_float4(zacc[hh][0], zacc[hh][1], zacc[hh][2], zacc[hh][3]);
-                    dst[2 * hh + 1] = make_float4(zacc[hh][4], zacc[hh][5], zacc[hh][6], zacc[hh][7]);
+                for (int h = 0; h < HQ; ++h) {
+                    dst[2 * h] = make_float4(zacc[h][0], zacc[h][1], zacc[h][2], zacc[h][3]);
+                    dst[2 * h + 1] = make_float4(zacc[h][4], zacc[h][5], zacc[h][6], zacc[h][7]);
                 }
             }
             __syncwarp();
-            if (lane == 0) bar_arrive(ZREADY + 8 * zb);
+            if (lane == 0) bar_arrive(ZREADY);
         }
     } else {
         // ---------------- drain: tensor memory -> registers -> partial states ----------------
         const int q = w;   // head of the quad; tensor-memory lanes 32q + c
         const float nanv = __int_as_float(0x7fc00000);
-        Ring tr = {0, 0u}, zr = {0, 0u};   // TMEM full, key sum ready
+        Ring tr = {0, 0u}, zr = {0, 0u};   // TMEM full, key sum ready (1 slot)
         bool ok = true;
-        for (long long u = blockIdx.x; u < nunits; u += gridDim.x) {
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
             const int head = HQ * x.hq + q;
             float *dst = part + (((size_t)x.s * p.B + x.b) * p.H + (head < p.H ? head : 0)) * LCLA_SZ;
@@ -578,7 +611,6 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                     for (int part_ = 0; part_ < 2; ++part_) {   // hi columns, then lo columns
                         uint32_t v[32];
                         tmem_ld32(ta + 32 * part_, v);
-                        tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) sacc[j] += __uint_as_float(v[j]);
                     }
@@ -587,19 +619,17 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                     if (lane == 0) bar_arrive(TFREE + 8 * tb);
                 }
                 if (ok) {
-                    const int zb = zr.idx;
-                    if (!__all_sync(ALL, bar_wait(ZREADY + 8 * zr.idx, zr.phase, abort_flag))) {
+                    if (!__all_sync(ALL, bar_wait(ZREADY, zr.phase, abort_flag))) {
                         ok = false;
                     } else {
-                        ring_next<2>(zr);
-                        // z[e], e = lane: quarter e >> 3, element e & 7, summed over group (q >> 1)'s warps
-                        const float *zp = zbuf + ((zb * NPRO + 8 * (q >> 1)) * 4 + (lane >> 3)) * 16 + (q & 1) * 8 +
-                                          (lane & 7);
+                        ring_next<1>(zr);
+                        // z[e], e = lane: quarter e >> 3, element e & 7 of head q, over the prologue warps
+                        const float *zp = zbuf + (lane >> 3) * (HQ * 8) + q * 8 + (lane & 7);
                         float zs = 0.f;
 #pragma unroll
-                        for (int pw = 0; pw < 8; ++pw) zs += zp[pw * 4 * 16];
+                        for (int pw = 0; pw < NPRO; ++pw) zs += zp[pw * 4 * HQ * 8];
                         __syncwarp();
-                        if (lane == 0) bar_arrive(ZFREE + 8 * zb);
+                        if (lane == 0) bar_arrive(ZFREE);
                         if (head < p.H) {   // row c = lane of S, then z
                             float4 *row = reinterpret_cast<float4 *>(dst + lane * LCLA_D);
 #pragma unroll
@@ -638,13 +668,16 @@ struct LayC {
     static constexpr int D_OFF = O_OFF + 4 * 2 * 4096;              // 1/den ring [ND][4 heads][64 tok]
     static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
     static constexpr int ND = 4;                                    // 1/den ring
-    static constexpr int CTRL = D_OFF + ND * HQ * T * 4;
-    static constexpr int BYTES = CTRL + 256 + 1024;
-    static constexpr int NTHREADS = 704;                            // epilogue 0-3, producer 4, MMA 5, prologue 6-21
+    static constexpr int CTRL = D_OFF + ND * HQ * T * 4;            // mbarriers, tensor-memory slot, abort flag
+    static constexpr int BYTES = CTRL + CTRL_BYTES + 1024;          // + worst-case 1024-byte alignment pad
+    static constexpr int NTHREADS = 448;                            // epilogue 0-3, producer 4, MMA 5, prologue 6-13
     static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6;
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
     static constexpr int TMEM_COLS = NTM * 256;
+    static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 2 * ND + 2;
 };
+static_assert(LayC::BYTES <= SMEM_MAX, "pass C shared memory");
+static_assert(8 * LayC::NBARS + 8 <= CTRL_BYTES, "pass C control block");
 
 __global__ void __launch_bounds__(LayC::NTHREADS, 1)
 pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mc,
@@ -661,12 +694,12 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
     const uint32_t FULL = sb + L::CTRL, EMPTY = FULL + 8 * S, KREADY = EMPTY + 8 * S, CFULL = KREADY + 8 * S,
                    CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
                    DREADY = TFREE + 8 * NTM, DFREE = DREADY + 8 * ND, PFREE = DFREE + 8 * ND;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * (3 * S + 2 * NT + 2 * NTM + 2 * ND + 2));
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * L::NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     float *dens = reinterpret_cast<float *>(sm + L::D_OFF);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const long long nunits = (long long)p.nseg * p.nquads * p.B;
+    const int nunits = p.nseg * p.nquads * p.B;
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
@@ -716,7 +749,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             int ub = 0, issued = 0, last_tb = 0;
             uint32_t last_phase = 0;
             bool ok = true;
-            for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const Unit x = unit_at(p, u);
                 if (x.ntile == 0) continue;
                 const uint64_t pd = pdesc0 + (uint64_t)((ub * L::P_BYTES) >> 4);
@@ -751,12 +784,12 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         }
     } else if (w >= L::W_PRO0) {
         // ---------------- prologue: prefix staging, phi, 1/den, rotary, hi/lo split ----------------
-        const int pw = w - L::W_PRO0, pt = tid - 32 * L::W_PRO0, g = pw >> 3;   // heads 2g, 2g+1
-        const int r = 8 * (pw & 7) + (lane >> 2), f = lane & 3;                  // token row, quarter
+        const int pw = w - L::W_PRO0, pt = tid - 32 * L::W_PRO0;
+        const ProOffs o = pro_offsets(pw, lane);
         pdl_wait();   // the prefix states come from the previous kernel
         Ring fr = {0, 0u}, cr = {0, 0u}, dr = {0, 1u}, br = {0, 1u};   // stage full, table full, 1/den free, P free
         bool ok = true;
-        for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+        for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
             if (x.ntile == 0) continue;
             const int ub = br.idx;
@@ -766,39 +799,52 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 break;
             }
             ring_next<2>(br);
-            {   // the quad's prefix state -> A operand rows m = (head, c): [P hi | P lo]; thread = (m, quarter of e)
-                const int m = pt >> 2, qq = pt & 3, head = HQ * x.hq + (m >> 5);
-                float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            {   // the quad's prefix state -> A operand rows m = (head, c): [P hi | P lo]; thread = (m, half of e)
+                const int m = pt >> 1, half = pt & 1, head = HQ * x.hq + (m >> 5);
+                float y[16];
                 if (head < p.H) {
                     const float4 *src =
-                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + (m & 31) * LCLA_D + 8 * qq);
-                    a = src[0];
-                    b = src[1];
-                }
-                const float y[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-                uint32_t hw[4], lw[4];
+                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + (m & 31) * LCLA_D + 16 * half);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 v4 = src[j];
+                        y[4 * j] = v4.x;
+                        y[4 * j + 1] = v4.y;
+                        y[4 * j + 2] = v4.z;
+                        y[4 * j + 3] = v4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) y[j] = 0.f;
+                }
+                uint32_t hw[8], lw[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
                     const float2 hf = __bfloat1622float2(h2);
                     hw[j] = bf2_bits(h2);
                     lw[j] = pack_bf2(y[2 * j] - hf.x, y[2 * j + 1] - hf.y);
                 }
-                store_quarter_hi_lo(sm + L::P_OFF + ub * L::P_BYTES, m, qq, hw, lw);
+                unsigned char *row = sm + L::P_OFF + ub * L::P_BYTES + m * 128;
+                const int sw = m & 7;
+                sts128(row + (((2 * half) ^ sw) << 4), hw);
+                sts128(row + (((2 * half + 1) ^ sw) << 4), hw + 4);
+                sts128(row + (((4 + 2 * half) ^ sw) << 4), lw);
+                sts128(row + (((5 + 2 * half) ^ sw) << 4), lw + 4);
             }
-            float zq[2][8];   // z[8f, 8f+8) of heads 2g, 2g+1
+            float zq[HQ][8];   // z[8f, 8f+8) of each head of the quad
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int head = HQ * x.hq + 2 * g + hh;
-                float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            for (int h = 0; h < HQ; ++h) {
+                const int head = HQ * x.hq + h;
+                float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
                 if (head < p.H) {
                     const float4 *src =
-                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + LCLA_D * LCLA_D + 8 * f);
-                    a = src[0];
-                    b = src[1];
+                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + LCLA_D * LCLA_D + 8 * o.f);
+                    a4 = src[0];
+                    b4 = src[1];
                 }
-                zq[hh][0] = a.x; zq[hh][1] = a.y; zq[hh][2] = a.z; zq[hh][3] = a.w;
-                zq[hh][4] = b.x; zq[hh][5] = b.y; zq[hh][6] = b.z; zq[hh][7] = b.w;
+                zq[h][0] = a4.x; zq[h][1] = a4.y; zq[h][2] = a4.z; zq[h][3] = a4.w;
+                zq[h][4] = b4.x; zq[h][5] = b4.y; zq[h][6] = b4.z; zq[h][7] = b4.w;
             }
             for (int i = 0; i < x.ntile; ++i) {
                 const int st = fr.idx, ct = cr.idx, db = dr.idx;
@@ -814,40 +860,43 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 ring_next<ND>(dr);
                 unsigned char *stg = sm + st * L::STAGE;
                 const unsigned char *tab = sm + L::C_OFF + ct * TAB_BYTES;
-                const float4 c4 = load_quarter_table(tab, r, f);
-                const float4 s4 = load_quarter_table(tab + TAB_BYTES / 2, r, f);
-                const uint4 q0 = load_quarter_row(stg + g * 8192, r, 0, f);   // head 2g
-                const uint4 q1 = load_quarter_row(stg + g * 8192, r, 1, f);   // head 2g+1
-                __syncwarp();
-                if (lane == 0) bar_arrive(CEMPTY + 8 * ct);   // table rows consumed
-                float den[2];
+                const float4 c4 = ldsf4(tab + o.tab);
+                const float4 s4 = ldsf4(tab + TAB_BYTES / 2 + o.tab);
+                uint4 qr[HQ];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const uint4 qv = hh ? q1 : q0;
-                    uint32_t fw[4] = {qv.x, qv.y, qv.z, qv.w}, hi[4], lo[4];
+                for (int h = 0; h < HQ; ++h) qr[h] = lds128(stg + raw_off(o, h));
+                float den[HQ];
+#pragma unroll
+                for (int h = 0; h < HQ; ++h) {
+                    uint32_t fw[4] = {qr[h].x, qr[h].y, qr[h].z, qr[h].w}, hi[4], lo[4];
                     float dd = 0.f;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         fw[j] = relu2(fw[j]);
-                        dd = fmaf(bf_lo(fw[j]), zq[hh][2 * j], dd);
-                        dd = fmaf(bf_hi(fw[j]), zq[hh][2 * j + 1], dd);
+                        dd = fmaf(bf_lo(fw[j]), zq[h][2 * j], dd);
+                        dd = fmaf(bf_hi(fw[j]), zq[h][2 * j + 1], dd);
                     }
-                    den[hh] = dd;
+                    den[h] = dd;
                     rope_split4(fw, c4, s4, hi, lo);
-                    store_quarter_hi_lo(stg + atom_of(2 * g + hh) * 8192, r, f, hi, lo);
+                    unsigned char *blk = stg + atom_of(h) * 8192;
+                    sts128(blk + o.a, hi);
+                    sts128(blk + o.b, lo);
                 }
                 // z . phi(q) of each head over the token's four quarters (lanes 4(r & 7) .. +3)
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    den[hh] += __shfl_xor_sync(ALL, den[hh], 1);
-                    den[hh] += __shfl_xor_sync(ALL, den[hh], 2);
+                for (int h = 0; h < HQ; ++h) {
+                    den[h] += __shfl_xor_sync(ALL, den[h], 1);
+                    den[h] += __shfl_xor_sync(ALL, den[h], 2);
                 }
-                if (f < 2) dens[(db * HQ + 2 * g + f) * T + r] = 1.0f / ((f ? den[1] : den[0]) + eps);
+                const int f = o.f;
+                const float mine = f == 0 ? den[0] : f == 1 ? den[1] : f == 2 ? den[2] : den[3];
+                dens[(db * HQ + f) * T + o.r] = 1.0f / (mine + eps);   // lane f: head f
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
                     bar_arrive(KREADY + 8 * st);
                     bar_arrive(DREADY + 8 * db);
+                    bar_arrive(CEMPTY + 8 * ct);   // after the rows have been used: see release_after_use
                 }
             }
         }
@@ -860,7 +909,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         int ob = 0;
         Ring tr = {0, 0u}, dr = {0, 0u};   // TMEM full, 1/den ready
         bool ok = true;
-        for (long long u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+        for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
             const int head = HQ * x.hq + q;
             for (int i = 0; i < x.ntile; ++i) {
@@ -889,7 +938,6 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 for (int half = 0; half < 2; ++half) {   // tokens [32 half, 32 half + 32)
                     uint32_t v[32], word[16];
                     tmem_ld32(ta + 32 * half, v);
-                    tmem_wait_ld();
                     // own column c for tokens (2m, 2m+1) packed; lane pairs (2i, 2i+1) trade them so that
                     // the even lane holds row 2m's (c, c+1) and the odd lane row 2m+1's
 #pragma unroll
