@@ -140,6 +140,25 @@ unsigned scan_blocks(const LclaPlan &p)
     return (unsigned)((n + lcla::SCAN_THREADS - 1) / lcla::SCAN_THREADS);
 }
 
+// Partials -> prefixes: the grouped two-phase scan when its group sums fit in
+// shared memory, else the one-thread-per-column serial scan.
+void launch_scan(const LclaPlan &p, const float *part, float *pref, const float *state_in, float *state_out,
+                 cudaStream_t st)
+{
+    const int ngroups = p.chunk ? p.nseg : p.nb;
+    if (ngroups <= lcla::SCANG_MAX_GROUPS) {
+        const size_t n4 = (size_t)p.B * p.H * (LCLA_SZ / lcla::SCAN_VEC);
+        const int smem = ngroups * 32 * 16;
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(lcla::scan_states_grouped, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        launch_pdl(lcla::scan_states_grouped, dim3((unsigned)((n4 + 31) / 32)), dim3(32 * lcla::SCANG_WARPS),
+                   (size_t)smem, st, p, part, pref, state_in, state_out);
+    } else {
+        launch_pdl(lcla::scan_states, dim3(scan_blocks(p)), dim3(lcla::SCAN_THREADS), 0, st, p, part, pref,
+                   state_in, state_out);
+    }
+}
+
 template <typename F>
 void set_smem(F *kernel, int bytes)
 {
@@ -176,14 +195,14 @@ bool map_tokens(CUtensorMap *m, const void *base, int B, int N, int H)
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [B, N, H*d] bf16 output blocks of one head x 64 tokens, no swizzle (TMA stores).
+// [B, N, H*d] bf16 output blocks of one head x 32 tokens, no swizzle (TMA stores).
 bool map_out_blocks(CUtensorMap *m, const void *base, int B, int N, int H)
 {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)H * LCLA_D, (cuuint64_t)N, (cuuint64_t)B};
     cuuint64_t strides[2] = {(cuuint64_t)H * LCLA_D * 2, (cuuint64_t)N * H * LCLA_D * 2};
-    cuuint32_t box[3] = {LCLA_D, LCLA_TC_T, 1};
+    cuuint32_t box[3] = {LCLA_D, LCLA_TC_T / 2, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -227,8 +246,7 @@ bool launch_tc(const void *q, const void *k, const void *v, const float *rc, con
     lcla::tc::pass_a_tc<<<grid, lcla::tc::LayA::NTHREADS, lcla::tc::LayA::BYTES, st>>>(mk, mv, mc, ms, p, part,
                                                                                        status);
     if (ev) cudaEventRecord(ev[1], st);
-    launch_pdl(lcla::scan_states, dim3(scan_blocks(p)), dim3(lcla::SCAN_THREADS), 0, st, p, part, pref,
-               state_in, state_out);
+    launch_scan(p, part, pref, state_in, state_out, st);
     if (ev) cudaEventRecord(ev[2], st);
     launch_pdl(lcla::tc::pass_c_tc, grid, dim3(lcla::tc::LayC::NTHREADS), lcla::tc::LayC::BYTES, st, mq, mc, ms, mo, p,
                (const float *)pref, eps, (__nv_bfloat16 *)out, status);
@@ -254,8 +272,7 @@ int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const 
     lcla::pass_a_ffma<Tin><<<grid, 256, smem_a, st>>>(k, v, rc, rs, p, part);
 
     if (ev) cudaEventRecord(ev[1], st);
-    launch_pdl(lcla::scan_states, dim3(scan_blocks(p)), dim3(lcla::SCAN_THREADS), 0, st, p, part, pref,
-               state_in, state_out);
+    launch_scan(p, part, pref, state_in, state_out, st);
     if (ev) cudaEventRecord(ev[2], st);
 
     if (!p.chunk) {

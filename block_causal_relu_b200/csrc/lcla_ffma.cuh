@@ -679,4 +679,58 @@ scan_states(const LclaPlan p, const float *__restrict__ part, float *__restrict_
     if (state_out) reinterpret_cast<float4 *>(state_out)[x] = acc;
 }
 
+// Grouped scan: the same prefixes in two phases, for up to SCANG_MAX_GROUPS
+// groups (block mode: a block's nsb segments; chunk mode: one segment).  A
+// CTA owns 32 float4 columns of the state slice; phase 1 has its 8 warps sum
+// the groups' segment partials in parallel (all loads of a group in flight)
+// into shared memory; phase 2 has one warp run the prefix over the group sums
+// in group order and write pref (inclusive per block in block mode,
+// exclusive per segment in chunk mode) and the total.
+// ---------------------------------------------------------------------------
+constexpr int SCANG_WARPS = 8;
+constexpr int SCANG_MAX_GROUPS = 256;   // shared memory: groups x 32 x 16 B
+
+__global__ void __launch_bounds__(32 * SCANG_WARPS)
+scan_states_grouped(const LclaPlan p, const float *__restrict__ part, float *__restrict__ pref,
+                    const float *state_in, float *state_out)
+{
+    extern __shared__ float4 gsum[];   // [groups][32]
+    const size_t n4 = (size_t)p.B * p.H * (LCLA_SZ / SCAN_VEC);
+    const int lane = threadIdx.x & 31, wg = threadIdx.x >> 5;
+    const size_t x = (size_t)blockIdx.x * 32 + lane;
+    const bool live = x < n4;
+    const int ngroups = p.chunk ? p.nseg : p.nb, per = p.chunk ? 1 : p.nsb;
+    const float4 *part4 = reinterpret_cast<const float4 *>(part);
+    pdl_wait();
+    pdl_trigger();
+    for (int gi = wg; gi < ngroups; gi += SCANG_WARPS) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (live) {
+            constexpr int BATCH = 8;
+            for (int s0 = 0; s0 < per; s0 += BATCH) {
+                float4 v[BATCH];
+#pragma unroll
+                for (int j = 0; j < BATCH; ++j)
+                    if (s0 + j < per) v[j] = __ldcg(part4 + ((size_t)gi * per + s0 + j) * n4 + x);
+#pragma unroll
+                for (int j = 0; j < BATCH; ++j)
+                    if (s0 + j < per) add4(acc, v[j]);
+            }
+        }
+        gsum[gi * 32 + lane] = acc;
+    }
+    __syncthreads();
+    if (wg == 0 && live) {
+        float4 *pref4 = reinterpret_cast<float4 *>(pref);
+        float4 acc = state_in ? reinterpret_cast<const float4 *>(state_in)[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int gi = 0; gi < ngroups; ++gi) {
+            const float4 v = gsum[gi * 32 + lane];
+            if (p.chunk) pref4[(size_t)gi * n4 + x] = acc;
+            add4(acc, v);
+            if (!p.chunk) pref4[(size_t)gi * n4 + x] = acc;
+        }
+        if (state_out) reinterpret_cast<float4 *>(state_out)[x] = acc;
+    }
+}
+
 }  // namespace lcla

@@ -21,8 +21,10 @@
 //                   row of all four heads, so each rotary entry is read once
 //                   and the fixed per-tile work (waits, fences, arrivals) is
 //                   spread over 32 elements per thread;
-//   drain/epilogue  (warps 0-3; warp q owns head q of the quad and tensor
-//                   memory lanes 32q..32q+31) tensor memory -> registers.
+//   drain/epilogue  tensor memory -> registers: warp w reads tensor memory
+//                   lanes 32(w & 3)..+31, which belong to head w & 3 of the
+//                   quad (pass A: 4 drain warps; pass C: 8 epilogue warps,
+//                   two per head, one per half of the tile's tokens).
 // Roles talk only through mbarriers.  A stage holds one tile from its TMA
 // load until the tile's MMAs complete; the table slot is released as soon as
 // the prologue has read it.
@@ -39,8 +41,9 @@
 // hi + lo, rows (head, token), K-major [q~hi | q~lo]:
 //     D[(h', c)][(h, tok)] = Phi.q~hi + Plo.q~hi + Phi.q~lo   (6 MMAs of K = 16).
 // Warp q scales the diagonal block by 1 / (z . phi(q) + eps), computed by the
-// prologue, writes it as bf16 [64 tok][32 c] into shared memory and stores it
-// with one TMA store (ragged tiles: plain stores of the valid rows).
+// prologue, writes it as bf16 [32 tok][32 c] into shared memory and stores it
+// with one TMA store; two epilogue warps share a head, one per 32 tokens
+// (ragged tiles: plain stores of the valid rows).
 //
 // Every mbarrier wait is bounded (LCLA_TC_WAIT_NS of globaltimer) and gives
 // up when another role has set the CTA's abort flag; each warp makes the
@@ -664,14 +667,14 @@ struct LayC {
     static constexpr int STAGE = 32768;
     static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
     static constexpr int P_OFF = C_OFF + NT * TAB_BYTES, P_BYTES = 16384;   // 2 x [128 rows (head, c)][P hi | P lo]
-    static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 4 warps x 2 x [64 tok][32 c] bf16
-    static constexpr int D_OFF = O_OFF + 4 * 2 * 4096;              // 1/den ring [ND][4 heads][64 tok]
+    static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 8 warps x 2 x [32 tok][32 c] bf16
+    static constexpr int D_OFF = O_OFF + 8 * 2 * 2048;              // 1/den ring [ND][4 heads][64 tok]
     static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
     static constexpr int ND = 4;                                    // 1/den ring
     static constexpr int CTRL = D_OFF + ND * HQ * T * 4;            // mbarriers, tensor-memory slot, abort flag
     static constexpr int BYTES = CTRL + CTRL_BYTES + 1024;          // + worst-case 1024-byte alignment pad
-    static constexpr int NTHREADS = 448;                            // epilogue 0-3, producer 4, MMA 5, prologue 6-13
-    static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6;
+    static constexpr int NTHREADS = 576;                            // epilogue 0-7, producer 8, MMA 9, prologue 10-17
+    static constexpr int W_PROD = 8, W_MMA = 9, W_PRO0 = 10, NEPI = 8;
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
     static constexpr int TMEM_COLS = NTM * 256;
     static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 2 * ND + 2;
@@ -713,11 +716,11 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         }
         for (int i = 0; i < NTM; ++i) {
             bar_init(TFULL + 8 * i, 1);
-            bar_init(TFREE + 8 * i, 4);
+            bar_init(TFREE + 8 * i, L::NEPI);
         }
         for (int i = 0; i < ND; ++i) {
             bar_init(DREADY + 8 * i, NPRO);
-            bar_init(DFREE + 8 * i, 4);
+            bar_init(DFREE + 8 * i, L::NEPI);
         }
         for (int i = 0; i < 2; ++i) bar_init(PFREE + 8 * i, 1);
         *abort_flag = 0;
@@ -902,10 +905,11 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         }
     } else {
         // ---------------- epilogue: tensor memory -> scaled bf16 -> TMA store ----------------
-        const int q = w;   // head of the quad; tensor-memory lanes 32q + c, c = lane
+        // warp e: head q = e & 3 (tensor-memory lanes 32q + c, c = lane), tokens [32 hf, 32 hf + 32), hf = e >> 2
+        const int q = w & 3, hf = w >> 2;
         const int odd = lane & 1;
         const size_t tstride = (size_t)p.H * LCLA_D;   // elements per token
-        unsigned char *ob0 = sm + L::O_OFF + q * 2 * 4096;
+        unsigned char *ob0 = sm + L::O_OFF + w * 2 * 2048;
         int ob = 0;
         Ring tr = {0, 0u}, dr = {0, 0u};   // TMEM full, 1/den ready
         bool ok = true;
@@ -925,42 +929,25 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 tc_after();
                 const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
                 const bool whole = nt == T;
-                uint32_t *obuf = reinterpret_cast<uint32_t *>(ob0 + ob * 4096);
+                uint32_t *obuf = reinterpret_cast<uint32_t *>(ob0 + ob * 2048);
                 if (whole) {
                     if (lane == 0) bulk_wait_read1();   // this buffer's previous store has read it
                     __syncwarp();
                 }
-                const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q);
-                const float4 *iv = reinterpret_cast<const float4 *>(dens + (db * HQ + q) * T);
-                uint32_t *gout = reinterpret_cast<uint32_t *>(out + ((size_t)x.b * p.N + t) * tstride +
-                                                              (size_t)head * LCLA_D + (lane & ~1));
+                uint32_t v[32], word[16];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q) + 32 * hf, v);
+                const float4 *iv = reinterpret_cast<const float4 *>(dens + (db * HQ + q) * T + 32 * hf);
+                // own column c for tokens (2m, 2m+1) packed; lane pairs (2i, 2i+1) trade them so that the
+                // even lane holds row 2m's (c, c+1) and the odd lane row 2m+1's
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {   // tokens [32 half, 32 half + 32)
-                    uint32_t v[32], word[16];
-                    tmem_ld32(ta + 32 * half, v);
-                    // own column c for tokens (2m, 2m+1) packed; lane pairs (2i, 2i+1) trade them so that
-                    // the even lane holds row 2m's (c, c+1) and the odd lane row 2m+1's
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 s = iv[j4];
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 s = iv[8 * half + j4];
-#pragma unroll
-                        for (int k = 0; k < 2; ++k) {
-                            const uint32_t mine = pack_bf2(__uint_as_float(v[4 * j4 + 2 * k]) * (k ? s.z : s.x),
-                                                           __uint_as_float(v[4 * j4 + 2 * k + 1]) * (k ? s.w : s.y));
-                            const uint32_t other = __shfl_xor_sync(ALL, mine, 1);
-                            word[2 * j4 + k] = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
-                        }
-                    }
-                    // word[j] is row 2(16 half + j) + odd; branch once per half, outside the arithmetic
-                    if (whole) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) obuf[(32 * half + 2 * j + odd) * 16 + (lane >> 1)] = word[j];
-                    } else if (head < p.H) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int tok = 32 * half + 2 * j + odd;
-                            if (tok < nt) gout[(size_t)tok * (tstride / 2)] = word[j];
-                        }
+                    for (int k = 0; k < 2; ++k) {
+                        const uint32_t mine = pack_bf2(__uint_as_float(v[4 * j4 + 2 * k]) * (k ? s.z : s.x),
+                                                       __uint_as_float(v[4 * j4 + 2 * k + 1]) * (k ? s.w : s.y));
+                        const uint32_t other = __shfl_xor_sync(ALL, mine, 1);
+                        word[2 * j4 + k] = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
                     }
                 }
                 tc_before();
@@ -969,14 +956,25 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     bar_arrive(TFREE + 8 * tb);
                     bar_arrive(DFREE + 8 * db);
                 }
+                // word[j] is row 2j + odd of this warp's 32 tokens; branch once, outside the arithmetic
                 if (whole) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) obuf[(2 * j + odd) * 16 + (lane >> 1)] = word[j];
                     fence_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        if (head < p.H) tma_store3(&mo, s32(obuf), LCLA_D * head, t, x.b);
+                        if (head < p.H) tma_store3(&mo, s32(obuf), LCLA_D * head, t + 32 * hf, x.b);
                         bulk_commit();   // one group per buffer use keeps the read-wait accounting exact
                     }
                     ob ^= 1;
+                } else if (head < p.H) {
+                    uint32_t *gout = reinterpret_cast<uint32_t *>(out + ((size_t)x.b * p.N + t + 32 * hf) * tstride +
+                                                                  (size_t)head * LCLA_D + (lane & ~1));
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int tok = 2 * j + odd;
+                        if (32 * hf + tok < nt) gout[(size_t)tok * (tstride / 2)] = word[j];
+                    }
                 }
             }
         }
