@@ -15,12 +15,12 @@
 //   producer warp   TMA loads of each tile's q or k, v boxes into a ring of
 //                   stages and of its rotary rows into a smaller table ring;
 //   MMA warp        one thread issues tcgen05.mma and tcgen05.commit;
-//   prologue warps  (8) ReLU, rotary, bf16 hi + lo split of q or k, written
-//                   in place over the stage's raw input as the MMA operand;
-//                   thread (token r, quarter f) does a quarter of one token
-//                   row of all four heads, so each rotary entry is read once
-//                   and the fixed per-tile work (waits, fences, arrivals) is
-//                   spread over 32 elements per thread;
+//   prologue warps  ReLU, rotary, bf16 hi + lo split of q or k, written in
+//                   place over the stage's raw input as the MMA operand
+//                   (pass A: 8 warps, a thread doing one token quarter of all
+//                   four heads; pass C: 16 warps, one token quarter of a head
+//                   pair -- pass C's register budget is shared with its 8
+//                   epilogue warps);
 //   drain/epilogue  tensor memory -> registers: warp w reads tensor memory
 //                   lanes 32(w & 3)..+31, which belong to head w & 3 of the
 //                   quad (pass A: 4 drain warps; pass C: 8 epilogue warps,
@@ -303,6 +303,31 @@ __device__ __forceinline__ ProOffs pro_offsets(int pw, int lane)
 }
 // Raw input quarter of head h in a stage (box h >> 1, chunk f or 4 + f).
 __device__ __forceinline__ int raw_off(const ProOffs &o, int h) { return (h >> 1) * 8192 + ((h & 1) ? o.b : o.a); }
+
+// Pass C's prologue has 16 warps, a thread doing one token quarter of one
+// head pair g = lane & 1 (heads 2g, 2g+1), quarter f = (lane >> 1) & 3, on
+// one of the warp's four rows {8k, 8k+1, 8k+4, 8k+5} + 2 (pw & 1), k = pw >> 1
+// (bank-conflict free; the two pairs' identical rotary reads are one
+// broadcast).  in0 / in1: the raw chunks of heads 2g / 2g+1 in box g, which
+// are also atom g's hi / lo chunks; out2 / out3: atom 2+g's hi / lo chunks.
+struct PairOffs {
+    int g, f, r, in0, in1, out2, out3, tab;
+};
+__device__ __forceinline__ PairOffs pair_offsets(int pw, int lane)
+{
+    PairOffs o;
+    o.g = lane & 1;
+    o.f = (lane >> 1) & 3;
+    const int rr = lane >> 3;
+    o.r = 8 * (pw >> 1) + 2 * (pw & 1) + (rr & 1) + 4 * (rr >> 1);
+    const int sw = o.r & 7, row = o.r * 128;
+    o.in0 = o.g * 8192 + row + ((o.f ^ sw) << 4);
+    o.in1 = o.g * 8192 + row + (((4 + o.f) ^ sw) << 4);
+    o.out2 = (2 + o.g) * 8192 + row + ((o.f ^ sw) << 4);
+    o.out3 = (2 + o.g) * 8192 + row + (((4 + o.f) ^ sw) << 4);
+    o.tab = o.r * 64 + ((o.f ^ ((o.r >> 1) & 3)) << 4);
+    return o;
+}
 __device__ __forceinline__ uint4 lds128(const unsigned char *p) { return *reinterpret_cast<const uint4 *>(p); }
 __device__ __forceinline__ float4 ldsf4(const unsigned char *p) { return *reinterpret_cast<const float4 *>(p); }
 __device__ __forceinline__ void sts128(unsigned char *p, const uint32_t *w)
@@ -340,7 +365,8 @@ constexpr int NT = 3;             // rotary-table ring slots ([cos 4 KB | sin 4 
 constexpr int CTRL_BYTES = 512;   // control block: mbarriers (8 B each), tensor-memory slot, abort flag
 constexpr int SMEM_MAX = 232448;  // dynamic shared memory a CTA may opt in to
 constexpr int TAB_BYTES = 8192;
-constexpr int NPRO = 8;           // prologue warps
+constexpr int NPRO = 8;           // pass A prologue warps
+constexpr int NPRO_C = 16;        // pass C prologue warps
 
 // Producer: per tile, TMA loads of the quad's input boxes into the stage ring
 // (two [64 token][2 heads] boxes per tensor map, heads past H read as zeros)
@@ -673,7 +699,7 @@ struct LayC {
     static constexpr int ND = 4;                                    // 1/den ring
     static constexpr int CTRL = D_OFF + ND * HQ * T * 4;            // mbarriers, tensor-memory slot, abort flag
     static constexpr int BYTES = CTRL + CTRL_BYTES + 1024;          // + worst-case 1024-byte alignment pad
-    static constexpr int NTHREADS = 576;                            // epilogue 0-7, producer 8, MMA 9, prologue 10-17
+    static constexpr int NTHREADS = 832;                            // epilogue 0-7, producer 8, MMA 9, prologue 10-25
     static constexpr int W_PROD = 8, W_MMA = 9, W_PRO0 = 10, NEPI = 8;
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
     static constexpr int TMEM_COLS = NTM * 256;
@@ -708,18 +734,18 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         for (int i = 0; i < S; ++i) {
             bar_init(FULL + 8 * i, 1);
             bar_init(EMPTY + 8 * i, 1);
-            bar_init(KREADY + 8 * i, NPRO);
+            bar_init(KREADY + 8 * i, NPRO_C);
         }
         for (int i = 0; i < NT; ++i) {
             bar_init(CFULL + 8 * i, 1);
-            bar_init(CEMPTY + 8 * i, NPRO);
+            bar_init(CEMPTY + 8 * i, NPRO_C);
         }
         for (int i = 0; i < NTM; ++i) {
             bar_init(TFULL + 8 * i, 1);
             bar_init(TFREE + 8 * i, L::NEPI);
         }
         for (int i = 0; i < ND; ++i) {
-            bar_init(DREADY + 8 * i, NPRO);
+            bar_init(DREADY + 8 * i, NPRO_C);
             bar_init(DFREE + 8 * i, L::NEPI);
         }
         for (int i = 0; i < 2; ++i) bar_init(PFREE + 8 * i, 1);
@@ -788,7 +814,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
     } else if (w >= L::W_PRO0) {
         // ---------------- prologue: prefix staging, phi, 1/den, rotary, hi/lo split ----------------
         const int pw = w - L::W_PRO0, pt = tid - 32 * L::W_PRO0;
-        const ProOffs o = pro_offsets(pw, lane);
+        const PairOffs o = pair_offsets(pw, lane);
         pdl_wait();   // the prefix states come from the previous kernel
         Ring fr = {0, 0u}, cr = {0, 0u}, dr = {0, 1u}, br = {0, 1u};   // stage full, table full, 1/den free, P free
         bool ok = true;
@@ -802,43 +828,30 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 break;
             }
             ring_next<2>(br);
-            {   // the quad's prefix state -> A operand rows m = (head, c): [P hi | P lo]; thread = (m, half of e)
-                const int m = pt >> 1, half = pt & 1, head = HQ * x.hq + (m >> 5);
-                float y[16];
+            {   // the quad's prefix state -> A operand rows m = (head, c): [P hi | P lo]; thread = (m, quarter of e)
+                const int m = pt >> 2, qq = pt & 3, head = HQ * x.hq + (m >> 5);
+                float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
                 if (head < p.H) {
                     const float4 *src =
-                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + (m & 31) * LCLA_D + 16 * half);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float4 v4 = src[j];
-                        y[4 * j] = v4.x;
-                        y[4 * j + 1] = v4.y;
-                        y[4 * j + 2] = v4.z;
-                        y[4 * j + 3] = v4.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) y[j] = 0.f;
+                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + (m & 31) * LCLA_D + 8 * qq);
+                    a4 = src[0];
+                    b4 = src[1];
                 }
-                uint32_t hw[8], lw[8];
+                const float y[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+                uint32_t hw[4], lw[4];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 4; ++j) {
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
                     const float2 hf = __bfloat1622float2(h2);
                     hw[j] = bf2_bits(h2);
                     lw[j] = pack_bf2(y[2 * j] - hf.x, y[2 * j + 1] - hf.y);
                 }
-                unsigned char *row = sm + L::P_OFF + ub * L::P_BYTES + m * 128;
-                const int sw = m & 7;
-                sts128(row + (((2 * half) ^ sw) << 4), hw);
-                sts128(row + (((2 * half + 1) ^ sw) << 4), hw + 4);
-                sts128(row + (((4 + 2 * half) ^ sw) << 4), lw);
-                sts128(row + (((5 + 2 * half) ^ sw) << 4), lw + 4);
+                store_quarter_hi_lo(sm + L::P_OFF + ub * L::P_BYTES, m, qq, hw, lw);
             }
-            float zq[HQ][8];   // z[8f, 8f+8) of each head of the quad
+            float zq[2][8];   // z[8f, 8f+8) of heads 2g, 2g+1
 #pragma unroll
-            for (int h = 0; h < HQ; ++h) {
-                const int head = HQ * x.hq + h;
+            for (int hh = 0; hh < 2; ++hh) {
+                const int head = HQ * x.hq + 2 * o.g + hh;
                 float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
                 if (head < p.H) {
                     const float4 *src =
@@ -846,8 +859,8 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     a4 = src[0];
                     b4 = src[1];
                 }
-                zq[h][0] = a4.x; zq[h][1] = a4.y; zq[h][2] = a4.z; zq[h][3] = a4.w;
-                zq[h][4] = b4.x; zq[h][5] = b4.y; zq[h][6] = b4.z; zq[h][7] = b4.w;
+                zq[hh][0] = a4.x; zq[hh][1] = a4.y; zq[hh][2] = a4.z; zq[hh][3] = a4.w;
+                zq[hh][4] = b4.x; zq[hh][5] = b4.y; zq[hh][6] = b4.z; zq[hh][7] = b4.w;
             }
             for (int i = 0; i < x.ntile; ++i) {
                 const int st = fr.idx, ct = cr.idx, db = dr.idx;
@@ -865,35 +878,33 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 const unsigned char *tab = sm + L::C_OFF + ct * TAB_BYTES;
                 const float4 c4 = ldsf4(tab + o.tab);
                 const float4 s4 = ldsf4(tab + TAB_BYTES / 2 + o.tab);
-                uint4 qr[HQ];
+                const uint4 q0 = lds128(stg + o.in0);   // head 2g
+                const uint4 q1 = lds128(stg + o.in1);   // head 2g+1
+                float den[2];
 #pragma unroll
-                for (int h = 0; h < HQ; ++h) qr[h] = lds128(stg + raw_off(o, h));
-                float den[HQ];
-#pragma unroll
-                for (int h = 0; h < HQ; ++h) {
-                    uint32_t fw[4] = {qr[h].x, qr[h].y, qr[h].z, qr[h].w}, hi[4], lo[4];
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint4 qv = hh ? q1 : q0;
+                    uint32_t fw[4] = {qv.x, qv.y, qv.z, qv.w}, hi[4], lo[4];
                     float dd = 0.f;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         fw[j] = relu2(fw[j]);
-                        dd = fmaf(bf_lo(fw[j]), zq[h][2 * j], dd);
-                        dd = fmaf(bf_hi(fw[j]), zq[h][2 * j + 1], dd);
+                        dd = fmaf(bf_lo(fw[j]), zq[hh][2 * j], dd);
+                        dd = fmaf(bf_hi(fw[j]), zq[hh][2 * j + 1], dd);
                     }
-                    den[h] = dd;
+                    den[hh] = dd;
                     rope_split4(fw, c4, s4, hi, lo);
-                    unsigned char *blk = stg + atom_of(h) * 8192;
-                    sts128(blk + o.a, hi);
-                    sts128(blk + o.b, lo);
+                    // head 2g -> atom g (over the raw chunks just read), head 2g+1 -> atom 2+g
+                    sts128(stg + (hh ? o.out2 : o.in0), hi);
+                    sts128(stg + (hh ? o.out3 : o.in1), lo);
                 }
-                // z . phi(q) of each head over the token's four quarters (lanes 4(r & 7) .. +3)
+                // z . phi(q) of each head over the token's four quarters (lane bits 1-2)
 #pragma unroll
-                for (int h = 0; h < HQ; ++h) {
-                    den[h] += __shfl_xor_sync(ALL, den[h], 1);
-                    den[h] += __shfl_xor_sync(ALL, den[h], 2);
+                for (int hh = 0; hh < 2; ++hh) {
+                    den[hh] += __shfl_xor_sync(ALL, den[hh], 2);
+                    den[hh] += __shfl_xor_sync(ALL, den[hh], 4);
                 }
-                const int f = o.f;
-                const float mine = f == 0 ? den[0] : f == 1 ? den[1] : f == 2 ? den[2] : den[3];
-                dens[(db * HQ + f) * T + o.r] = 1.0f / (mine + eps);   // lane f: head f
+                if (o.f < 2) dens[(db * HQ + 2 * o.g + o.f) * T + o.r] = 1.0f / ((o.f ? den[1] : den[0]) + eps);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
