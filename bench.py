@@ -327,12 +327,15 @@ def main():
     bytes_a = 2 * tok_bytes + tab_bytes + nseg * sl
     bytes_c = 2 * tok_bytes + tab_bytes + npref * sl
     bytes_s = nseg * sl + npref * sl + sl
+    # the grouped scan serves plans with at most 256 prefix groups (blocks, or segments in chunk mode)
+    scan_name = "scan_states_grouped" if (plan["segments"] if plan["chunk_mode"] else plan["prefixes"]) <= 256 \
+        else "scan_states"
     if plan["tensor_cores"]:
         name_a, name_c = "pass_a_tc", "pass_c_tc"
     else:
         name_a, name_c = "pass_a_ffma", "pass_c_chunk_ffma" if plan["chunk_mode"] else "pass_c_ffma"
     passes = {"pass_a": (statistics.mean(pa), bytes_a, name_a),
-              "scan": (statistics.mean(sc), bytes_s, "scan_states"),
+              "scan": (statistics.mean(sc), bytes_s, scan_name),
               "pass_c": (statistics.mean(pc), bytes_c, name_c)}
     dom = max(passes, key=lambda kk: passes[kk][0])
     dms, dbytes, dname = passes[dom]
