@@ -190,6 +190,50 @@ def cpu_baseline(inp, seconds):
                       f"state), fp64, {threads} OpenMP threads, {el:.1f} s"}
 
 
+class Ranks:
+    """One process per GPU (torchrun): rank, world size and the two collectives
+    the timing needs -- a barrier and the max over ranks of a duration.  The
+    data path has none: every rank solves its own problem."""
+
+    def __init__(self, world, rank, backend, device=None, timeout_s=120):
+        import torch.distributed as dist
+        self.world, self.rank, self.backend, self.device = world, rank, backend, device
+        self.dist = dist
+        if world > 1:
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            if self.backend == "nccl":
+                self.dist.barrier(device_ids=[self.device.index])
+            else:
+                self.dist.barrier()
+
+    def max(self, x):
+        if self.world == 1:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=self.device if self.backend == "nccl" else "cpu")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+def rank_spec(base, rank):
+    """Rank r's problem: the same workload with its own seed (independent replicas)."""
+    from dataclasses import replace
+    return replace(base, seed=base.seed + 1000 * rank)
+
+
+def whole_job_rate(world, units, steps, ms):
+    """Units processed by all ranks per second, timed by the slowest rank (ms over `steps`)."""
+    return world * units * steps / (ms / 1e3)
+
+
 def run_reference(args):
     """Reference arm: the fp64 CPU oracle, rank 0 only, each step a bounded
     sample (a subset of heads) of the same workload."""
@@ -235,7 +279,6 @@ def main():
         return run_reference(args)
 
     import torch
-    import torch.distributed as dist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -244,27 +287,17 @@ def main():
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=device)
+    ranks = Ranks(world, rank, "nccl", device)
 
     def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local])
+        ranks.barrier()
         torch.cuda.synchronize(device)
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    max_over_ranks = ranks.max
 
     import block_causal_relu_b200 as lcla
 
-    base = NAMED[args.workload]
-    from dataclasses import replace
-    spec = replace(base, seed=base.seed + 1000 * rank)       # independent problem per rank
+    spec = rank_spec(NAMED[args.workload], rank)             # independent problem per rank
     inp = make_inputs(spec)
 
     def to_dev(a):
@@ -306,7 +339,7 @@ def main():
     ms_total = max_over_ranks(e0.elapsed_time(e1))
     ms = ms_total / K
     units = spec.token_heads
-    value = world * units * K / (ms_total / 1e3)
+    value = whole_job_rate(world, units, K, ms_total)
     # timed region 2: the same steps with events recorded between the passes
     # (lcla_forward_timed) for the per-kernel durations of the roofline
     for i in range(K):
@@ -378,7 +411,7 @@ def main():
         ems = max_over_ranks(a0.elapsed_time(a1))
         h2d = 3 * tok_bytes + tab_bytes
         d2h = tok_bytes + sl
-        e2e = {"value": world * units * KE / (ems / 1e3), "unit": UNIT,
+        e2e = {"value": whole_job_rate(world, units, KE, ems), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ems / KE, "steps": KE}
 
@@ -396,8 +429,7 @@ def main():
                 "pass_ms": pass_ms, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": 3 * K, "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
 
 
 if __name__ == "__main__":

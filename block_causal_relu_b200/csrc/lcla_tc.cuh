@@ -947,6 +947,9 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 }
                 uint32_t v[32], word[16];
                 tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q) + 32 * hf, v);
+                tc_before();
+                __syncwarp();
+                if (lane == 0) bar_arrive(TFREE + 8 * tb);   // the accumulator is in registers: free the slot
                 const float4 *iv = reinterpret_cast<const float4 *>(dens + (db * HQ + q) * T + 32 * hf);
                 // own column c for tokens (2m, 2m+1) packed; lane pairs (2i, 2i+1) trade them so that the
                 // even lane holds row 2m's (c, c+1) and the odd lane row 2m+1's
@@ -961,12 +964,8 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                         word[2 * j4 + k] = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
                     }
                 }
-                tc_before();
                 __syncwarp();
-                if (lane == 0) {
-                    bar_arrive(TFREE + 8 * tb);
-                    bar_arrive(DFREE + 8 * db);
-                }
+                if (lane == 0) bar_arrive(DFREE + 8 * db);   // 1/den values consumed above
                 // word[j] is row 2j + odd of this warp's 32 tokens; branch once, outside the arithmetic
                 if (whole) {
 #pragma unroll
