@@ -195,7 +195,7 @@ bool map_tokens(CUtensorMap *m, const void *base, int B, int N, int H)
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [B, N, H*d] bf16 output blocks of one head x 32 tokens, no swizzle (TMA stores).
+// [B, N, H*d] bf16 output blocks of one head x 32 tokens, 64-byte swizzle (TMA stores).
 bool map_out_blocks(CUtensorMap *m, const void *base, int B, int N, int H)
 {
     auto fn = encode_fn();
@@ -205,7 +205,7 @@ bool map_out_blocks(CUtensorMap *m, const void *base, int B, int N, int H)
     cuuint32_t box[3] = {LCLA_D, LCLA_TC_T / 2, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -15,7 +15,8 @@
 //   producer warp   TMA loads of each tile's q or k, v boxes into a ring of
 //                   stages and of its rotary rows into a smaller table ring;
 //   MMA warp        one thread issues tcgen05.mma and tcgen05.commit;
-//   prologue warps  ReLU, rotary, bf16 hi + lo split of q or k, written in
+//   prologue warps  ReLU, rotary (pass C: and the normaliser), bf16 hi + lo
+//                   split of q or k, written in
 //                   place over the stage's raw input as the MMA operand
 //                   (pass A: 8 warps, a thread doing one token quarter of all
 //                   four heads; pass C: 16 warps, one token quarter of a head
@@ -37,13 +38,16 @@
 // registers; the unrotated key sum z comes from the prologue's registers.
 //
 // Pass C.  A = the block's prefix state P of the quad split into hi + lo,
-// rows (h', c), K-major [P hi | P lo]; B = the rotated queries split into
+// rows (h', c), K-major [P hi | P lo]; B = the rotated queries, already
+// divided by their normaliser z . phi(q) + eps (fp32, before the split), in
 // hi + lo, rows (head, token), K-major [q~hi | q~lo]:
-//     D[(h', c)][(h, tok)] = Phi.q~hi + Plo.q~hi + Phi.q~lo   (6 MMAs of K = 16).
-// Warp q scales the diagonal block by 1 / (z . phi(q) + eps), computed by the
-// prologue, writes it as bf16 [32 tok][32 c] into shared memory and stores it
-// with one TMA store; two epilogue warps share a head, one per 32 tokens
-// (ragged tiles: plain stores of the valid rows).
+//     D[(h', c)][(h, tok)] = Phi.q~hi + Plo.q~hi + Phi.q~lo   (6 MMAs of K = 16),
+// so the diagonal block h = h' is the output itself.  Epilogue warp q reads it
+// in the 16x256b fragment (two c rows x two tokens per thread), packs token
+// pairs to bf16 and writes the [32 tok][32 c] box transposed with stmatrix
+// into a 64-byte-swizzled buffer, stored by one TMA store; two epilogue warps
+// share a head, one per 32 tokens (ragged tiles: the valid rows are copied
+// out of the same buffer with plain stores).
 //
 // Every mbarrier wait is bounded (LCLA_TC_WAIT_NS of globaltimer) and gives
 // up when another role has set the CTA's abort flag; each warp makes the
@@ -225,6 +229,35 @@ __device__ __forceinline__ void tmem_ld32(uint32_t ta, uint32_t *r)
         : "memory");
 }
 
+// Two 16-lane halves of a warp's lane quarter, 32 columns each (shape 16x256b,
+// four repeats): thread t gets, for half L (tensor-memory lanes ta + 16L + ...),
+// r[16L + 4j + i] = lane t/4 + 8(i >> 1), column 8j + 2(t % 4) + (i & 1) --
+// the accumulator fragment that stmatrix takes.  Loads and wait in one asm
+// statement, as in tmem_ld32.
+__device__ __forceinline__ void tmem_ld16x256_x4x2(uint32_t ta, uint32_t tb, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%32];\n"
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%33];\n"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(ta), "r"(tb)
+        : "memory");
+}
+
+// Four 8x8 b16 matrices stored transposed: matrix m's fragment (thread t holds
+// row t/4, columns 2(t%4), 2(t%4)+1 in w[m]) lands with fragment column k at
+// the 16-byte row whose address thread 8m + k passes.
+__device__ __forceinline__ void stsm4_trans(uint32_t addr, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3)
+{
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
+                 "r"(w2), "r"(w3)
+                 : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout, version 1).
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo)
 {
@@ -257,6 +290,22 @@ __device__ __forceinline__ void rope_split4(const uint32_t *fw, const float4 &c4
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         const float a = bf_lo(fw[p]), b = bf_hi(fw[p]);
+        const float y0 = a * cv[p] - b * sv[p];
+        const float y1 = a * sv[p] + b * cv[p];
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+        const float2 hf = __bfloat1622float2(h2);
+        hi[p] = bf2_bits(h2);
+        lo[p] = pack_bf2(y0 - hf.x, y1 - hf.y);
+    }
+}
+// rope_split4 of the features times a per-row factor g (applied in fp32, before the split).
+__device__ __forceinline__ void rope_split4_scaled(const uint32_t *fw, const float4 &c4, const float4 &s4, float g,
+                                                   uint32_t *hi, uint32_t *lo)
+{
+    const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float a = bf_lo(fw[p]) * g, b = bf_hi(fw[p]) * g;
         const float y0 = a * cv[p] - b * sv[p];
         const float y1 = a * sv[p] + b * cv[p];
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
@@ -694,19 +743,19 @@ struct LayC {
     static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
     static constexpr int P_OFF = C_OFF + NT * TAB_BYTES, P_BYTES = 16384;   // 2 x [128 rows (head, c)][P hi | P lo]
     static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 8 warps x 2 x [32 tok][32 c] bf16
-    static constexpr int D_OFF = O_OFF + 8 * 2 * 2048;              // 1/den ring [ND][4 heads][64 tok]
-    static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
-    static constexpr int ND = 4;                                    // 1/den ring
-    static constexpr int CTRL = D_OFF + ND * HQ * T * 4;            // mbarriers, tensor-memory slot, abort flag
+    static constexpr int OBUF = 2048;
+    static constexpr int CTRL = O_OFF + 8 * 2 * OBUF;               // mbarriers, tensor-memory slot, abort flag
     static constexpr int BYTES = CTRL + CTRL_BYTES + 1024;          // + worst-case 1024-byte alignment pad
     static constexpr int NTHREADS = 832;                            // epilogue 0-7, producer 8, MMA 9, prologue 10-25
     static constexpr int W_PROD = 8, W_MMA = 9, W_PRO0 = 10, NEPI = 8;
+    static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
     static constexpr int TMEM_COLS = NTM * 256;
-    static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 2 * ND + 2;
+    static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 2;
 };
 static_assert(LayC::BYTES <= SMEM_MAX, "pass C shared memory");
 static_assert(8 * LayC::NBARS + 8 <= CTRL_BYTES, "pass C control block");
+static_assert(LayC::O_OFF % 1024 == 0 && LayC::OBUF % 512 == 0, "64-byte-swizzled output boxes need 512-byte alignment");
 
 __global__ void __launch_bounds__(LayC::NTHREADS, 1)
 pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mc,
@@ -714,7 +763,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
           const float *__restrict__ pref, const float eps, __nv_bfloat16 *__restrict__ out, int *__restrict__ status)
 {
     using L = LayC;
-    constexpr int S = L::STAGES, NTM = L::NTM, ND = L::ND;
+    constexpr int S = L::STAGES, NTM = L::NTM;
     extern __shared__ __align__(1024) unsigned char smraw[];
     const uint32_t raw = s32(smraw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -722,10 +771,9 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
     const uint32_t sb = raw + pad;
     const uint32_t FULL = sb + L::CTRL, EMPTY = FULL + 8 * S, KREADY = EMPTY + 8 * S, CFULL = KREADY + 8 * S,
                    CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
-                   DREADY = TFREE + 8 * NTM, DFREE = DREADY + 8 * ND, PFREE = DFREE + 8 * ND;
+                   PFREE = TFREE + 8 * NTM;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * L::NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
-    float *dens = reinterpret_cast<float *>(sm + L::D_OFF);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int nunits = p.nseg * p.nquads * p.B;
@@ -743,10 +791,6 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         for (int i = 0; i < NTM; ++i) {
             bar_init(TFULL + 8 * i, 1);
             bar_init(TFREE + 8 * i, L::NEPI);
-        }
-        for (int i = 0; i < ND; ++i) {
-            bar_init(DREADY + 8 * i, NPRO_C);
-            bar_init(DFREE + 8 * i, L::NEPI);
         }
         for (int i = 0; i < 2; ++i) bar_init(PFREE + 8 * i, 1);
         *abort_flag = 0;
@@ -812,11 +856,11 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             if (!ok && issued > 0) bar_wait_quiet(TFULL + 8 * last_tb, last_phase);
         }
     } else if (w >= L::W_PRO0) {
-        // ---------------- prologue: prefix staging, phi, 1/den, rotary, hi/lo split ----------------
+        // ---------------- prologue: prefix staging, phi, normaliser, rotary, hi/lo split ----------------
         const int pw = w - L::W_PRO0, pt = tid - 32 * L::W_PRO0;
         const PairOffs o = pair_offsets(pw, lane);
         pdl_wait();   // the prefix states come from the previous kernel
-        Ring fr = {0, 0u}, cr = {0, 0u}, dr = {0, 1u}, br = {0, 1u};   // stage full, table full, 1/den free, P free
+        Ring fr = {0, 0u}, cr = {0, 0u}, br = {0, 1u};   // stage full, table full, P free
         bool ok = true;
         for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
@@ -863,40 +907,33 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 zq[hh][4] = b4.x; zq[hh][5] = b4.y; zq[hh][6] = b4.z; zq[hh][7] = b4.w;
             }
             for (int i = 0; i < x.ntile; ++i) {
-                const int st = fr.idx, ct = cr.idx, db = dr.idx;
+                const int st = fr.idx, ct = cr.idx;
                 bool fine = bar_wait(FULL + 8 * fr.idx, fr.phase, abort_flag);
                 fine = bar_wait(CFULL + 8 * cr.idx, cr.phase, abort_flag) && fine;
-                fine = bar_wait(DFREE + 8 * dr.idx, dr.phase, abort_flag) && fine;
                 if (!__all_sync(ALL, fine)) {
                     ok = false;
                     break;
                 }
                 ring_next<S>(fr);
                 ring_next<NT>(cr);
-                ring_next<ND>(dr);
                 unsigned char *stg = sm + st * L::STAGE;
                 const unsigned char *tab = sm + L::C_OFF + ct * TAB_BYTES;
                 const float4 c4 = ldsf4(tab + o.tab);
                 const float4 s4 = ldsf4(tab + TAB_BYTES / 2 + o.tab);
                 const uint4 q0 = lds128(stg + o.in0);   // head 2g
                 const uint4 q1 = lds128(stg + o.in1);   // head 2g+1
+                uint32_t fw[2][4] = {{q0.x, q0.y, q0.z, q0.w}, {q1.x, q1.y, q1.z, q1.w}};
                 float den[2];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const uint4 qv = hh ? q1 : q0;
-                    uint32_t fw[4] = {qv.x, qv.y, qv.z, qv.w}, hi[4], lo[4];
                     float dd = 0.f;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        fw[j] = relu2(fw[j]);
-                        dd = fmaf(bf_lo(fw[j]), zq[hh][2 * j], dd);
-                        dd = fmaf(bf_hi(fw[j]), zq[hh][2 * j + 1], dd);
+                        fw[hh][j] = relu2(fw[hh][j]);
+                        dd = fmaf(bf_lo(fw[hh][j]), zq[hh][2 * j], dd);
+                        dd = fmaf(bf_hi(fw[hh][j]), zq[hh][2 * j + 1], dd);
                     }
                     den[hh] = dd;
-                    rope_split4(fw, c4, s4, hi, lo);
-                    // head 2g -> atom g (over the raw chunks just read), head 2g+1 -> atom 2+g
-                    sts128(stg + (hh ? o.out2 : o.in0), hi);
-                    sts128(stg + (hh ? o.out3 : o.in1), lo);
                 }
                 // z . phi(q) of each head over the token's four quarters (lane bits 1-2)
 #pragma unroll
@@ -904,88 +941,90 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     den[hh] += __shfl_xor_sync(ALL, den[hh], 2);
                     den[hh] += __shfl_xor_sync(ALL, den[hh], 4);
                 }
-                if (o.f < 2) dens[(db * HQ + 2 * o.g + o.f) * T + o.r] = 1.0f / ((o.f ? den[1] : den[0]) + eps);
+                // 1 / (z . phi(q) + eps): quarters with even f divide for head 2g, odd f for head 2g+1,
+                // and trade the results (lane bit 1 is bit 0 of f)
+                const float mine = 1.0f / (((o.f & 1) ? den[1] : den[0]) + eps);
+                const float theirs = __shfl_xor_sync(ALL, mine, 2);
+                const float g0 = (o.f & 1) ? theirs : mine, g1 = (o.f & 1) ? mine : theirs;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t hi[4], lo[4];
+                    rope_split4_scaled(fw[hh], c4, s4, hh ? g1 : g0, hi, lo);
+                    // head 2g -> atom g (over the raw chunks just read), head 2g+1 -> atom 2+g
+                    sts128(stg + (hh ? o.out2 : o.in0), hi);
+                    sts128(stg + (hh ? o.out3 : o.in1), lo);
+                }
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
                     bar_arrive(KREADY + 8 * st);
-                    bar_arrive(DREADY + 8 * db);
                     bar_arrive(CEMPTY + 8 * ct);   // after the rows have been used: see release_after_use
                 }
             }
         }
     } else {
-        // ---------------- epilogue: tensor memory -> scaled bf16 -> TMA store ----------------
-        // warp e: head q = e & 3 (tensor-memory lanes 32q + c, c = lane), tokens [32 hf, 32 hf + 32), hf = e >> 2
+        // ---------------- epilogue: tensor memory -> bf16 -> transposed into a TMA store box ----------------
+        // warp e: head q = e & 3 (tensor-memory lanes 32q + c), tokens [32 hf, 32 hf + 32), hf = e >> 2.
+        // The accumulator already carries 1 / (z . phi(q) + eps): the epilogue only converts and moves.
         const int q = w & 3, hf = w >> 2;
-        const int odd = lane & 1;
         const size_t tstride = (size_t)p.H * LCLA_D;   // elements per token
-        unsigned char *ob0 = sm + L::O_OFF + w * 2 * 2048;
+        const uint32_t obs0 = sb + L::O_OFF + w * 2 * L::OBUF;
+        const unsigned char *obp0 = sm + L::O_OFF + w * 2 * L::OBUF;
+        // stmatrix row of this lane: c group m = lane >> 3 (c in [8m, 8m + 8)), token 8j + k, k = lane & 7;
+        // the box is [32 tok][32 c] bf16 with the 64-byte swizzle (16-byte chunk m of row r at m ^ ((r >> 1) & 3))
+        const int smm = lane >> 3, smk = lane & 7;
         int ob = 0;
-        Ring tr = {0, 0u}, dr = {0, 0u};   // TMEM full, 1/den ready
+        Ring tr = {0, 0u};   // TMEM full
         bool ok = true;
         for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
             const int head = HQ * x.hq + q;
             for (int i = 0; i < x.ntile; ++i) {
-                const int tb = tr.idx, db = dr.idx;
-                bool fine = bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag);
-                fine = bar_wait(DREADY + 8 * dr.idx, dr.phase, abort_flag) && fine;
-                if (!__all_sync(ALL, fine)) {
+                const int tb = tr.idx;
+                if (!__all_sync(ALL, bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag))) {
                     ok = false;
                     break;
                 }
                 ring_next<NTM>(tr);
-                ring_next<ND>(dr);
                 tc_after();
                 const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
-                const bool whole = nt == T;
-                uint32_t *obuf = reinterpret_cast<uint32_t *>(ob0 + ob * 2048);
-                if (whole) {
-                    if (lane == 0) bulk_wait_read1();   // this buffer's previous store has read it
-                    __syncwarp();
-                }
-                uint32_t v[32], word[16];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q) + 32 * hf, v);
+                if (lane == 0) bulk_wait_read1();   // this buffer's previous store has read it
+                __syncwarp();
+                uint32_t v[32];
+                const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q) + 32 * hf;
+                tmem_ld16x256_x4x2(ta, ta + (16u << 16), v);
                 tc_before();
                 __syncwarp();
                 if (lane == 0) bar_arrive(TFREE + 8 * tb);   // the accumulator is in registers: free the slot
-                const float4 *iv = reinterpret_cast<const float4 *>(dens + (db * HQ + q) * T + 32 * hf);
-                // own column c for tokens (2m, 2m+1) packed; lane pairs (2i, 2i+1) trade them so that the
-                // even lane holds row 2m's (c, c+1) and the odd lane row 2m+1's
+                // v[16 L + 4 j + i] = D[c = 16 L + lane / 4 + 8 (i >> 1)][tok = 8 j + 2 (lane % 4) + (i & 1)]
+                const uint32_t obs = obs0 + ob * L::OBUF;
 #pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                    const float4 s = iv[j4];
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const uint32_t mine = pack_bf2(__uint_as_float(v[4 * j4 + 2 * k]) * (k ? s.z : s.x),
-                                                       __uint_as_float(v[4 * j4 + 2 * k + 1]) * (k ? s.w : s.y));
-                        const uint32_t other = __shfl_xor_sync(ALL, mine, 1);
-                        word[2 * j4 + k] = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
-                    }
+                for (int j = 0; j < 4; ++j) {
+                    const int tok = 8 * j + smk;
+                    stsm4_trans(obs + tok * 64 + ((smm ^ ((tok >> 1) & 3)) << 4),
+                                pack_bf2(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1])),
+                                pack_bf2(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])),
+                                pack_bf2(__uint_as_float(v[16 + 4 * j]), __uint_as_float(v[16 + 4 * j + 1])),
+                                pack_bf2(__uint_as_float(v[16 + 4 * j + 2]), __uint_as_float(v[16 + 4 * j + 3])));
                 }
-                __syncwarp();
-                if (lane == 0) bar_arrive(DFREE + 8 * db);   // 1/den values consumed above
-                // word[j] is row 2j + odd of this warp's 32 tokens; branch once, outside the arithmetic
-                if (whole) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) obuf[(2 * j + odd) * 16 + (lane >> 1)] = word[j];
+                if (nt == T) {
                     fence_async_smem();
                     __syncwarp();
-                    if (lane == 0) {
-                        if (head < p.H) tma_store3(&mo, s32(obuf), LCLA_D * head, t + 32 * hf, x.b);
-                        bulk_commit();   // one group per buffer use keeps the read-wait accounting exact
-                    }
-                    ob ^= 1;
-                } else if (head < p.H) {
-                    uint32_t *gout = reinterpret_cast<uint32_t *>(out + ((size_t)x.b * p.N + t + 32 * hf) * tstride +
-                                                                  (size_t)head * LCLA_D + (lane & ~1));
+                    if (lane == 0 && head < p.H) tma_store3(&mo, obs, LCLA_D * head, t + 32 * hf, x.b);
+                } else {   // ragged tile: lane = token, its 64-byte row back from the box to global memory
+                    __syncwarp();
+                    const int tok = lane;
+                    if (head < p.H && 32 * hf + tok < nt) {
+                        const unsigned char *row = obp0 + ob * L::OBUF + tok * 64;
+                        uint4 *g = reinterpret_cast<uint4 *>(out + ((size_t)x.b * p.N + t + 32 * hf + tok) * tstride +
+                                                             (size_t)head * LCLA_D);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int tok = 2 * j + odd;
-                        if (32 * hf + tok < nt) gout[(size_t)tok * (tstride / 2)] = word[j];
+                        for (int m = 0; m < 4; ++m) g[m] = lds128(row + ((m ^ ((tok >> 1) & 3)) << 4));
                     }
+                    __syncwarp();
                 }
+                if (lane == 0) bulk_commit();   // one group per buffer use keeps the read-wait accounting exact
+                ob ^= 1;
             }
         }
         if (lane == 0) bulk_wait_all();
