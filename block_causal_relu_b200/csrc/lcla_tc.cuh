@@ -229,6 +229,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t ta, uint32_t *r)
         : "memory");
 }
 
+// 32 lanes x 16 columns, as tmem_ld32.
+__device__ __forceinline__ void tmem_ld16(uint32_t ta, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(ta)
+        : "memory");
+}
+
 // Two 16-lane halves of a warp's lane quarter, 32 columns each (shape 16x256b,
 // four repeats): thread t gets, for half L (tensor-memory lanes ta + 16L + ...),
 // r[16L + 4j + i] = lane t/4 + 8(i >> 1), column 8j + 2(t % 4) + (i & 1) --
@@ -273,6 +285,7 @@ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major)
 
 __device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t *>(&v); }
 __device__ __forceinline__ uint32_t pack_bf2(float a, float b) { return bf2_bits(__floats2bfloat162_rn(a, b)); }
+
 
 // ReLU on two packed bf16 (NaN passes through).
 __device__ __forceinline__ uint32_t relu2(uint32_t w)
@@ -331,29 +344,7 @@ __device__ __forceinline__ void store_quarter_hi_lo(unsigned char *tile, int r, 
 // chunks it has read -- and head 2b+1's into the fresh atom 2+b.
 __device__ __forceinline__ int atom_of(int h) { return (h >> 1) + 2 * (h & 1); }
 
-// Prologue thread (warp pw in 0..7, lane): token row r = 8 pw + (lane >> 2),
-// quarter f = lane & 3.  Inside a 128-byte-swizzled [64][128 B] box, chunk f
-// of row r is at `a`, chunk 4 + f at `b`; eight consecutive rows per warp keep
-// every 128-bit shared access free of bank conflicts.  `tab` is the row's
-// quarter f inside a [64][16] fp32 rotary box (64-byte swizzle).
-struct ProOffs {
-    int r, f, a, b, tab;
-};
-__device__ __forceinline__ ProOffs pro_offsets(int pw, int lane)
-{
-    ProOffs o;
-    o.f = lane & 3;
-    o.r = 8 * pw + (lane >> 2);
-    const int sw = o.r & 7;
-    o.a = o.r * 128 + ((o.f ^ sw) << 4);
-    o.b = o.r * 128 + (((4 + o.f) ^ sw) << 4);
-    o.tab = o.r * 64 + ((o.f ^ ((o.r >> 1) & 3)) << 4);
-    return o;
-}
-// Raw input quarter of head h in a stage (box h >> 1, chunk f or 4 + f).
-__device__ __forceinline__ int raw_off(const ProOffs &o, int h) { return (h >> 1) * 8192 + ((h & 1) ? o.b : o.a); }
-
-// Pass C's prologue has 16 warps, a thread doing one token quarter of one
+// Both prologues have 16 warps, a thread doing one token quarter of one
 // head pair g = lane & 1 (heads 2g, 2g+1), quarter f = (lane >> 1) & 3, on
 // one of the warp's four rows {8k, 8k+1, 8k+4, 8k+5} + 2 (pw & 1), k = pw >> 1
 // (bank-conflict free; the two pairs' identical rotary reads are one
@@ -414,14 +405,14 @@ constexpr int NT = 3;             // rotary-table ring slots ([cos 4 KB | sin 4 
 constexpr int CTRL_BYTES = 512;   // control block: mbarriers (8 B each), tensor-memory slot, abort flag
 constexpr int SMEM_MAX = 232448;  // dynamic shared memory a CTA may opt in to
 constexpr int TAB_BYTES = 8192;
-constexpr int NPRO = 8;           // pass A prologue warps
-constexpr int NPRO_C = 16;        // pass C prologue warps
+constexpr int NPRO = 16;          // prologue warps (both passes)
 
 // Producer: per tile, TMA loads of the quad's input boxes into the stage ring
-// (two [64 token][2 heads] boxes per tensor map, heads past H read as zeros)
+// (NBOX boxes of [64 token][4 / NBOX heads] per tensor map, heads past H read
+// as zeros)
 // and of the tile's rotary rows into the table ring.  On abort, waits
 // (bounded) for the loads already issued before returning.
-template <int S, int STAGE, int NMAP>
+template <int S, int STAGE, int NMAP, int NBOX>
 __device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t sb, uint32_t tab0,
                                         uint32_t FULL, uint32_t EMPTY, uint32_t CFULL, uint32_t CEMPTY,
                                         const CUtensorMap *const (&maps)[NMAP], const int (&offs)[NMAP],
@@ -440,12 +431,13 @@ __device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t 
                 break;
             }
             const uint32_t base = sb + er.idx * STAGE, fb = FULL + 8 * er.idx;
-            bar_expect_tx(fb, (uint32_t)(NMAP * 2 * 8192));
+            bar_expect_tx(fb, (uint32_t)(NMAP * HQ * LCLA_D * T * 2));
 #pragma unroll
-            for (int m = 0; m < NMAP; ++m) {
-                tma_load3(base + offs[m], maps[m], fb, x0, t, x.b);
-                tma_load3(base + offs[m] + 8192, maps[m], fb, x0 + 2 * LCLA_D, t, x.b);
-            }
+            for (int m = 0; m < NMAP; ++m)
+#pragma unroll
+                for (int j = 0; j < NBOX; ++j)   // box j: heads [j HQ / NBOX, (j + 1) HQ / NBOX) of the quad
+                    tma_load3(base + offs[m] + j * (HQ * LCLA_D * T * 2 / NBOX), maps[m], fb,
+                              x0 + j * (HQ * LCLA_D / NBOX), t, x.b);
             ring_next<S>(er);
             ++issued;
             if (!bar_wait(CEMPTY + 8 * cr.idx, cr.phase, abort_flag)) {
@@ -476,19 +468,25 @@ struct LayA {
     // stage: [k~ operand, 4 atoms of [64 tok][hi 32 | lo 32] (raw k lands in atoms 0-1) | v, 2 boxes]
     static constexpr int K_OFF = 0, V_OFF = 32768, STAGE = 49152;
     static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
-    static constexpr int Z_OFF = C_OFF + NT * TAB_BYTES;            // key-sum parts [8 warps][4 f][4 heads][8]
-    static constexpr int Z_BYTES = NPRO * 4 * HQ * 8 * 4;
+    static constexpr int Z_OFF = C_OFF + NT * TAB_BYTES;            // key-sum parts [16 warps][2 g][4 f][2 heads][8]
+    static constexpr int Z_BYTES = NPRO * 2 * 4 * 2 * 8 * 4;
     static constexpr int CTRL = Z_OFF + Z_BYTES;                    // mbarriers, tensor-memory slot, abort flag
     static constexpr int BYTES = CTRL + CTRL_BYTES + 1024;          // + worst-case 1024-byte alignment pad
-    static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
-    static constexpr int NTHREADS = 448;                            // drain 0-3, producer 4, MMA 5, prologue 6-13
+    static constexpr int NTM = 2;                                   // tensor-memory accumulators (256 columns each)
+    // tiles summed in one accumulator before the drain takes it: tensor-core
+    // accumulation over whole segments (~100 K-steps) was measured to lose
+    // about 1.6e-5 of max |S| against fp32 sums; 4 tiles (16 K-steps) keep the
+    // state well inside 1e-5, the rest is summed in registers
+    static constexpr int CHUNK = 4;
+    static constexpr int NTHREADS = 704;                            // drain 0-3, producer 4, MMA 5, prologue 6-21
     static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6;
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 1, 1);
     static constexpr int TMEM_COLS = NTM * 256;
-    static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 2;
+    static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 3;
 };
 static_assert(LayA::BYTES <= SMEM_MAX, "pass A shared memory");
 static_assert(8 * LayA::NBARS + 8 <= CTRL_BYTES, "pass A control block");
+static_assert(LayA::NTHREADS / 32 - LayA::W_PRO0 == NPRO, "pass A prologue warps: barrier counts use NPRO");
 
 __global__ void __launch_bounds__(LayA::NTHREADS, 1)
 pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
@@ -504,7 +502,7 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
     const uint32_t sb = raw + pad;
     const uint32_t FULL = sb + L::CTRL, EMPTY = FULL + 8 * S, KREADY = EMPTY + 8 * S, CFULL = KREADY + 8 * S,
                    CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
-                   ZREADY = TFREE + 8 * NTM, ZFREE = ZREADY + 8;
+                   ZREADY = TFREE + 8 * NTM, ZFREE = ZREADY + 8, MDONE = ZFREE + 8;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * L::NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     float *zbuf = reinterpret_cast<float *>(sm + L::Z_OFF);
@@ -528,6 +526,7 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
         }
         bar_init(ZREADY, NPRO);
         bar_init(ZFREE, 4);
+        bar_init(MDONE, 1);
         *abort_flag = 0;
         bar_fence_init();
     }
@@ -545,23 +544,23 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
         if (lane == 0) {
             const CUtensorMap *const maps[2] = {&mk, &mv};
             const int offs[2] = {L::K_OFF, L::V_OFF};
-            produce<S, L::STAGE, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc, &ms,
-                                    abort_flag);
+            produce<S, L::STAGE, 2, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc, &ms,
+                                       abort_flag);
         }
     } else if (w == L::W_MMA) {
-        // ---------------- MMA issuer ----------------
+        // ---------------- MMA issuer: one accumulator per chunk of CHUNK tiles ----------------
         if (lane == 0) {
-            Ring sr = {0, 0u}, tr = {0, 1u};   // stage (k~ ready), TMEM free
+            Ring sr = {0, 0u}, tr = {0, 1u};   // stage (k~ ready), accumulator free
             const uint64_t vdesc0 = desc_sw128(sb + L::V_OFF, 8192, 1024);
             const uint64_t kdesc0 = desc_sw128(sb + L::K_OFF, 8192, 1024);
-            int issued = 0, last_tb = 0;
-            uint32_t last_phase = 0;
+            int issued = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const Unit x = unit_at(p, u);
                 for (int i = 0; i < x.ntile; ++i) {
-                    if (!bar_wait(KREADY + 8 * sr.idx, sr.phase, abort_flag) ||
-                        !bar_wait(TFREE + 8 * tr.idx, tr.phase, abort_flag)) {
+                    const int ic = i % L::CHUNK;
+                    if ((ic == 0 && !bar_wait(TFREE + 8 * tr.idx, tr.phase, abort_flag)) ||
+                        !bar_wait(KREADY + 8 * sr.idx, sr.phase, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -570,32 +569,36 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                     // descriptor start addresses advance in 16-byte units; 16 tokens = 2048 B
                     const uint64_t so = (uint64_t)((sr.idx * L::STAGE) >> 4);
 #pragma unroll
-                    for (int j = 0; j < T / 16; ++j)   // v^T (x) [k~hi | k~lo]
-                        mma_bf16(d, vdesc0 + so + 128 * j, kdesc0 + so + 128 * j, L::IDESC, j > 0);
-                    mma_commit(TFULL + 8 * tr.idx);
+                    for (int j = 0; j < T / 16; ++j)   // D (+)= v^T (x) [k~hi | k~lo]
+                        mma_bf16(d, vdesc0 + so + 128 * j, kdesc0 + so + 128 * j, L::IDESC, (ic | j) != 0);
                     mma_commit(EMPTY + 8 * sr.idx);
-                    last_tb = tr.idx;
-                    last_phase = tr.phase ^ 1u;   // TFULL runs one phase behind TFREE's producer-side parity
                     ring_next<S>(sr);
-                    ring_next<NTM>(tr);
                     ++issued;
+                    if (ic == L::CHUNK - 1 || i == x.ntile - 1) {   // chunk complete: hand it to the drain
+                        mma_commit(TFULL + 8 * tr.idx);
+                        ring_next<NTM>(tr);
+                    }
                 }
             }
-            if (!ok && issued > 0) bar_wait_quiet(TFULL + 8 * last_tb, last_phase);
+            if (!ok && issued > 0) {   // let the MMAs in flight finish before the memory is released
+                mma_commit(MDONE);
+                bar_wait_quiet(MDONE, 0);
+            }
         }
     } else if (w >= L::W_PRO0) {
         // ---------------- prologue: phi, key sum, rotary, hi/lo split ----------------
         const int pw = w - L::W_PRO0;
-        const ProOffs o = pro_offsets(pw, lane);
+        const PairOffs o = pair_offsets(pw, lane);
         Ring fr = {0, 0u}, cr = {0, 0u}, zr = {0, 1u};   // stage full, table full, key-sum buffer free (1 slot)
         bool ok = true;
         for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
-            float zacc[HQ][8];
+            if (x.ntile == 0) continue;
+            float zacc[2][8];   // z[8f, 8f+8) of heads 2g, 2g+1 over this thread's rows
 #pragma unroll
-            for (int h = 0; h < HQ; ++h)
+            for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) zacc[h][j] = 0.f;
+                for (int j = 0; j < 8; ++j) zacc[hh][j] = 0.f;
             for (int i = 0; i < x.ntile; ++i) {
                 const int st = fr.idx, ct = cr.idx;
                 bool fine = bar_wait(FULL + 8 * fr.idx, fr.phase, abort_flag);
@@ -610,26 +613,28 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                 const unsigned char *tab = sm + L::C_OFF + ct * TAB_BYTES;
                 const float4 c4 = ldsf4(tab + o.tab);
                 const float4 s4 = ldsf4(tab + TAB_BYTES / 2 + o.tab);
-                uint4 kr[HQ];
-#pragma unroll
-                for (int h = 0; h < HQ; ++h) kr[h] = lds128(stg + L::K_OFF + raw_off(o, h));
+                const uint4 k0 = lds128(stg + L::K_OFF + o.in0);   // head 2g
+                const uint4 k1 = lds128(stg + L::K_OFF + o.in1);   // head 2g+1
                 const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
                 const bool valid = o.r < nt;
 #pragma unroll
-                for (int h = 0; h < HQ; ++h) {
-                    uint32_t fw[4] = {kr[h].x, kr[h].y, kr[h].z, kr[h].w}, hi[4], lo[4];
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint4 kv = hh ? k1 : k0;
+                    uint32_t fw[4] = {kv.x, kv.y, kv.z, kv.w}, hi[4], lo[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         fw[j] = valid ? relu2(fw[j]) : 0u;
-                        zacc[h][2 * j] += bf_lo(fw[j]);
-                        zacc[h][2 * j + 1] += bf_hi(fw[j]);
+                        zacc[hh][2 * j] += bf_lo(fw[j]);
+                        zacc[hh][2 * j + 1] += bf_hi(fw[j]);
                     }
                     rope_split4(fw, c4, s4, hi, lo);
-                    unsigned char *atom = stg + L::K_OFF + atom_of(h) * 8192;
-                    sts128(atom + o.a, hi);
-                    sts128(atom + o.b, lo);
-                    if (!valid)   // rows past the segment belong to another unit: zero this quarter of v
-                        *reinterpret_cast<uint4 *>(stg + L::V_OFF + raw_off(o, h)) = make_uint4(0u, 0u, 0u, 0u);
+                    // head 2g -> atom g (over the raw chunks just read), head 2g+1 -> atom 2+g
+                    sts128(stg + L::K_OFF + (hh ? o.out2 : o.in0), hi);
+                    sts128(stg + L::K_OFF + (hh ? o.out3 : o.in1), lo);
+                }
+                if (!valid) {   // rows past the segment belong to another unit: zero this quarter of v
+                    *reinterpret_cast<uint4 *>(stg + L::V_OFF + o.in0) = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4 *>(stg + L::V_OFF + o.in1) = make_uint4(0u, 0u, 0u, 0u);
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -639,44 +644,50 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                 }
             }
             if (!ok) break;
-            // unit done: this warp's key-sum parts (its 8 token rows) for the drain
+            // unit done: sum this warp's four rows (lane bits 3-4) and hand the parts to the drain
 #pragma unroll
-            for (int h = 0; h < HQ; ++h)
+            for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-#pragma unroll
-                    for (int m = 4; m <= 16; m <<= 1) zacc[h][j] += __shfl_xor_sync(ALL, zacc[h][j], m);
+                for (int j = 0; j < 8; ++j) {
+                    zacc[hh][j] += __shfl_xor_sync(ALL, zacc[hh][j], 8);
+                    zacc[hh][j] += __shfl_xor_sync(ALL, zacc[hh][j], 16);
+                }
             if (!__all_sync(ALL, bar_wait(ZFREE, zr.phase, abort_flag))) {
                 ok = false;
                 break;
             }
             ring_next<1>(zr);
-            if (lane < 4) {   // lane = quarter f
-                float4 *dst = reinterpret_cast<float4 *>(zbuf + (pw * 4 + o.f) * (HQ * 8));
+            if (lane < 8) {   // lane = (g, f)
+                float4 *dst = reinterpret_cast<float4 *>(zbuf + ((pw * 2 + o.g) * 4 + o.f) * 16);
 #pragma unroll
-                for (int h = 0; h < HQ; ++h) {
-                    dst[2 * h] = make_float4(zacc[h][0], zacc[h][1], zacc[h][2], zacc[h][3]);
-                    dst[2 * h + 1] = make_float4(zacc[h][4], zacc[h][5], zacc[h][6], zacc[h][7]);
+                for (int hh = 0; hh < 2; ++hh) {
+                    dst[2 * hh] = make_float4(zacc[hh][0], zacc[hh][1], zacc[hh][2], zacc[hh][3]);
+                    dst[2 * hh + 1] = make_float4(zacc[hh][4], zacc[hh][5], zacc[hh][6], zacc[hh][7]);
                 }
             }
             __syncwarp();
             if (lane == 0) bar_arrive(ZREADY);
         }
     } else {
-        // ---------------- drain: tensor memory -> registers -> partial states ----------------
+        // ---------------- drain: chunk accumulators -> partial state of the unit ----------------
         const int q = w;   // head of the quad; tensor-memory lanes 32q + c
         const float nanv = __int_as_float(0x7fc00000);
-        Ring tr = {0, 0u}, zr = {0, 0u};   // TMEM full, key sum ready (1 slot)
+        Ring tr = {0, 0u}, zr = {0, 0u};   // accumulator full, key sum ready (1 slot)
         bool ok = true;
         for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
             const int head = HQ * x.hq + q;
             float *dst = part + (((size_t)x.s * p.B + x.b) * p.H + (head < p.H ? head : 0)) * LCLA_SZ;
+            if (ok && x.ntile == 0) {   // empty segment: nothing was loaded or summed
+                if (head < p.H)
+                    for (int e = lane; e < LCLA_SZ; e += 32) dst[e] = 0.f;
+                continue;
+            }
             if (ok) {
-                float sacc[32];
+                float sacc[32];   // S row c = lane, summed over the unit's chunks
 #pragma unroll
                 for (int j = 0; j < 32; ++j) sacc[j] = 0.f;
-                for (int i = 0; i < x.ntile; ++i) {
+                for (int i = 0; i < x.ntile; i += L::CHUNK) {
                     const int tb = tr.idx;
                     if (!__all_sync(ALL, bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag))) {
                         ok = false;
@@ -686,35 +697,32 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                     tc_after();
                     const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q);
 #pragma unroll
-                    for (int part_ = 0; part_ < 2; ++part_) {   // hi columns, then lo columns
-                        uint32_t v[32];
-                        tmem_ld32(ta + 32 * part_, v);
+                    for (int c4 = 0; c4 < 4; ++c4) {   // k~hi columns e = 0-15, 16-31, then k~lo
+                        uint32_t v[16];
+                        tmem_ld16(ta + 16 * c4, v);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) sacc[j] += __uint_as_float(v[j]);
+                        for (int j = 0; j < 16; ++j) sacc[16 * (c4 & 1) + j] += __uint_as_float(v[j]);
                     }
                     tc_before();
                     __syncwarp();
                     if (lane == 0) bar_arrive(TFREE + 8 * tb);
                 }
+                if (ok && !__all_sync(ALL, bar_wait(ZREADY, zr.phase, abort_flag))) ok = false;
                 if (ok) {
-                    if (!__all_sync(ALL, bar_wait(ZREADY, zr.phase, abort_flag))) {
-                        ok = false;
-                    } else {
-                        ring_next<1>(zr);
-                        // z[e], e = lane: quarter e >> 3, element e & 7 of head q, over the prologue warps
-                        const float *zp = zbuf + (lane >> 3) * (HQ * 8) + q * 8 + (lane & 7);
-                        float zs = 0.f;
+                    ring_next<1>(zr);
+                    // z[e], e = lane: head q = 2g + hh, quarter f = e >> 3, over the prologue warps
+                    const float *zp = zbuf + ((q >> 1) * 4 + (lane >> 3)) * 16 + (q & 1) * 8 + (lane & 7);
+                    float zs = 0.f;
 #pragma unroll
-                        for (int pw = 0; pw < NPRO; ++pw) zs += zp[pw * 4 * HQ * 8];
-                        __syncwarp();
-                        if (lane == 0) bar_arrive(ZFREE);
-                        if (head < p.H) {   // row c = lane of S, then z
-                            float4 *row = reinterpret_cast<float4 *>(dst + lane * LCLA_D);
+                    for (int pw = 0; pw < NPRO; ++pw) zs += zp[pw * 2 * 4 * 16];
+                    __syncwarp();
+                    if (lane == 0) bar_arrive(ZFREE);
+                    if (head < p.H) {   // row c = lane of S, then z
+                        float4 *row = reinterpret_cast<float4 *>(dst + lane * LCLA_D);
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                row[j] = make_float4(sacc[4 * j], sacc[4 * j + 1], sacc[4 * j + 2], sacc[4 * j + 3]);
-                            dst[LCLA_D * LCLA_D + lane] = zs;
-                        }
+                        for (int j = 0; j < 8; ++j)
+                            row[j] = make_float4(sacc[4 * j], sacc[4 * j + 1], sacc[4 * j + 2], sacc[4 * j + 3]);
+                        dst[LCLA_D * LCLA_D + lane] = zs;
                     }
                 }
             }
@@ -755,6 +763,7 @@ struct LayC {
 };
 static_assert(LayC::BYTES <= SMEM_MAX, "pass C shared memory");
 static_assert(8 * LayC::NBARS + 8 <= CTRL_BYTES, "pass C control block");
+static_assert(LayC::NTHREADS / 32 - LayC::W_PRO0 == NPRO, "pass C prologue warps: barrier counts use NPRO");
 static_assert(LayC::O_OFF % 1024 == 0 && LayC::OBUF % 512 == 0, "64-byte-swizzled output boxes need 512-byte alignment");
 
 __global__ void __launch_bounds__(LayC::NTHREADS, 1)
@@ -782,11 +791,11 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         for (int i = 0; i < S; ++i) {
             bar_init(FULL + 8 * i, 1);
             bar_init(EMPTY + 8 * i, 1);
-            bar_init(KREADY + 8 * i, NPRO_C);
+            bar_init(KREADY + 8 * i, NPRO);
         }
         for (int i = 0; i < NT; ++i) {
             bar_init(CFULL + 8 * i, 1);
-            bar_init(CEMPTY + 8 * i, NPRO_C);
+            bar_init(CEMPTY + 8 * i, NPRO);
         }
         for (int i = 0; i < NTM; ++i) {
             bar_init(TFULL + 8 * i, 1);
@@ -810,8 +819,8 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         if (lane == 0) {
             const CUtensorMap *const maps[1] = {&mq};
             const int offs[1] = {0};
-            produce<S, L::STAGE, 1>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc, &ms,
-                                    abort_flag);
+            produce<S, L::STAGE, 1, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc, &ms,
+                                       abort_flag);
         }
     } else if (w == L::W_MMA) {
         // ---------------- MMA issuer ----------------
