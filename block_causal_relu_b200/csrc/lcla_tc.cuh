@@ -345,21 +345,25 @@ __device__ __forceinline__ void store_quarter_hi_lo(unsigned char *tile, int r, 
 __device__ __forceinline__ int atom_of(int h) { return (h >> 1) + 2 * (h & 1); }
 
 // Both prologues have 16 warps, a thread doing one token quarter of one
-// head pair g = lane & 1 (heads 2g, 2g+1), quarter f = (lane >> 1) & 3, on
-// one of the warp's four rows {8k, 8k+1, 8k+4, 8k+5} + 2 (pw & 1), k = pw >> 1
-// (bank-conflict free; the two pairs' identical rotary reads are one
-// broadcast).  in0 / in1: the raw chunks of heads 2g / 2g+1 in box g, which
-// are also atom g's hi / lo chunks; out2 / out3: atom 2+g's hi / lo chunks.
+// head pair g = (lane >> 3) & 1 (heads 2g, 2g+1), quarter f = lane & 3, on one
+// of four rows of the 8-row block k = pw >> 1: {0, 5, 1, 4} for even pw,
+// {2, 7, 3, 6} for odd pw, picked by lane bits 2 and 4.  A 128-bit access is
+// served eight lanes at a time, and each group of eight lanes here holds two
+// rows whose 128-byte swizzles differ in bit 2 and whose parities differ: its
+// eight chunks of the stage (128-byte swizzle) and of the rotary rows (64-byte
+// swizzle) fall on eight different 16-byte bank groups.  in0 / in1: the raw
+// chunks of heads 2g / 2g+1 in box g, which are also atom g's hi / lo chunks;
+// out2 / out3: atom 2+g's hi / lo chunks.
 struct PairOffs {
     int g, f, r, in0, in1, out2, out3, tab;
 };
 __device__ __forceinline__ PairOffs pair_offsets(int pw, int lane)
 {
     PairOffs o;
-    o.g = lane & 1;
-    o.f = (lane >> 1) & 3;
-    const int rr = lane >> 3;
-    o.r = 8 * (pw >> 1) + 2 * (pw & 1) + (rr & 1) + 4 * (rr >> 1);
+    o.f = lane & 3;
+    o.g = (lane >> 3) & 1;
+    const int pr = ((lane >> 4) << 1) | ((lane >> 2) & 1);   // pair lane >> 4, member (lane >> 2) & 1
+    o.r = 8 * (pw >> 1) + 2 * (pw & 1) + (pr >> 1) + (pr & 1) * (5 - 2 * (pr >> 1));
     const int sw = o.r & 7, row = o.r * 128;
     o.in0 = o.g * 8192 + row + ((o.f ^ sw) << 4);
     o.in1 = o.g * 8192 + row + (((4 + o.f) ^ sw) << 4);
@@ -644,12 +648,12 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                 }
             }
             if (!ok) break;
-            // unit done: sum this warp's four rows (lane bits 3-4) and hand the parts to the drain
+            // unit done: sum this warp's four rows (lane bits 2 and 4) and hand the parts to the drain
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    zacc[hh][j] += __shfl_xor_sync(ALL, zacc[hh][j], 8);
+                    zacc[hh][j] += __shfl_xor_sync(ALL, zacc[hh][j], 4);
                     zacc[hh][j] += __shfl_xor_sync(ALL, zacc[hh][j], 16);
                 }
             if (!__all_sync(ALL, bar_wait(ZFREE, zr.phase, abort_flag))) {
@@ -657,7 +661,7 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                 break;
             }
             ring_next<1>(zr);
-            if (lane < 8) {   // lane = (g, f)
+            if ((lane & 0x14) == 0) {   // lanes 0-3 (g = 0) and 8-11 (g = 1), quarter f = lane & 3
                 float4 *dst = reinterpret_cast<float4 *>(zbuf + ((pw * 2 + o.g) * 4 + o.f) * 16);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -944,16 +948,16 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     }
                     den[hh] = dd;
                 }
-                // z . phi(q) of each head over the token's four quarters (lane bits 1-2)
+                // z . phi(q) of each head over the token's four quarters (lane bits 0-1)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
+                    den[hh] += __shfl_xor_sync(ALL, den[hh], 1);
                     den[hh] += __shfl_xor_sync(ALL, den[hh], 2);
-                    den[hh] += __shfl_xor_sync(ALL, den[hh], 4);
                 }
                 // 1 / (z . phi(q) + eps): quarters with even f divide for head 2g, odd f for head 2g+1,
-                // and trade the results (lane bit 1 is bit 0 of f)
+                // and trade the results (lane bit 0 is bit 0 of f)
                 const float mine = 1.0f / (((o.f & 1) ? den[1] : den[0]) + eps);
-                const float theirs = __shfl_xor_sync(ALL, mine, 2);
+                const float theirs = __shfl_xor_sync(ALL, mine, 1);
                 const float g0 = (o.f & 1) ? theirs : mine, g1 = (o.f & 1) ? mine : theirs;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
