@@ -360,9 +360,10 @@ def main():
     bytes_a = 2 * tok_bytes + tab_bytes + nseg * sl
     bytes_c = 2 * tok_bytes + tab_bytes + npref * sl
     bytes_s = nseg * sl + npref * sl + sl
-    # the grouped scan serves plans with at most 256 prefix groups (blocks, or segments in chunk mode)
+    # the grouped scan serves plans with at most 256 prefix groups (blocks, or segments in chunk mode);
+    # larger plans scan in chunks with two kernels, timed together
     scan_name = "scan_states_grouped" if (plan["segments"] if plan["chunk_mode"] else plan["prefixes"]) <= 256 \
-        else "scan_states"
+        else "scan_chunk_totals+scan_chunk_prefix"
     if plan["tensor_cores"]:
         name_a, name_c = "pass_a_tc", "pass_c_tc"
     else:

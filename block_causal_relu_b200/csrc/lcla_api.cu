@@ -48,7 +48,7 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
     if (N == 0) return p;
     p.nb = (int)(((long long)N + L - 1) / L);
     const long long units = (long long)p.ngroups * B;
-    if (L > LCLA_T) {
+    if (L >= LCLA_T) {
         p.chunk = 0;
         p.tc = dtype == LCLA_BF16;
         p.T = p.tc ? LCLA_TC_T : LCLA_T;
@@ -96,10 +96,18 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype)
         p.nseg = (int)((ntiles + tps - 1) / tps);
         p.npref = p.nseg;
     }
+    // the scan runs in one pass for up to SCANG_MAX_GROUPS groups (blocks, or segments in chunk mode);
+    // beyond that in chunks of SCAN_CHUNK_GROUPS whole groups, whose totals it keeps in the workspace
+    const int scan_groups = p.chunk ? p.nseg : p.nb;
+    if (scan_groups > lcla::SCANG_MAX_GROUPS) {
+        p.scs = lcla::SCAN_CHUNK_GROUPS * (p.chunk ? 1 : p.nsb);
+        p.nch = (p.nseg + p.scs - 1) / p.scs;
+    }
     const size_t slice = (size_t)B * H * LCLA_SZ * sizeof(float);
     p.part_off = kAlign;
     p.pref_off = p.part_off + round_up((size_t)p.nseg * slice);
-    p.ws_bytes = p.pref_off + round_up((size_t)p.npref * slice);
+    p.ctot_off = p.pref_off + round_up((size_t)p.npref * slice);
+    p.ws_bytes = p.ctot_off + (p.nch ? round_up((size_t)(p.nch + 1) * slice) : 0);
     return p;
 }
 
@@ -143,10 +151,10 @@ unsigned scan_blocks(const LclaPlan &p)
 // Partials -> prefixes: the grouped two-phase scan when its group sums fit in
 // shared memory, else the one-thread-per-column serial scan.
 void launch_scan(const LclaPlan &p, const float *part, float *pref, const float *state_in, float *state_out,
-                 cudaStream_t st)
+                 unsigned char *ws, cudaStream_t st)
 {
-    const int ngroups = p.chunk ? p.nseg : p.nb;
-    if (ngroups <= lcla::SCANG_MAX_GROUPS) {
+    if (p.nch == 0) {
+        const int ngroups = p.chunk ? p.nseg : p.nb;
         const size_t n4 = (size_t)p.B * p.H * (LCLA_SZ / lcla::SCAN_VEC);
         const int smem = ngroups * 32 * 16;
         if (smem > 48 * 1024)
@@ -154,8 +162,11 @@ void launch_scan(const LclaPlan &p, const float *part, float *pref, const float 
         launch_pdl(lcla::scan_states_grouped, dim3((unsigned)((n4 + 31) / 32)), dim3(32 * lcla::SCANG_WARPS),
                    (size_t)smem, st, p, part, pref, state_in, state_out);
     } else {
-        launch_pdl(lcla::scan_states, dim3(scan_blocks(p)), dim3(lcla::SCAN_THREADS), 0, st, p, part, pref,
-                   state_in, state_out);
+        float *ctot = reinterpret_cast<float *>(ws + p.ctot_off);
+        const dim3 grid(scan_blocks(p), (unsigned)p.nch);
+        launch_pdl(lcla::scan_chunk_totals, grid, dim3(lcla::SCAN_THREADS), 0, st, p, part, state_in, ctot);
+        launch_pdl(lcla::scan_chunk_prefix, grid, dim3(lcla::SCAN_THREADS), 0, st, p, part, (const float *)ctot,
+                   pref, state_out);
     }
 }
 
@@ -246,7 +257,7 @@ bool launch_tc(const void *q, const void *k, const void *v, const float *rc, con
     lcla::tc::pass_a_tc<<<grid, lcla::tc::LayA::NTHREADS, lcla::tc::LayA::BYTES, st>>>(mk, mv, mc, ms, p, part,
                                                                                        status);
     if (ev) cudaEventRecord(ev[1], st);
-    launch_scan(p, part, pref, state_in, state_out, st);
+    launch_scan(p, part, pref, state_in, state_out, ws, st);
     if (ev) cudaEventRecord(ev[2], st);
     launch_pdl(lcla::tc::pass_c_tc, grid, dim3(lcla::tc::LayC::NTHREADS), lcla::tc::LayC::BYTES, st, mq, mc, ms, mo, p,
                (const float *)pref, eps, (__nv_bfloat16 *)out, status);
@@ -272,7 +283,7 @@ int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const 
     lcla::pass_a_ffma<Tin><<<grid, 256, smem_a, st>>>(k, v, rc, rs, p, part);
 
     if (ev) cudaEventRecord(ev[1], st);
-    launch_scan(p, part, pref, state_in, state_out, st);
+    launch_scan(p, part, pref, state_in, state_out, ws, st);
     if (ev) cudaEventRecord(ev[2], st);
 
     if (!p.chunk) {

@@ -5,9 +5,9 @@
 // Attention for Long Video Generation with Sana", section "Chunk-Wise
 // Causality").  The kernels cut the sequence into *segments*, contiguous token
 // ranges that either
-//   - lie inside one block (block mode, block_len > LCLA_T): every token of
+//   - lie inside one block (block mode, block_len >= LCLA_T): every token of
 //     the segment uses the inclusive prefix state of its block; or
-//   - hold whole blocks only (chunk mode, block_len <= LCLA_T): tiles of
+//   - hold whole blocks only (chunk mode, block_len < LCLA_T): tiles of
 //     T = (LCLA_T / block_len) * block_len tokens, where a token uses the
 //     exclusive prefix at the tile start plus a masked term inside the tile.
 // Pass A reduces each segment to a partial state, the scan turns partials
@@ -37,7 +37,8 @@ struct LclaPlan {
     int npref;     // prefix entries: block mode nb, chunk mode nseg
     int ngroups;   // head groups of LCLA_HG heads (CUDA-core grid)
     int nquads;    // head groups of LCLA_TC_HQ heads (tensor-core work units)
-    size_t part_off, pref_off, ws_bytes;   // workspace layout (bytes)
+    int scs, nch;  // scan over many groups: segments per scan chunk (whole groups) and chunks; nch = 0: one pass
+    size_t part_off, pref_off, ctot_off, ws_bytes;   // workspace layout (bytes)
 };
 
 struct LclaSeg {

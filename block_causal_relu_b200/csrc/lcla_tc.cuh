@@ -174,6 +174,45 @@ __device__ __forceinline__ void tma_load2(uint32_t dst, const CUtensorMap *map, 
         ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(x), "r"(y)
         : "memory");
 }
+// L2 eviction policies: streamed tensors (read or written once) go first, the
+// small partial and prefix states that the next kernel reads back stay.
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void tma_load3_hint(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y, int z,
+                                               uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%3, %4, %5}], [%2], %6;"
+        ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(x), "r"(y), "r"(z), "l"(pol)
+        : "memory");
+}
+__device__ __forceinline__ void tma_store3_hint(const CUtensorMap *map, uint32_t src, int x, int y, int z, uint64_t pol)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;"
+                 ::"l"((uint64_t)map), "r"(src), "r"(x), "r"(y), "r"(z), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_v4_hint(float4 *p, float4 v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;"
+                 ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_f32_hint(float *p, float v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
 __device__ __forceinline__ void tma_store3(const CUtensorMap *map, uint32_t src, int x, int y, int z)
 {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
@@ -425,6 +464,7 @@ __device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t 
     Ring er = {0, 1u}, cr = {0, 1u};
     int issued = 0, tissued = 0;
     bool ok = true;
+    const uint64_t stream_pol = policy_evict_first();
     for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
         const Unit x = unit_at(p, u);
         const int x0 = HQ * LCLA_D * x.hq;
@@ -440,8 +480,8 @@ __device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t 
             for (int m = 0; m < NMAP; ++m)
 #pragma unroll
                 for (int j = 0; j < NBOX; ++j)   // box j: heads [j HQ / NBOX, (j + 1) HQ / NBOX) of the quad
-                    tma_load3(base + offs[m] + j * (HQ * LCLA_D * T * 2 / NBOX), maps[m], fb,
-                              x0 + j * (HQ * LCLA_D / NBOX), t, x.b);
+                    tma_load3_hint(base + offs[m] + j * (HQ * LCLA_D * T * 2 / NBOX), maps[m], fb,
+                                   x0 + j * (HQ * LCLA_D / NBOX), t, x.b, stream_pol);
             ring_next<S>(er);
             ++issued;
             if (!bar_wait(CEMPTY + 8 * cr.idx, cr.phase, abort_flag)) {
@@ -721,12 +761,14 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                     for (int pw = 0; pw < NPRO; ++pw) zs += zp[pw * 2 * 4 * 16];
                     __syncwarp();
                     if (lane == 0) bar_arrive(ZFREE);
-                    if (head < p.H) {   // row c = lane of S, then z
+                    if (head < p.H) {   // row c = lane of S, then z; kept in L2 for the scan
+                        const uint64_t keep = policy_evict_last();
                         float4 *row = reinterpret_cast<float4 *>(dst + lane * LCLA_D);
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
-                            row[j] = make_float4(sacc[4 * j], sacc[4 * j + 1], sacc[4 * j + 2], sacc[4 * j + 3]);
-                        dst[LCLA_D * LCLA_D + lane] = zs;
+                            st_v4_hint(row + j, make_float4(sacc[4 * j], sacc[4 * j + 1], sacc[4 * j + 2], sacc[4 * j + 3]),
+                                       keep);
+                        st_f32_hint(dst + LCLA_D * LCLA_D + lane, zs, keep);
                     }
                 }
             }
@@ -1023,7 +1065,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 if (nt == T) {
                     fence_async_smem();
                     __syncwarp();
-                    if (lane == 0 && head < p.H) tma_store3(&mo, obs, LCLA_D * head, t + 32 * hf, x.b);
+                    if (lane == 0 && head < p.H) tma_store3_hint(&mo, obs, LCLA_D * head, t + 32 * hf, x.b, policy_evict_first());
                 } else {   // ragged tile: lane = token, its 64-byte row back from the box to global memory
                     __syncwarp();
                     const int tok = lane;

@@ -44,6 +44,10 @@ SMALL = [  # (B, H, N, block_len, dtype, dist)
     (2, 7, 3001, 250, "bf16", "normal"),
     (1, 2, 1, 1, "f32", "normal"),
     (1, 2, 5, 9, "bf16", "normal"),
+    # more than 256 blocks: the scan runs in chunks (two kernels)
+    (1, 5, 20000, 64, "bf16", "normal"),
+    (2, 3, 17000, 64, "f32", "laplace_negrows"),
+    (1, 6, 30000, 100, "bf16", "laplace_negrows"),
 ]
 
 
