@@ -46,6 +46,10 @@ def _load() -> ctypes.CDLL:
     L.lcla_forward_timed.restype = I
     L.lcla_step.argtypes = [P, P, P, P, P, I, I, I, I, F, P, I, P, I, P, Z, P]
     L.lcla_step.restype = I
+    L.lcla_forward_blocks_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    L.lcla_forward_blocks_workspace_bytes.restype = Z
+    L.lcla_forward_blocks.argtypes = [P, P, P, P, P, I, I, I, I, P, I, F, P, P, I, P, Z, P]
+    L.lcla_forward_blocks.restype = I
     L.lcla_forward_plan_info.argtypes = [I, I, I, I, I, I, P]
     L.lcla_forward_plan_info.restype = I
     L.lcla_status_string.argtypes = [I]
@@ -94,6 +98,10 @@ def _inputs(q, k, v, cos, sin):
 
 def forward_workspace_bytes(B: int, H: int, N: int, d: int, block_len: int, dtype: int) -> int:
     return int(lib.lcla_forward_workspace_bytes(B, H, N, d, block_len, dtype))
+
+
+def forward_blocks_workspace_bytes(B: int, H: int, N: int, d: int, nblocks: int, dtype: int) -> int:
+    return int(lib.lcla_forward_blocks_workspace_bytes(B, H, N, d, nblocks, dtype))
 
 
 def step_workspace_bytes(B: int, H: int, L: int, d: int, dtype: int) -> int:
@@ -145,6 +153,34 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rope_cos: torch.T
                                   _ptr(state_out), code, _ptr(workspace),
                                   0 if workspace is None else workspace.numel(),
                                   _stream(stream, q.device), evp))
+    return out, state_out
+
+
+def forward_blocks(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rope_cos: torch.Tensor,
+                   rope_sin: torch.Tensor, block_offsets: torch.Tensor, eps: float = DEFAULT_EPS, *,
+                   out: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
+                   want_state: bool = True, workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """``lcla_forward_blocks``: as ``forward`` with explicit block boundaries,
+    ``block_offsets`` an int32 CUDA tensor [nblocks + 1] rising from 0 to N."""
+    B, N, H, d, code = _inputs(q, k, v, rope_cos, rope_sin)
+    if (not isinstance(block_offsets, torch.Tensor) or not block_offsets.is_cuda
+            or block_offsets.dtype != torch.int32 or block_offsets.dim() != 1
+            or not block_offsets.is_contiguous()):
+        raise ValueError("block_offsets must be a contiguous int32 CUDA tensor [nblocks + 1]")
+    nblocks = block_offsets.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, d + 1, d), dtype=torch.float32, device=q.device)
+    need = forward_blocks_workspace_bytes(B, H, N, d, nblocks, code)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(lib.lcla_forward_blocks(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin),
+                                   B, H, N, d, _ptr(block_offsets), nblocks, float(eps), _ptr(out),
+                                   _ptr(state_out), code, _ptr(workspace),
+                                   0 if workspace is None else workspace.numel(),
+                                   _stream(stream, q.device)))
     return out, state_out
 
 

@@ -37,18 +37,21 @@ int check_shape(int B, int H, int N, int d, int L, int dtype)
 }
 
 // Cut the problem into segments (see lcla_plan.h) and lay out the workspace:
-// [status word, 256 B][part: nseg x B x H x (d+1) x d fp32][pref: npref x B x H x (d+1) x d fp32].
-LclaPlan make_plan(int B, int H, int N, int L, int dtype)
+// [status word, 256 B][part: nseg x B x H x (d+1) x d fp32][pref: npref x B x H x (d+1) x d fp32]
+// [chunk totals of the scan, when it runs in chunks].  nblocks > 0: that many explicit blocks (their
+// offsets are read on the device), always in block mode, sized by their mean length.
+LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0)
 {
     LclaPlan p;
     memset(&p, 0, sizeof p);
+    if (nblocks > 0 && N > 0) L = (int)(((long long)N + nblocks - 1) / nblocks);
     p.B = B; p.H = H; p.N = N; p.L = L; p.dtype = dtype;
     p.ngroups = (H + LCLA_HG - 1) / LCLA_HG;
     p.nquads = (H + LCLA_TC_HQ - 1) / LCLA_TC_HQ;
     if (N == 0) return p;
-    p.nb = (int)(((long long)N + L - 1) / L);
+    p.nb = nblocks > 0 ? nblocks : (int)(((long long)N + L - 1) / L);
     const long long units = (long long)p.ngroups * B;
-    if (L >= LCLA_T) {
+    if (nblocks > 0 || L >= LCLA_T) {
         p.chunk = 0;
         p.tc = dtype == LCLA_BF16;
         p.T = p.tc ? LCLA_TC_T : LCLA_T;
@@ -407,6 +410,38 @@ int lcla_forward(const void *q, const void *k, const void *v, const float *rope_
 {
     return lcla_forward_timed(q, k, v, rope_cos, rope_sin, B, H, N, d, block_len, eps, out,
                               state_out, dtype, workspace, workspace_bytes, stream, nullptr);
+}
+
+size_t lcla_forward_blocks_workspace_bytes(int B, int H, int N, int d, int nblocks, int dtype)
+{
+    if (check_shape(B, H, N, d, 1, dtype) != LCLA_OK) return 0;
+    if (N > 0 && (nblocks < 1 || nblocks > N)) return 0;
+    const LclaPlan p = make_plan(B, H, N, 1, dtype, nblocks);
+    return grid_fits(p) ? p.ws_bytes : 0;
+}
+
+int lcla_forward_blocks(const void *q, const void *k, const void *v, const float *rope_cos,
+                        const float *rope_sin, int B, int H, int N, int d, const int *block_offsets,
+                        int nblocks, float eps, void *out, float *state_out, int dtype, void *workspace,
+                        size_t workspace_bytes, void *stream)
+{
+    int rc = check_shape(B, H, N, d, 1, dtype);
+    if (rc != LCLA_OK) return rc;
+    if (N > 0 && (nblocks < 1 || nblocks > N || !block_offsets)) return LCLA_ERR_INVALID_ARG;
+    if (N > 0 && ((uintptr_t)block_offsets & 3u)) return LCLA_ERR_MISALIGNED;
+    LclaPlan p = make_plan(B, H, N, 1, dtype, nblocks);
+    if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
+    rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, dtype, eps, workspace,
+                       workspace_bytes, p.ws_bytes);
+    if (rc != LCLA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        if (state_out && cudaMemsetAsync(state_out, 0, (size_t)B * H * LCLA_SZ * sizeof(float), st) != cudaSuccess)
+            return LCLA_ERR_CUDA;
+        return LCLA_OK;
+    }
+    p.boff = block_offsets;
+    return run(q, k, v, rope_cos, rope_sin, p, eps, out, nullptr, state_out, workspace, st, nullptr);
 }
 
 int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk, const float *cos_blk,

@@ -38,6 +38,8 @@ struct LclaPlan {
     int ngroups;   // head groups of LCLA_HG heads (CUDA-core grid)
     int nquads;    // head groups of LCLA_TC_HQ heads (tensor-core work units)
     int scs, nch;  // scan over many groups: segments per scan chunk (whole groups) and chunks; nch = 0: one pass
+    const int *boff;   // explicit blocks: device array of nb + 1 token offsets (block b = [boff[b], boff[b+1]));
+                       // null: uniform blocks of L tokens
     size_t part_off, pref_off, ctot_off, ws_bytes;   // workspace layout (bytes)
 };
 
@@ -64,8 +66,15 @@ LCLA_HD LclaSeg lcla_segment(const LclaPlan &p, int s)
     if (!p.chunk) {
         g.blk = s / p.nsb;
         const int j = s - g.blk * p.nsb;
-        const int b0 = g.blk * p.L;
-        const int bl = lcla_min_i(p.L, p.N - b0);
+        int b0, bl;
+        if (p.boff) {   // explicit blocks (device code only): clamped into [0, N], an inverted pair is empty
+            b0 = lcla_min_i(p.boff[g.blk] > 0 ? p.boff[g.blk] : 0, p.N);
+            const int b1 = lcla_min_i(p.boff[g.blk + 1] > 0 ? p.boff[g.blk + 1] : 0, p.N);
+            bl = b1 > b0 ? b1 - b0 : 0;
+        } else {
+            b0 = g.blk * p.L;
+            bl = lcla_min_i(p.L, p.N - b0);
+        }
         const int nt = (bl + p.T - 1) / p.T;               // tiles in this block
         const int per = (nt + p.nsb - 1) / p.nsb;          // tiles per segment
         g.t0 = b0 + lcla_min_i(lcla_min_i(j * per, nt) * p.T, bl);

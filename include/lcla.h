@@ -116,6 +116,39 @@ LCLA_API int lcla_forward_timed(const void *q, const void *k, const void *v,
                  void *workspace, size_t workspace_bytes, void *stream,
                  void *const *events);
 
+/*
+ * Workspace bytes lcla_forward_blocks needs for `nblocks` explicit blocks
+ * (0 when the arguments are invalid).  Depends only on the arguments.
+ */
+LCLA_API size_t lcla_forward_blocks_workspace_bytes(int B, int H, int N, int d, int nblocks, int dtype);
+
+/*
+ * Whole-sequence forward with explicit block boundaries instead of uniform
+ * blocks: block b holds tokens [block_offsets[b], block_offsets[b+1]), and a
+ * token attends to its own block and every earlier block, as in lcla_forward.
+ * The pages name a non-uniform partition as the one a released model
+ * configuration uses ("Add SANA-WM camera-controlled image-to-video
+ * pipeline", the review reply on uniform-only chunking: `first_chunk_plus_one`
+ * is the live configuration, e.g. a first block one latent frame longer).
+ *   block_offsets  int32 device array of nblocks + 1 offsets, 4-byte aligned,
+ *                  0 = o[0] < o[1] < ... < o[nblocks] = N.  Read only, on the
+ *                  device: the host cannot check it.  Offsets outside [0, N]
+ *                  are clamped and an inverted pair is an empty block, so a
+ *                  malformed array never reads or writes out of bounds, but
+ *                  the outputs of tokens it misses or covers twice are then
+ *                  undefined.
+ *   nblocks        1 <= nblocks <= N when N > 0.
+ * Every other argument, ownership and error as lcla_forward; the workspace is
+ * sized by lcla_forward_blocks_workspace_bytes.  Blocks of any length run on
+ * the whole-block path (tensor cores for bf16), with ragged tiles at block
+ * ends.
+ */
+LCLA_API int lcla_forward_blocks(const void *q, const void *k, const void *v,
+                 const float *rope_cos, const float *rope_sin,
+                 int B, int H, int N, int d, const int *block_offsets, int nblocks, float eps,
+                 void *out, float *state_out, int dtype,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
 /* Workspace bytes lcla_step needs (0 when the arguments are invalid). */
 LCLA_API size_t lcla_step_workspace_bytes(int B, int H, int L, int d, int dtype);
 
@@ -144,11 +177,11 @@ LCLA_API int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk,
 
 /*
  * How lcla_forward cuts this problem, for benchmarks and tests: writes
- * info[0] = 1 when tiles hold whole blocks (block_len <= 64), else 0;
+ * info[0] = 1 when tiles hold whole blocks (block_len < 64), else 0;
  * info[1] = segments (partial states written by the first pass);
  * info[2] = prefix states (blocks, or segments when info[0] = 1);
  * info[3] = tokens per tile; info[4] = 1 when the tensor-core kernels run
- * (bf16 with block_len > 64), else 0.  `info` holds 5 ints.  Returns an
+ * (bf16 with block_len >= 64), else 0.  `info` holds 5 ints.  Returns an
  * lcla_status; touches no device.
  */
 LCLA_API int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,

@@ -9,6 +9,8 @@ Routes (see ``lcla_oracle.c`` for the definition each one follows):
     masked(...)      the definition, pair by pair, O(N^2 d)
     recurrence(...)  per-block local states with a running inclusive sum
     step(...)        one block against a carried state, optional save
+    blocks(...)      explicit block boundaries: the step route chained over the
+                     blocks, each one saved into the carried state
     literal(...)     the printed non-causal formula (block_len = N), numpy
 
 Inputs are numpy arrays: q, k, v [B, N, H, d] as uint16 bf16 bit patterns or
@@ -126,6 +128,26 @@ class Oracle:
         return out
 
 
+    def blocks(self, q, k, v, rope_cos, rope_sin, offsets, eps: float = 1e-8,
+               state_in: Optional[np.ndarray] = None):
+        """Block boundaries given as token offsets 0 = o[0] < ... < o[nb] = N:
+        block b is [o[b], o[b+1]) and attends to itself and every earlier
+        block, which is the step route run block after block with save.
+        Returns (out [B, N, H, d], state_out [B, H, d+1, d]), float64."""
+        q = np.ascontiguousarray(q)
+        B, N, H, d = q.shape
+        o = [int(x) for x in np.asarray(offsets).ravel()]
+        if len(o) < 2 or o[0] != 0 or o[-1] != N or any(b <= a for a, b in zip(o, o[1:])):
+            raise ValueError("offsets must rise strictly from 0 to N")
+        state = np.zeros((B, H, d + 1, d), np.float64) if state_in is None else \
+            np.array(state_in, dtype=np.float64, order="C", copy=True)
+        out = np.empty((B, N, H, d), np.float64)
+        for a, b in zip(o, o[1:]):
+            out[:, a:b] = self.step(q[:, a:b], np.asarray(k)[:, a:b], np.asarray(v)[:, a:b],
+                                    np.asarray(rope_cos)[a:b], np.asarray(rope_sin)[a:b], state, True, eps)
+        return out, state
+
+
 _default: Optional[Oracle] = None
 
 
@@ -154,6 +176,10 @@ def recurrence(*a, **kw):
 
 def step(*a, **kw):
     return default().step(*a, **kw)
+
+
+def blocks(*a, **kw):
+    return default().blocks(*a, **kw)
 
 
 def _prep(q, k, v, rope_cos, rope_sin):

@@ -360,6 +360,54 @@ def pin_bf16_widening(orc):
     rows_close(orc.recurrence(*bits, c, s, 9, 1e-8)[0], ref, 1e-12, "bf16 vs printed formula")
 
 
+def masked_blocks_numpy(q, k, v, cos, sin, offsets, eps):
+    """The definition pair by pair with an explicit block id per token:
+    blk(n) = b for o[b] <= n < o[b+1]; token i takes every j with
+    blk(j) <= blk(i).  Plain numpy, complex rotary; small N only."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    N = q.shape[1]
+    blk = np.searchsorted(np.asarray(offsets), np.arange(N), side="right") - 1
+    fq, fk = np.maximum(q, 0), np.maximum(k, 0)
+    rq, rk = _complex_rotary(fq, cos, sin), _complex_rotary(fk, cos, sin)
+    mask = (blk[None, :] <= blk[:, None]).astype(np.float64)          # [i, j]
+    a = np.einsum("bihe,bjhe->bhij", rq, rk) * mask                    # rotated scores
+    g = np.einsum("bihe,bjhe->bhij", fq, fk) * mask                    # normaliser terms
+    num = np.einsum("bhij,bjhc->bihc", a, v)
+    den = np.einsum("bhij->bih", g)[..., None] + eps
+    return num / den
+
+
+def pin_explicit_blocks(orc):
+    """Explicit block boundaries (the blocks route, a step chain): random
+    offsets with blocks of a single token, a first block one frame longer than
+    the rest, and one block, against the pair-by-pair definition; uniform
+    offsets against the block recurrence."""
+    rng = np.random.default_rng(41)
+    for seed, N, offs in [(41, 37, None), (42, 40, [0, 12, 20, 28, 36, 40]),   # 4 + 4k "frames" of 4
+                          (43, 23, [0, 23]), (44, 30, [0, 1, 2, 3, 17, 18, 30])]:
+        if offs is None:
+            cuts = np.sort(rng.choice(np.arange(1, N), size=9, replace=False))
+            offs = [0] + [int(c) for c in cuts] + [N]
+        for dtype, dist in [("f32", "normal"), ("bf16", "laplace_negrows")]:
+            inp = small(seed, N=N, d=8, dtype=dtype, dist=dist)
+            out, st = orc.blocks(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, offs, 1e-8)
+            ref = masked_blocks_numpy(inp.as_f32("q"), inp.as_f32("k"), inp.as_f32("v"),
+                                      inp.rope_cos, inp.rope_sin, offs, 1e-8)
+            rows_close(out, ref, 1e-12, f"blocks vs definition {offs}")
+            # the final state is the sum over all tokens whatever the partition
+            _, st1, _ = orc.recurrence(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, N, 1e-8)
+            assert np.abs(st - st1).max() <= 1e-12 * np.abs(st1).max(), "blocks state vs total"
+    inp = small(45, N=33, d=8)
+    L = 7
+    offs = list(range(0, 33, L)) + [33]
+    a, sa = orc.blocks(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, offs, 1e-8)
+    b, sb, _ = orc.recurrence(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, L, 1e-8)
+    rows_close(a, b, 1e-12, "uniform offsets vs recurrence")
+
+
 ALL_PINS = [pin_masked_equals_recurrence, pin_single_block_equals_printed_formula,
             pin_block_len_one_is_token_causal, pin_step_chain_equals_forward,
-            pin_exact_rational, pin_closed_forms, pin_symmetries, pin_bf16_widening]
+            pin_exact_rational, pin_closed_forms, pin_symmetries, pin_bf16_widening,
+            pin_explicit_blocks]

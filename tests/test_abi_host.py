@@ -21,7 +21,8 @@ def declared_symbols():
 def test_every_declared_symbol_is_exported():
     names = declared_symbols()
     assert {"lcla_forward", "lcla_step", "lcla_forward_workspace_bytes",
-            "lcla_step_workspace_bytes", "lcla_status_string", "lcla_version"} <= set(names)
+            "lcla_step_workspace_bytes", "lcla_status_string", "lcla_version",
+            "lcla_forward_blocks", "lcla_forward_blocks_workspace_bytes"} <= set(names)
     lib = ctypes.CDLL(lcla.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -105,3 +106,25 @@ def test_step_rejects(kw, code):
 def test_trivial_calls_need_no_gpu():
     # an empty block is a valid no-op and touches nothing
     assert stp(L=0, q=None, k=None, v=None, c=None, s=None, out=None, ws=None, wsb=0) == OK
+
+
+def test_explicit_blocks_workspace_and_arguments():
+    f = lcla.forward_blocks_workspace_bytes
+    # the same cut as uniform blocks of the mean length
+    assert f(1, 70, 32760, 32, 7, lcla.BF16) == lcla.forward_workspace_bytes(1, 70, 32760, 32, 4680, lcla.BF16)
+    assert f(1, 4, 100, 32, 0, lcla.BF16) == 0          # no blocks
+    assert f(1, 4, 100, 32, 101, lcla.BF16) == 0        # more blocks than tokens
+    assert f(1, 4, 100, 32, 3, lcla.BF16) > 0
+    assert f(1, 4, 100, 64, 3, lcla.BF16) == 0          # d = 64 not served
+    import ctypes
+    a = 1 << 20
+    fn = lcla.lib.lcla_forward_blocks
+    # argument errors return before any launch (no device memory is touched)
+    rc = fn(a, 2 * a, 3 * a, 4 * a, 5 * a, 1, 4, 100, 32, None, 3, 1e-8, 6 * a, None, lcla.BF16, None, 0, None)
+    assert rc == 1                                      # offsets missing
+    rc = fn(a, 2 * a, 3 * a, 4 * a, 5 * a, 1, 4, 100, 32, 7 * a + 2, 3, 1e-8, 6 * a, None, lcla.BF16, None, 0, None)
+    assert rc == 3                                      # offsets not 4-byte aligned
+    rc = fn(a, 2 * a, 3 * a, 4 * a, 5 * a, 1, 4, 100, 32, 7 * a, 101, 1e-8, 6 * a, None, lcla.BF16, None, 0, None)
+    assert rc == 1                                      # more blocks than tokens
+    rc = fn(a, 2 * a, 3 * a, 4 * a, 5 * a, 1, 4, 100, 32, 7 * a, 3, 1e-8, 6 * a, None, lcla.BF16, None, 0, None)
+    assert rc == 4                                      # workspace missing

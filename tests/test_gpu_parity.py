@@ -191,3 +191,73 @@ def test_repeated_calls_bit_identical(name):
         torch.cuda.synchronize()
         assert torch.equal(st, st0), "state differs between identical calls"
         assert torch.equal(out, out0), "output differs between identical calls"
+
+
+def _random_offsets(N, nblocks, seed, min_len=1):
+    rng = np.random.default_rng(seed)
+    cuts = np.sort(rng.choice(np.arange(min_len, N - min_len + 1), size=nblocks - 1, replace=False))
+    return [0] + [int(c) for c in cuts] + [N]
+
+
+FRAME = 130   # tokens per latent frame in the small explicit-block cases
+BLOCK_CASES = [  # (B, H, N, offsets, dtype, dist)
+    # first block one latent frame longer than the others (4 + 3 + 3 + 3 frames)
+    (1, 6, 13 * FRAME, [0, 4 * FRAME, 7 * FRAME, 10 * FRAME, 13 * FRAME], "bf16", "normal"),
+    (2, 3, 13 * FRAME, [0, 4 * FRAME, 7 * FRAME, 10 * FRAME, 13 * FRAME], "f32", "laplace_negrows"),
+    # random lengths: single tokens, blocks shorter than a tile, long blocks
+    (1, 5, 3000, _random_offsets(3000, 23, 7), "bf16", "laplace_negrows"),
+    (1, 4, 2000, _random_offsets(2000, 31, 8), "f32", "normal"),
+    (2, 7, 1500, [0, 1, 2, 3, 64, 65, 200, 1000, 1499, 1500], "bf16", "normal"),
+    # one block; one block per token; more than 256 blocks (chunked scan)
+    (1, 2, 300, [0, 300], "bf16", "normal"),
+    (1, 2, 150, list(range(151)), "f32", "normal"),
+    (1, 3, 5000, _random_offsets(5000, 300, 9), "bf16", "laplace_negrows"),
+]
+
+
+@pytest.mark.parametrize("B,H,N,offs,dtype,dist", BLOCK_CASES,
+                         ids=[f"case{i}" for i in range(len(BLOCK_CASES))])
+def test_explicit_blocks_full(B, H, N, offs, dtype, dist):
+    """lcla_forward_blocks against the oracle's blocks route (the step route
+    chained over the given blocks), every output and the state."""
+    spec = Spec("blocks", B, H, N, 32, N, dtype, 500 + len(offs), qk_dist=dist, v_sigma=2.0)
+    inp = make_inputs(spec, threads=1)
+    q, k, v, c, s = inputs_to_dev(inp)
+    o = torch.tensor(offs, dtype=torch.int32, device="cuda")
+    out, st = lcla.forward_blocks(q, k, v, c, s, o, spec.eps)
+    torch.cuda.synchronize()
+    ref, ref_st = oracle.blocks(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, offs, spec.eps)
+    check_outputs(host(out), ref, dtype, f"blocks {offs[:6]}...")
+    check_state(host(st), ref_st, f"blocks state {offs[:6]}...")
+
+
+def test_explicit_blocks_uniform_match_forward():
+    """Uniform offsets give the uniform forward's results (both rounded to
+    bf16, one ulp apart at most)."""
+    spec = Spec("blocks_uniform", 1, 9, 4000, 32, 700, "bf16", 61, qk_dist="laplace_negrows", v_sigma=2.0)
+    inp = make_inputs(spec, threads=1)
+    q, k, v, c, s = inputs_to_dev(inp)
+    offs = list(range(0, spec.N, spec.block_len)) + [spec.N]
+    a, sa = lcla.forward(q, k, v, c, s, spec.block_len, spec.eps)
+    b, sb = lcla.forward_blocks(q, k, v, c, s, torch.tensor(offs, dtype=torch.int32, device="cuda"), spec.eps)
+    torch.cuda.synchronize()
+    check_outputs(host(b), host(a), "bf16", "blocks vs uniform forward", ulps=1.0)
+    check_state(host(sb), host(sa), "blocks vs uniform state")
+
+
+def test_explicit_blocks_480p_first_block_longer():
+    """The 480p-like forward (21 latent frames of 30 x 52 tokens) cut as a
+    first block of 4 frames, then 3-frame blocks and a 2-frame tail, at full
+    size in the launch configuration the benchmark uses, every output against
+    the oracle."""
+    spec = NAMED["fwd480p_bf16"]
+    F = 30 * 52
+    offs = [0, 4 * F] + [4 * F + 3 * F * i for i in range(1, 6)] + [spec.N]
+    assert offs[-2] < spec.N and len(offs) == 8
+    inp = make_inputs(spec)
+    q, k, v, c, s = inputs_to_dev(inp)
+    out, st = lcla.forward_blocks(q, k, v, c, s, torch.tensor(offs, dtype=torch.int32, device="cuda"), spec.eps)
+    torch.cuda.synchronize()
+    ref, ref_st = oracle.blocks(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, offs, spec.eps)
+    check_outputs(host(out), ref, "bf16", "480p explicit blocks")
+    check_state(host(st), ref_st, "480p explicit blocks state")
