@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--op", choices=["attention", "tconv"], default="attention",
+                    help="attention: the block-causal attention forward (the headline); "
+                         "tconv: the causal temporal convolution with a cached last frame")
     return ap.parse_args()
 
 
@@ -273,10 +276,93 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+TCONV = {"name": "tconv480p_bf16", "B": 1, "F": 21, "S": 30 * 52, "C": 2240, "dtype": "bf16", "seed": 11}
+
+
+def run_tconv(args):
+    """One GPU: lcla_temporal_conv over the 480p-like latent (21 frames of
+    30 x 52 tokens, width 2240 = 70 heads x 32), with a cached previous frame
+    saved each step; inputs resident in HBM and larger than L2.  The JSON line
+    keeps the headline's keys with this op's metric."""
+    import torch
+    import block_causal_relu_b200 as lcla
+    from oracle.tconv import temporal_conv as tconv_oracle
+    from workloads import f64_to_bf16_bits
+    w = TCONV
+    B, F, S, C = w["B"], w["F"], w["S"], w["C"]
+    rng = np.random.default_rng(w["seed"])
+    x_bits = f64_to_bf16_bits(rng.standard_normal(B * F * S * C)).reshape(B, F * S, C)
+    c_bits = f64_to_bf16_bits(rng.standard_normal(B * S * C)).reshape(B, S, C)
+    wt = rng.standard_normal((2, C)).astype(np.float32)
+    bias = rng.standard_normal(C).astype(np.float32)
+    dev = torch.device("cuda", 0)
+    x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    cache = torch.from_numpy(c_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    wd, bd = torch.from_numpy(wt).to(dev), torch.from_numpy(bias).to(dev)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        lcla.temporal_conv(x, S, wd, bd, cache, save=True, out=y, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        e0.record(stream)
+        for _ in range(K):
+            lcla.temporal_conv(x, S, wd, bd, cache, save=True, out=y, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / K
+    units = B * F * S * C
+    bytes_step = 2 * units * 2 + 2 * B * S * C * 2 + 3 * C * 4     # x in, y out, cache in and out, weights
+    peak, peak_src = measured_peak()
+    achieved = bytes_step / (ms / 1e3) / 1e9
+    # end to end: x from pinned host memory, the call, y back
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    KE = max(1, min(args.e2e_steps, K))
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(KE):
+        x.copy_(xh, non_blocking=True)
+        lcla.temporal_conv(x, S, wd, bd, cache, save=True, out=y, stream=stream)
+        yh.copy_(y, non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ems = t0.elapsed_time(t1) / KE
+    # the fp64 oracle on the host, same workload, bounded
+    n, c0 = 0, time.perf_counter()
+    while True:
+        tconv_oracle(x_bits, S, wt, bias, c_bits)
+        n += 1
+        el = time.perf_counter() - c0
+        if el >= max(1.0, args.cpu_seconds) or n >= 20:
+            break
+    line = {"metric": "temporal-conv tokens*channels/s and achieved HBM GB/s, 1 GPU", "op": "tconv",
+            "value": units / (ms / 1e3), "unit": "token*channels/s", "n_gpus": 1, "steps": K, "warmup": W,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded)",
+            "config": {"workload": f"{w['name']}: B={B} F={F} S={S} C={C}", "cache": "previous frame, saved",
+                       "l2": f"x and y {2 * units * 2 / 1e6:.0f} MB per step > 126 MB"},
+            "roofline": {"bound": "hbm", "kernel": "temporal_conv_k2", "achieved": achieved, "peak": peak,
+                         "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "algorithmic_bytes": bytes_step},
+            "cpu_baseline": {"value": n * units / el, "unit": "token*channels/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{n} whole call(s) of the numpy fp64 oracle, {el:.1f} s"},
+            "e2e": {"value": units / (ems / 1e3), "unit": "token*channels/s",
+                    "h2d_bytes_per_step": units * 2, "d2h_bytes_per_step": units * 2, "ms_per_step": ems,
+                    "steps": KE},
+            "gpu_launches": K, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "tconv":
+        return run_tconv(args)
 
     import torch
 

@@ -50,6 +50,8 @@ def _load() -> ctypes.CDLL:
     L.lcla_forward_blocks_workspace_bytes.restype = Z
     L.lcla_forward_blocks.argtypes = [P, P, P, P, P, I, I, I, I, P, I, F, P, P, I, P, Z, P]
     L.lcla_forward_blocks.restype = I
+    L.lcla_temporal_conv.argtypes = [P, I, I, I, I, P, P, P, I, P, I, P]
+    L.lcla_temporal_conv.restype = I
     L.lcla_forward_plan_info.argtypes = [I, I, I, I, I, I, P]
     L.lcla_forward_plan_info.restype = I
     L.lcla_status_string.argtypes = [I]
@@ -202,4 +204,33 @@ def step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cos: torch.Tensor,
     _check(lib.lcla_step(_ptr(q), _ptr(k), _ptr(v), _ptr(cos), _ptr(sin), B, H, L, d, float(eps),
                          _ptr(state), int(bool(save)), _ptr(out), code, _ptr(workspace),
                          0 if workspace is None else workspace.numel(), _stream(stream, q.device)))
+    return out
+
+
+def temporal_conv(x: torch.Tensor, tokens_per_frame: int, weight: torch.Tensor,
+                  bias: Optional[torch.Tensor] = None, cache: Optional[torch.Tensor] = None,
+                  save: bool = False, *, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``lcla_temporal_conv``: causal size-2 depthwise convolution over latent
+    frames of ``x`` [B, F * S, C] (S = ``tokens_per_frame``), with weight [2, C]
+    and bias [C] fp32 and the previous frame from ``cache`` [B, S, C] (zeros
+    when None); ``save`` overwrites the cache with x's last frame."""
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or not x.is_contiguous() or x.dim() != 3:
+        raise ValueError("x must be a contiguous CUDA tensor [B, F * S, C]")
+    B, N, C = x.shape
+    S = int(tokens_per_frame)
+    if S < 1 or N % S:
+        raise ValueError("x's token count must be a whole number of frames")
+    code = _dtype_code(x)
+    for name, t, shape in (("weight", weight, (2, C)), ("bias", bias, (C,))):
+        if t is None:
+            continue
+        if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor {list(shape)}")
+    if cache is not None and (not cache.is_cuda or cache.dtype != x.dtype or not cache.is_contiguous()
+                              or tuple(cache.shape) != (B, S, C)):
+        raise ValueError("cache must be a contiguous CUDA tensor [B, S, C] of x's dtype")
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib.lcla_temporal_conv(_ptr(x), B, N // S, S, C, _ptr(weight), _ptr(bias), _ptr(cache),
+                                  int(bool(save)), _ptr(out), code, _stream(stream, x.device)))
     return out

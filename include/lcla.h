@@ -149,6 +149,32 @@ LCLA_API int lcla_forward_blocks(const void *q, const void *k, const void *v,
                  void *out, float *state_out, int dtype,
                  void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Causal temporal convolution of the Mix-FFN with a cached last frame, the
+ * step after attention in a block.  The pages say the causal Mix-FFN keeps
+ * the previous block's last frame for its temporal convolution ("Block Causal
+ * Linear Attention", section "What SANA-Video Actually Uses"; "[feat]
+ * LongSANA": causal computation for the Mix-FFN, the convolution in the MLP)
+ * and give no kernel size; one retained frame is read as a depthwise causal
+ * convolution of size 2 over latent frames:
+ *   y[b, f, s, c] = weight[0][c] x[b, f, s, c] + weight[1][c] x[b, f-1, s, c]
+ *                   + bias[c]
+ * where x[b, -1, s, c] is cache[b, s, c] (zeros when cache is NULL).
+ *   x, y     [B, F * S, C] device, dtype (token f * S + s of frame f); F >= 0
+ *            frames of S >= 1 tokens; C >= 8, a multiple of 8.  y must not
+ *            overlap x, the cache, weight or bias.
+ *   weight   [2][C] float32 device; bias [C] float32 device or NULL.
+ *   cache    [B, S, C] device, dtype, or NULL (no earlier frame).  Read; with
+ *            save = 1 it is overwritten with the last frame x[b, F-1] (the
+ *            next block's history); save = 0 leaves it bit-unchanged (several
+ *            denoising steps per block).  It must not overlap x.
+ * Every pointer 16-byte aligned.  Computed in fp32, y rounded to dtype.
+ * Returns an lcla_status (F = 0: LCLA_OK, nothing enqueued).
+ */
+LCLA_API int lcla_temporal_conv(const void *x, int B, int F, int S, int C,
+                 const float *weight, const float *bias, void *cache, int save,
+                 void *y, int dtype, void *stream);
+
 /* Workspace bytes lcla_step needs (0 when the arguments are invalid). */
 LCLA_API size_t lcla_step_workspace_bytes(int B, int H, int L, int d, int dtype);
 

@@ -22,7 +22,7 @@ def test_every_declared_symbol_is_exported():
     names = declared_symbols()
     assert {"lcla_forward", "lcla_step", "lcla_forward_workspace_bytes",
             "lcla_step_workspace_bytes", "lcla_status_string", "lcla_version",
-            "lcla_forward_blocks", "lcla_forward_blocks_workspace_bytes"} <= set(names)
+            "lcla_forward_blocks", "lcla_forward_blocks_workspace_bytes", "lcla_temporal_conv"} <= set(names)
     lib = ctypes.CDLL(lcla.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -128,3 +128,15 @@ def test_explicit_blocks_workspace_and_arguments():
     assert rc == 1                                      # more blocks than tokens
     rc = fn(a, 2 * a, 3 * a, 4 * a, 5 * a, 1, 4, 100, 32, 7 * a, 3, 1e-8, 6 * a, None, lcla.BF16, None, 0, None)
     assert rc == 4                                      # workspace missing
+
+
+def test_temporal_conv_arguments():
+    fn = lcla.lib.lcla_temporal_conv
+    a = 1 << 20
+    # argument errors return before any launch (no device memory is touched)
+    assert fn(a, 1, 2, 3, 12, 2 * a, None, None, 0, 3 * a, lcla.BF16, None) == 1   # C not a multiple of 8
+    assert fn(a, 1, 2, 3, 16, 2 * a, None, None, 0, 3 * a, 7, None) == 1            # bad dtype
+    assert fn(a + 8, 1, 2, 3, 16, 2 * a, None, None, 0, 3 * a, lcla.BF16, None) == 3   # misaligned x
+    assert fn(a, 1, 2, 3, 16, 2 * a, None, a + 64, 0, 3 * a, lcla.BF16, None) == 1     # cache inside x
+    assert fn(a, 1, 0, 3, 16, 2 * a, None, None, 0, 3 * a, lcla.BF16, None) == 0       # no frames: nothing to do
+    assert fn(None, 1, 2, 3, 16, 2 * a, None, None, 0, 3 * a, lcla.BF16, None) == 1    # x missing
