@@ -9,11 +9,13 @@ end-to-end number through the same call with host buffers, the roofline of
 the dominant kernel, and the fp64 CPU oracle timed on the host as a baseline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-e2e] [--cpu-seconds S]
+                    [--workload NAME] [--no-e2e] [--cpu-seconds S] [--parallel replicas|seq]
 
-N > 1 is launched by torchrun (one rank per GPU): every rank runs its own
-independent copy of the workload (different seed), no data-path collective;
-timing is the max over ranks.
+N > 1 is launched by torchrun (one rank per GPU): by default every rank runs
+its own independent copy of the workload (different seed), no data-path
+collective; ``--parallel seq`` instead cuts one sequence into runs of whole
+blocks, one per rank, with one all-gather of state totals per step.  Timing
+is the max over ranks.
 """
 from __future__ import annotations
 
@@ -51,6 +53,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--parallel", choices=["replicas", "seq"], default="replicas",
+                    help="N > 1: replicas = one independent copy of the workload per rank (weak scaling); "
+                         "seq = one sequence cut into runs of whole blocks, one per rank, with one "
+                         "all-gather of state totals per step (strong scaling)")
     ap.add_argument("--op", choices=["attention", "tconv"], default="attention",
                     help="attention: the block-causal attention forward (the headline); "
                          "tconv: the causal temporal convolution with a cached last frame")
@@ -357,12 +363,100 @@ def run_tconv(args):
     print(json.dumps(line), flush=True)
 
 
+def run_seq(args):
+    """Sequence-sharded forward: every rank holds the whole-block run
+    ``shard_bounds(N, block_len, world)[rank]`` of one sequence; a step is
+    lcla_shard_begin, one NCCL all-gather of the state totals, lcla_shard_end.
+    The value counts the sequence's token-heads once (strong scaling)."""
+    import torch
+    import block_causal_relu_b200 as lcla
+    from block_causal_relu_b200.seqshard import gather_totals, shard_bounds
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    ranks = Ranks(world, rank, "nccl", device)
+    spec = NAMED[args.workload]                                # one sequence, the same on every rank
+    inp = make_inputs(spec)
+    t0, t1 = shard_bounds(spec.N, spec.block_len, world)[rank]
+    Nr = t1 - t0
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(a).to(device)
+
+    q, k, v = (to_dev(a[:, t0:t1]) for a in (inp.q, inp.k, inp.v))
+    c, s = to_dev(inp.rope_cos[t0:t1]), to_dev(inp.rope_sin[t0:t1])
+    code = lcla.BF16 if spec.dtype == "bf16" else lcla.F32
+    out = torch.empty_like(q)
+    st = torch.empty((spec.B, spec.H, 33, 32), dtype=torch.float32, device=device)
+    total = torch.empty_like(st)
+    ws = torch.empty(max(1, lcla.shard_workspace_bytes(spec.B, spec.H, Nr, 32, spec.block_len, code)),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        lcla.shard_begin(k, v, c, s, spec.block_len, total_out=total, workspace=ws, stream=stream)
+        totals = gather_totals(total)
+        lcla.shard_end(q, k, v, c, s, spec.block_len, totals, rank, ws, spec.eps, out=out, state_out=st,
+                       stream=stream)
+
+    def barrier():
+        ranks.barrier()
+        torch.cuda.synchronize(device)
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device) as clk:
+        e0.record(stream)
+        for _ in range(K):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier()
+    ms_total = ranks.max(e0.elapsed_time(e1))
+    ms = ms_total / K
+    plan = lcla.plan_info(spec.B, spec.H, max(Nr, 1), 32, spec.block_len, code)
+    esz = spec.elem_bytes
+    local_bytes = 4 * spec.B * Nr * spec.H * spec.d * esz + 2 * 2 * Nr * (spec.d // 2) * 4
+    slowest_bytes = ranks.max(float(local_bytes))
+    peak, peak_kind = measured_peak()
+    achieved = slowest_bytes / (ms / 1e3) / 1e9
+    if rank == 0:
+        ngroups = plan["segments"] if plan["chunk_mode"] else plan["prefixes"]
+        scan_k = 1 if ngroups <= 256 else 2
+        cfg = workload_config(spec, world)
+        cfg["parallelism"] = (f"sequence sharded over {world} rank(s): whole blocks per rank, "
+                              f"one all-gather of {spec.B * spec.H * STATE_BYTES} B per rank per step")
+        line = {"metric": METRIC, "value": spec.token_heads / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+                "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+                "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic (seeded)", "config": cfg,
+                "roofline": {"bound": "hbm", "kernel": "whole sharded step (largest shard)", "achieved": achieved,
+                             "peak": peak, "peak_source": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": None, "algorithmic_bytes": slowest_bytes},
+                "cpu_baseline": None, "e2e": None,
+                "gpu_launches": K * (2 + 2 * scan_k + 1), "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    ranks.close()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.op == "tconv":
         return run_tconv(args)
+    if args.parallel == "seq":
+        return run_seq(args)
 
     import torch
 

@@ -16,6 +16,8 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["forward", "step", "forward_workspace_bytes", "step_workspace_bytes", "plan_info",
+           "forward_blocks", "forward_blocks_workspace_bytes", "temporal_conv",
+           "shard_begin", "shard_end", "shard_workspace_bytes",
            "LclaError", "LIB_PATH", "lib", "BF16", "F32", "D"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblcla.so")
@@ -52,6 +54,12 @@ def _load() -> ctypes.CDLL:
     L.lcla_forward_blocks.restype = I
     L.lcla_temporal_conv.argtypes = [P, I, I, I, I, P, P, P, I, P, I, P]
     L.lcla_temporal_conv.restype = I
+    L.lcla_shard_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    L.lcla_shard_workspace_bytes.restype = Z
+    L.lcla_shard_begin.argtypes = [P, P, P, P, I, I, I, I, I, P, I, P, Z, P]
+    L.lcla_shard_begin.restype = I
+    L.lcla_shard_end.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P, I, I, P, P, P, I, P, Z, P]
+    L.lcla_shard_end.restype = I
     L.lcla_forward_plan_info.argtypes = [I, I, I, I, I, I, P]
     L.lcla_forward_plan_info.restype = I
     L.lcla_status_string.argtypes = [I]
@@ -183,6 +191,67 @@ def forward_blocks(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rope_cos: 
                                    _ptr(state_out), code, _ptr(workspace),
                                    0 if workspace is None else workspace.numel(),
                                    _stream(stream, q.device)))
+    return out, state_out
+
+
+def shard_workspace_bytes(B: int, H: int, N: int, d: int, block_len: int, dtype: int) -> int:
+    return int(lib.lcla_shard_workspace_bytes(B, H, N, d, block_len, dtype))
+
+
+def _state_tensor(name: str, t: Optional[torch.Tensor], B: int, H: int, d: int, lead=()) -> None:
+    if t is None:
+        return
+    if (not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32
+            or not t.is_contiguous() or tuple(t.shape) != (*lead, B, H, d + 1, d)):
+        raise ValueError(f"{name} must be a contiguous float32 CUDA tensor {[*lead, B, H, d + 1, d]}")
+
+
+def shard_begin(k: torch.Tensor, v: torch.Tensor, rope_cos: torch.Tensor, rope_sin: torch.Tensor,
+                block_len: int, *, total_out: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None,
+                stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """``lcla_shard_begin``: this rank's state total over its tokens k, v
+    [B, N, H, d] (whole blocks of the sequence, tables at their absolute
+    positions).  Returns (total [B, H, d+1, d] fp32, workspace); pass the same
+    workspace to ``shard_end``."""
+    B, N, H, d, code = _inputs(k, k, v, rope_cos, rope_sin)
+    if total_out is None:
+        total_out = torch.empty((B, H, d + 1, d), dtype=torch.float32, device=k.device)
+    _state_tensor("total_out", total_out, B, H, d)
+    need = shard_workspace_bytes(B, H, N, d, block_len, code)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
+    _check(lib.lcla_shard_begin(_ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), B, H, N, d, int(block_len),
+                                _ptr(total_out), code, _ptr(workspace),
+                                0 if workspace is None else workspace.numel(), _stream(stream, k.device)))
+    return total_out, workspace
+
+
+def shard_end(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rope_cos: torch.Tensor,
+              rope_sin: torch.Tensor, block_len: int, totals: torch.Tensor, rank: int,
+              workspace: Optional[torch.Tensor], eps: float = DEFAULT_EPS, *,
+              state_in: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+              state_out: Optional[torch.Tensor] = None, want_state: bool = True,
+              stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """``lcla_shard_end``: this rank's outputs from the gathered ``totals``
+    [R, B, H, d+1, d] (every rank's ``shard_begin`` total, in rank order) and
+    the workspace ``shard_begin`` filled.  Returns (out, state after the whole
+    sequence, or None)."""
+    B, N, H, d, code = _inputs(q, k, v, rope_cos, rope_sin)
+    if not isinstance(totals, torch.Tensor) or totals.dim() != 5:
+        raise ValueError("totals must be [R, B, H, d+1, d]")
+    nranks = totals.shape[0]
+    _state_tensor("totals", totals, B, H, d, lead=(nranks,))
+    _state_tensor("state_in", state_in, B, H, d)
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, d + 1, d), dtype=torch.float32, device=q.device)
+    _state_tensor("state_out", state_out, B, H, d)
+    _check(lib.lcla_shard_end(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), B, H, N, d,
+                              int(block_len), float(eps), _ptr(totals), nranks, int(rank), _ptr(state_in),
+                              _ptr(out), _ptr(state_out), code, _ptr(workspace),
+                              0 if workspace is None else workspace.numel(), _stream(stream, q.device)))
     return out, state_out
 
 

@@ -16,6 +16,7 @@
 #include "lcla.h"
 #include "lcla_ffma.cuh"
 #include "lcla_plan.h"
+#include "lcla_shard.cuh"
 #include "lcla_tc.cuh"
 
 namespace {
@@ -113,6 +114,12 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0)
     p.ws_bytes = p.ctot_off + (p.nch ? round_up((size_t)(p.nch + 1) * slice) : 0);
     return p;
 }
+
+// What one call runs: the whole forward, or one of the two halves that a
+// sequence-sharded forward splits it into (lcla_shard_begin: pass A and the
+// shard's total state; lcla_shard_end: the scan from the carried-in state and
+// pass C, reading the partials that the begin call left in the workspace).
+enum Phase { PH_ALL, PH_BEGIN, PH_END };
 
 // The launch grid flattens (segment, head group) into blockIdx.x.
 bool grid_fits(const LclaPlan &p) { return (long long)p.nseg * p.ngroups <= 0x7fffffffLL; }
@@ -241,11 +248,12 @@ bool map_table(CUtensorMap *m, const float *base, int N)
 // be encoded, so that the caller can run the CUDA-core kernels instead.
 bool launch_tc(const void *q, const void *k, const void *v, const float *rc, const float *rs,
                const LclaPlan &p, float eps, void *out, const float *state_in, float *state_out,
-               unsigned char *ws, cudaStream_t st, cudaEvent_t const *ev, int *rc_out)
+               unsigned char *ws, cudaStream_t st, cudaEvent_t const *ev, int *rc_out, Phase ph = PH_ALL)
 {
     CUtensorMap mq, mk, mv, mo, mc, ms;
-    if (!map_tokens(&mq, q, p.B, p.N, p.H) || !map_tokens(&mk, k, p.B, p.N, p.H) ||
-        !map_tokens(&mv, v, p.B, p.N, p.H) || !map_out_blocks(&mo, out, p.B, p.N, p.H) ||
+    const bool a = ph != PH_END, c = ph != PH_BEGIN;
+    if ((a && (!map_tokens(&mk, k, p.B, p.N, p.H) || !map_tokens(&mv, v, p.B, p.N, p.H))) ||
+        (c && (!map_tokens(&mq, q, p.B, p.N, p.H) || !map_out_blocks(&mo, out, p.B, p.N, p.H))) ||
         !map_table(&mc, rc, p.N) || !map_table(&ms, rs, p.N))
         return false;
     float *part = reinterpret_cast<float *>(ws + p.part_off);
@@ -253,18 +261,22 @@ bool launch_tc(const void *q, const void *k, const void *v, const float *rc, con
     int *status = reinterpret_cast<int *>(ws);
     const long long units = (long long)p.nseg * p.nquads * p.B;
     const dim3 grid((unsigned)(units < LCLA_TC_CTAS ? units : LCLA_TC_CTAS));
-    set_smem(lcla::tc::pass_a_tc, lcla::tc::LayA::BYTES);
-    set_smem(lcla::tc::pass_c_tc, lcla::tc::LayC::BYTES);
-    cudaMemsetAsync(status, 0, sizeof(int), st);
-    if (ev) cudaEventRecord(ev[0], st);
-    lcla::tc::pass_a_tc<<<grid, lcla::tc::LayA::NTHREADS, lcla::tc::LayA::BYTES, st>>>(mk, mv, mc, ms, p, part,
-                                                                                       status);
-    if (ev) cudaEventRecord(ev[1], st);
+    if (a) {
+        set_smem(lcla::tc::pass_a_tc, lcla::tc::LayA::BYTES);
+        cudaMemsetAsync(status, 0, sizeof(int), st);
+        if (ev) cudaEventRecord(ev[0], st);
+        lcla::tc::pass_a_tc<<<grid, lcla::tc::LayA::NTHREADS, lcla::tc::LayA::BYTES, st>>>(mk, mv, mc, ms, p,
+                                                                                           part, status);
+        if (ev) cudaEventRecord(ev[1], st);
+    }
     launch_scan(p, part, pref, state_in, state_out, ws, st);
-    if (ev) cudaEventRecord(ev[2], st);
-    launch_pdl(lcla::tc::pass_c_tc, grid, dim3(lcla::tc::LayC::NTHREADS), lcla::tc::LayC::BYTES, st, mq, mc, ms, mo, p,
-               (const float *)pref, eps, (__nv_bfloat16 *)out, status);
-    if (ev) cudaEventRecord(ev[3], st);
+    if (c) {
+        set_smem(lcla::tc::pass_c_tc, lcla::tc::LayC::BYTES);
+        if (ev) cudaEventRecord(ev[2], st);
+        launch_pdl(lcla::tc::pass_c_tc, grid, dim3(lcla::tc::LayC::NTHREADS), lcla::tc::LayC::BYTES, st, mq, mc,
+                   ms, mo, p, (const float *)pref, eps, (__nv_bfloat16 *)out, status);
+        if (ev) cudaEventRecord(ev[3], st);
+    }
     *rc_out = cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
     return true;
 }
@@ -272,21 +284,22 @@ bool launch_tc(const void *q, const void *k, const void *v, const float *rc, con
 template <typename Tin>
 int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const float *rs,
                const LclaPlan &p, float eps, Tin *out, const float *state_in, float *state_out,
-               unsigned char *ws, cudaStream_t st, cudaEvent_t const *ev)
+               unsigned char *ws, cudaStream_t st, cudaEvent_t const *ev, Phase ph)
 {
     using G = lcla::Geo<Tin>;
     float *part = reinterpret_cast<float *>(ws + p.part_off);
     float *pref = reinterpret_cast<float *>(ws + p.pref_off);
     const dim3 grid(p.nseg * p.ngroups, p.B);
-    cudaMemsetAsync(ws, 0, sizeof(int), st);   // status word (no CUDA-core kernel sets it)
-
-    const int smem_a = 2 * (2 * G::TILE_IN + 2 * G::TILE_TAB) + G::TILE_F;
-    set_smem(lcla::pass_a_ffma<Tin>, smem_a);
-    if (ev) cudaEventRecord(ev[0], st);
-    lcla::pass_a_ffma<Tin><<<grid, 256, smem_a, st>>>(k, v, rc, rs, p, part);
-
-    if (ev) cudaEventRecord(ev[1], st);
+    if (ph != PH_END) {
+        cudaMemsetAsync(ws, 0, sizeof(int), st);   // status word (no CUDA-core kernel sets it)
+        const int smem_a = 2 * (2 * G::TILE_IN + 2 * G::TILE_TAB) + G::TILE_F;
+        set_smem(lcla::pass_a_ffma<Tin>, smem_a);
+        if (ev) cudaEventRecord(ev[0], st);
+        lcla::pass_a_ffma<Tin><<<grid, 256, smem_a, st>>>(k, v, rc, rs, p, part);
+        if (ev) cudaEventRecord(ev[1], st);
+    }
     launch_scan(p, part, pref, state_in, state_out, ws, st);
+    if (ph == PH_BEGIN) return cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
     if (ev) cudaEventRecord(ev[2], st);
 
     if (!p.chunk) {
@@ -305,23 +318,23 @@ int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const 
     return cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
 }
 
-// Shared body of lcla_forward and lcla_step once the arguments are checked.
+// Shared body of every entry point once the arguments are checked.
 int run(const void *q, const void *k, const void *v, const float *rc, const float *rs,
         const LclaPlan &p, float eps, void *out, const float *state_in, float *state_out,
-        void *ws, cudaStream_t st, cudaEvent_t const *ev = nullptr)
+        void *ws, cudaStream_t st, cudaEvent_t const *ev = nullptr, Phase ph = PH_ALL)
 {
     if (p.tc) {
         int status = LCLA_OK;
-        if (launch_tc(q, k, v, rc, rs, p, eps, out, state_in, state_out, (unsigned char *)ws, st, ev, &status))
+        if (launch_tc(q, k, v, rc, rs, p, eps, out, state_in, state_out, (unsigned char *)ws, st, ev, &status, ph))
             return status;
     }
     if (p.dtype == LCLA_BF16)
         return launch_all<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
                                          (const __nv_bfloat16 *)v, rc, rs, p, eps,
                                          (__nv_bfloat16 *)out, state_in, state_out,
-                                         (unsigned char *)ws, st, ev);
+                                         (unsigned char *)ws, st, ev, ph);
     return launch_all<float>((const float *)q, (const float *)k, (const float *)v, rc, rs, p, eps,
-                             (float *)out, state_in, state_out, (unsigned char *)ws, st, ev);
+                             (float *)out, state_in, state_out, (unsigned char *)ws, st, ev, ph);
 }
 
 // Pointer, alignment, overlap and workspace checks for one call.
@@ -358,6 +371,21 @@ int check_buffers(const void *q, const void *k, const void *v, const float *rc, 
                   overlaps(state, nst, rs, ntab)))
         return LCLA_ERR_INVALID_ARG;
     return LCLA_OK;
+}
+
+// Sequence sharding keeps the forward's workspace and, after it, the rank's
+// carried-in state (one [B, H, d+1, d] fp32 slice).
+size_t shard_ws_bytes(const LclaPlan &p)
+{
+    return p.N == 0 ? 0 : p.ws_bytes + round_up((size_t)p.B * p.H * LCLA_SZ * sizeof(float));
+}
+
+void launch_combine(const float *totals, int nranks, int rank, const float *state_in, float *carry,
+                    float *state_final, int B, int H, cudaStream_t st)
+{
+    const size_t n4 = (size_t)B * H * (LCLA_SZ / lcla::SCAN_VEC);
+    lcla::combine_rank_totals<<<(unsigned)((n4 + lcla::SCAN_THREADS - 1) / lcla::SCAN_THREADS), lcla::SCAN_THREADS,
+                                0, st>>>(totals, nranks, rank, n4, state_in, carry, state_final);
 }
 
 }  // namespace
@@ -442,6 +470,80 @@ int lcla_forward_blocks(const void *q, const void *k, const void *v, const float
     }
     p.boff = block_offsets;
     return run(q, k, v, rope_cos, rope_sin, p, eps, out, nullptr, state_out, workspace, st, nullptr);
+}
+
+size_t lcla_shard_workspace_bytes(int B, int H, int N, int d, int block_len, int dtype)
+{
+    if (check_shape(B, H, N, d, block_len, dtype) != LCLA_OK) return 0;
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    return grid_fits(p) ? shard_ws_bytes(p) : 0;
+}
+
+int lcla_shard_begin(const void *k, const void *v, const float *rope_cos, const float *rope_sin, int B, int H,
+                     int N, int d, int block_len, float *total_out, int dtype, void *workspace,
+                     size_t workspace_bytes, void *stream)
+{
+    int rc = check_shape(B, H, N, d, block_len, dtype);
+    if (rc != LCLA_OK) return rc;
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
+    if (!total_out) return LCLA_ERR_INVALID_ARG;
+    if (misaligned(total_out)) return LCLA_ERR_MISALIGNED;
+    const size_t nst = (size_t)B * H * LCLA_SZ * sizeof(float);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) return cudaMemsetAsync(total_out, 0, nst, st) == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
+    if (!k || !v || !rope_cos || !rope_sin) return LCLA_ERR_INVALID_ARG;
+    if (misaligned(k) || misaligned(v) || misaligned(rope_cos) || misaligned(rope_sin) ||
+        (workspace && misaligned(workspace)))
+        return LCLA_ERR_MISALIGNED;
+    const size_t need = shard_ws_bytes(p);
+    if (!workspace || workspace_bytes < need) return LCLA_ERR_WORKSPACE;
+    const size_t nio = (size_t)B * N * H * LCLA_D * (dtype == LCLA_BF16 ? 2 : 4);
+    const size_t ntab = (size_t)N * (LCLA_D / 2) * sizeof(float);
+    const void *reads[4] = {k, v, rope_cos, rope_sin};
+    const size_t rlen[4] = {nio, nio, ntab, ntab};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(total_out, nst, reads[i], rlen[i]) || overlaps(workspace, need, reads[i], rlen[i]))
+            return LCLA_ERR_INVALID_ARG;
+    if (overlaps(total_out, nst, workspace, need)) return LCLA_ERR_INVALID_ARG;
+    return run(nullptr, k, v, rope_cos, rope_sin, p, 0.f, nullptr, nullptr, total_out, workspace, st, nullptr,
+               PH_BEGIN);
+}
+
+int lcla_shard_end(const void *q, const void *k, const void *v, const float *rope_cos, const float *rope_sin,
+                   int B, int H, int N, int d, int block_len, float eps, const float *totals, int nranks, int rank,
+                   const float *state_in, void *out, float *state_out, int dtype, void *workspace,
+                   size_t workspace_bytes, void *stream)
+{
+    int rc = check_shape(B, H, N, d, block_len, dtype);
+    if (rc != LCLA_OK) return rc;
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
+    if (nranks < 1 || rank < 0 || rank >= nranks || !totals) return LCLA_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !isfinite(eps)) return LCLA_ERR_INVALID_ARG;
+    if (misaligned(totals) || (state_in && misaligned(state_in)) || (state_out && misaligned(state_out)))
+        return LCLA_ERR_MISALIGNED;
+    const size_t nst = (size_t)B * H * LCLA_SZ * sizeof(float);
+    const size_t ntot = nst * (size_t)nranks;
+    // state_out may be state_in itself, but no other overlap with the states it is summed from
+    if (overlaps(state_out, nst, totals, ntot) || (state_in != state_out && overlaps(state_out, nst, state_in, nst)))
+        return LCLA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        if (state_out) launch_combine(totals, nranks, rank, state_in, nullptr, state_out, B, H, st);
+        return cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
+    }
+    const size_t need = shard_ws_bytes(p);
+    rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, dtype, eps, workspace,
+                       workspace_bytes, need);
+    if (rc != LCLA_OK) return rc;
+    const size_t nio = (size_t)B * N * H * LCLA_D * (dtype == LCLA_BF16 ? 2 : 4);
+    if (overlaps(out, nio, totals, ntot) || overlaps(workspace, need, totals, ntot) ||
+        overlaps(out, nio, state_in, nst) || overlaps(workspace, need, state_in, nst))
+        return LCLA_ERR_INVALID_ARG;
+    float *carry = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + p.ws_bytes);
+    launch_combine(totals, nranks, rank, state_in, carry, state_out, B, H, st);
+    return run(q, k, v, rope_cos, rope_sin, p, eps, out, carry, nullptr, workspace, st, nullptr, PH_END);
 }
 
 int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk, const float *cos_blk,

@@ -175,6 +175,75 @@ LCLA_API int lcla_temporal_conv(const void *x, int B, int F, int S, int C,
                  const float *weight, const float *bias, void *cache, int save,
                  void *y, int dtype, void *stream);
 
+/*
+ * Sequence-sharded forward, in two calls per rank with one exchange between
+ * them.  The pages carry one fixed-size cumulative state from earlier blocks
+ * to later ones ("Block Causal Linear Attention", introduction and section
+ * "What SANA-Video Actually Uses": a block needs only the cumulative
+ * attention state and key summary of the blocks before it), so a sequence
+ * cut into runs of whole blocks, one per rank, needs from the ranks before
+ * it only the sum of their states.  Rank r of R holds tokens
+ * [t_r, t_{r+1}) with t_r a multiple of block_len (the last rank may end in
+ * a ragged block), the tables' rows at those absolute positions, and N =
+ * t_{r+1} - t_r >= 0 (a rank may hold no tokens).
+ *
+ *   1. lcla_shard_begin: the state total (S, z summed over the rank's tokens,
+ *      [B, H, d+1, d] fp32) into total_out.
+ *   2. The caller gathers the R totals in rank order into one device array
+ *      [R][B, H, d+1, d] (one all-gather of B*H*(d+1)*d*4 bytes per rank).
+ *   3. lcla_shard_end: the rank's outputs, each block using state_in plus the
+ *      totals of ranks 0..r-1 plus its own blocks; and, if state_out is not
+ *      NULL, the state after the whole sequence, state_in plus all R totals,
+ *      summed in rank order so that every rank writes the same bits.
+ *
+ * The outputs equal those of lcla_forward on the whole sequence with
+ * state_in added to every block's state, up to the order of fp32 additions.
+ * Both calls take the same B, H, N, d, block_len, dtype and the same
+ * workspace, whose contents lcla_shard_end reads (pass A's partial states):
+ * nothing else may use it in between.  A mismatch is not detected and gives
+ * wrong outputs.
+ */
+LCLA_API size_t lcla_shard_workspace_bytes(int B, int H, int N, int d, int block_len, int dtype);
+
+/*
+ *   k, v         [B, N, H, d] device, dtype: the rank's tokens.  Read only.
+ *   rope_cos/sin [N, d/2] float32 device, rows at the tokens' absolute
+ *                positions.  Read only.
+ *   total_out    [B, H, d+1, d] float32 device.  Written (zeros when N = 0).
+ *   workspace    at least lcla_shard_workspace_bytes(...) bytes, 16-byte
+ *                aligned; it must not overlap the other arrays.
+ * Returns an lcla_status.
+ */
+LCLA_API int lcla_shard_begin(const void *k, const void *v,
+                 const float *rope_cos, const float *rope_sin,
+                 int B, int H, int N, int d, int block_len,
+                 float *total_out, int dtype,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ *   q, k, v      [B, N, H, d] device, dtype: the rank's tokens (k and v as
+ *                given to lcla_shard_begin; they are read again only when
+ *                block_len < 64).  Read only.
+ *   rope_cos/sin as for lcla_shard_begin.
+ *   totals       [nranks][B, H, d+1, d] float32 device: every rank's
+ *                total_out, in rank order.  Read only.
+ *   nranks >= 1, 0 <= rank < nranks.
+ *   state_in     [B, H, d+1, d] float32 device, or NULL (zero): the state
+ *                before the whole sequence.  Read only.
+ *   out          [B, N, H, d] device, dtype.  Written.
+ *   state_out    [B, H, d+1, d] float32 device, or NULL.  Written with the
+ *                state after the whole sequence; may be state_in itself, but
+ *                must not otherwise overlap it or totals.
+ *   workspace    the one lcla_shard_begin used, unchanged since.
+ * With N = 0 only state_out is written.  Returns an lcla_status.
+ */
+LCLA_API int lcla_shard_end(const void *q, const void *k, const void *v,
+                 const float *rope_cos, const float *rope_sin,
+                 int B, int H, int N, int d, int block_len, float eps,
+                 const float *totals, int nranks, int rank, const float *state_in,
+                 void *out, float *state_out, int dtype,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
 /* Workspace bytes lcla_step needs (0 when the arguments are invalid). */
 LCLA_API size_t lcla_step_workspace_bytes(int B, int H, int L, int d, int dtype);
 

@@ -22,7 +22,8 @@ def test_every_declared_symbol_is_exported():
     names = declared_symbols()
     assert {"lcla_forward", "lcla_step", "lcla_forward_workspace_bytes",
             "lcla_step_workspace_bytes", "lcla_status_string", "lcla_version",
-            "lcla_forward_blocks", "lcla_forward_blocks_workspace_bytes", "lcla_temporal_conv"} <= set(names)
+            "lcla_forward_blocks", "lcla_forward_blocks_workspace_bytes", "lcla_temporal_conv",
+            "lcla_shard_begin", "lcla_shard_end", "lcla_shard_workspace_bytes"} <= set(names)
     lib = ctypes.CDLL(lcla.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -140,3 +141,37 @@ def test_temporal_conv_arguments():
     assert fn(a, 1, 2, 3, 16, 2 * a, None, a + 64, 0, 3 * a, lcla.BF16, None) == 1     # cache inside x
     assert fn(a, 1, 0, 3, 16, 2 * a, None, None, 0, 3 * a, lcla.BF16, None) == 0       # no frames: nothing to do
     assert fn(None, 1, 2, 3, 16, 2 * a, None, None, 0, 3 * a, lcla.BF16, None) == 1    # x missing
+
+
+def test_shard_workspace_and_arguments():
+    f = lcla.shard_workspace_bytes
+    # the forward's workspace plus one [B, H, d+1, d] fp32 carry slice
+    assert f(1, 70, 18720, 32, 4680, lcla.BF16) == \
+        lcla.forward_workspace_bytes(1, 70, 18720, 32, 4680, lcla.BF16) + 70 * 33 * 32 * 4
+    assert f(1, 4, 0, 32, 16, lcla.BF16) == 0            # an empty shard needs nothing
+    assert f(1, 4, 100, 64, 16, lcla.BF16) == 0          # d = 64 not served
+    a = 1 << 20
+    begin, end = lcla.lib.lcla_shard_begin, lcla.lib.lcla_shard_end
+    # argument errors return before any launch (no device memory is touched)
+    assert begin(a, 2 * a, 3 * a, 4 * a, 1, 4, 100, 32, 16, None, 0, 8 * a, 1 << 20, None) == INVALID
+    assert begin(a, 2 * a, 3 * a, 4 * a, 1, 4, 100, 32, 16, 5 * a + 4, 0, 8 * a, 1 << 20, None) == MISALIGNED
+    assert begin(a, 2 * a, 3 * a, 4 * a, 1, 4, 100, 32, 16, 5 * a, 0, None, 0, None) == WORKSPACE
+    assert begin(a, 2 * a, 3 * a, 4 * a, 1, 4, 100, 32, 16, a + 64, 0, 8 * a, 1 << 20, None) == INVALID  # total in k
+    assert begin(None, 2 * a, 3 * a, 4 * a, 1, 4, 100, 32, 16, 5 * a, 0, 8 * a, 1 << 20, None) == INVALID
+    assert begin(a, 2 * a, 3 * a, 4 * a, 1, 4, 100, 48, 16, 5 * a, 0, 8 * a, 1 << 20, None) == UNSUPPORTED
+
+    def e(**kw):
+        args = dict(q=a, k=2 * a, v=3 * a, c=4 * a, s=5 * a, B=1, H=4, N=100, d=32, L=16, eps=1e-8,
+                    tot=6 * a, R=2, r=1, sin=None, out=7 * a, sout=None, dtype=0, ws=8 * a, wsb=1 << 20)
+        args.update(kw)
+        return end(*args.values(), None)
+    assert e(R=0, r=0) == INVALID                        # no ranks
+    assert e(r=2) == INVALID                             # rank out of range
+    assert e(r=-1) == INVALID
+    assert e(tot=None) == INVALID                        # totals missing
+    assert e(tot=6 * a + 8) == MISALIGNED
+    assert e(eps=-1.0) == INVALID
+    assert e(sout=6 * a + 256) == INVALID                # final state inside the totals
+    assert e(sin=9 * a, sout=9 * a + 128) == INVALID     # partial overlap of state_in and state_out
+    assert e(ws=None, wsb=0) == WORKSPACE
+    assert e(out=6 * a) == INVALID                       # out over the totals
