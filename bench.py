@@ -39,7 +39,6 @@ from workloads import NAMED, make_inputs  # noqa: E402
 METRIC = "attended tokens*heads/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
 UNIT = "token*heads/s"
 L2_BYTES = 126 * 1024 * 1024
-STATE_BYTES = 33 * 32 * 4
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -395,9 +394,9 @@ def run_seq(args):
     c, s = to_dev(inp.rope_cos[t0:t1]), to_dev(inp.rope_sin[t0:t1])
     code = lcla.BF16 if spec.dtype == "bf16" else lcla.F32
     out = torch.empty_like(q)
-    st = torch.empty((spec.B, spec.H, 33, 32), dtype=torch.float32, device=device)
+    st = torch.empty((spec.B, spec.H, spec.d + 1, spec.d), dtype=torch.float32, device=device)
     total = torch.empty_like(st)
-    ws = torch.empty(max(1, lcla.shard_workspace_bytes(spec.B, spec.H, Nr, 32, spec.block_len, code)),
+    ws = torch.empty(max(1, lcla.shard_workspace_bytes(spec.B, spec.H, Nr, spec.d, spec.block_len, code)),
                      dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
@@ -425,7 +424,7 @@ def run_seq(args):
     barrier()
     ms_total = ranks.max(e0.elapsed_time(e1))
     ms = ms_total / K
-    plan = lcla.plan_info(spec.B, spec.H, max(Nr, 1), 32, spec.block_len, code)
+    plan = lcla.plan_info(spec.B, spec.H, max(Nr, 1), spec.d, spec.block_len, code)
     esz = spec.elem_bytes
     local_bytes = 4 * spec.B * Nr * spec.H * spec.d * esz + 2 * 2 * Nr * (spec.d // 2) * 4
     slowest_bytes = ranks.max(float(local_bytes))
@@ -436,7 +435,7 @@ def run_seq(args):
         scan_k = 1 if ngroups <= 256 else 2
         cfg = workload_config(spec, world)
         cfg["parallelism"] = (f"sequence sharded over {world} rank(s): whole blocks per rank, "
-                              f"one all-gather of {spec.B * spec.H * STATE_BYTES} B per rank per step")
+                              f"one all-gather of {spec.B * spec.H * (spec.d + 1) * spec.d * 4} B per rank per step")
         line = {"metric": METRIC, "value": spec.token_heads / (ms / 1e3), "unit": UNIT, "n_gpus": world,
                 "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
                 "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic (seeded)", "config": cfg,
@@ -488,8 +487,8 @@ def main():
     q, k, v, c, s = (to_dev(a) for a in (inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin))
     code = lcla.BF16 if spec.dtype == "bf16" else lcla.F32
     out = torch.empty_like(q)
-    st = torch.empty((spec.B, spec.H, 33, 32), dtype=torch.float32, device=device)
-    ws = torch.empty(max(1, lcla.forward_workspace_bytes(spec.B, spec.H, spec.N, 32,
+    st = torch.empty((spec.B, spec.H, spec.d + 1, spec.d), dtype=torch.float32, device=device)
+    ws = torch.empty(max(1, lcla.forward_workspace_bytes(spec.B, spec.H, spec.N, spec.d,
                                                          spec.block_len, code)),
                      dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
@@ -534,9 +533,9 @@ def main():
     esz = spec.elem_bytes
     tok_bytes = spec.B * spec.N * spec.H * spec.d * esz             # one [B, N, H, d] tensor
     tab_bytes = 2 * spec.N * (spec.d // 2) * 4
-    plan = lcla.plan_info(spec.B, spec.H, spec.N, 32, spec.block_len, code)
+    plan = lcla.plan_info(spec.B, spec.H, spec.N, spec.d, spec.block_len, code)
     nseg, npref = plan["segments"], plan["prefixes"]
-    sl = spec.B * spec.H * STATE_BYTES
+    sl = spec.B * spec.H * (spec.d + 1) * spec.d * 4
     bytes_a = 2 * tok_bytes + tab_bytes + nseg * sl
     bytes_c = 2 * tok_bytes + tab_bytes + npref * sl
     bytes_s = nseg * sl + npref * sl + sl
@@ -546,6 +545,8 @@ def main():
         else "scan_chunk_totals+scan_chunk_prefix"
     if plan["tensor_cores"]:
         name_a, name_c = "pass_a_tc", "pass_c_tc"
+    elif spec.d != 32:
+        name_a, name_c = "pass_a_gen", "pass_c_gen"
     else:
         name_a, name_c = "pass_a_ffma", "pass_c_chunk_ffma" if plan["chunk_mode"] else "pass_c_ffma"
     passes = {"pass_a": (statistics.mean(pa), bytes_a, name_a),

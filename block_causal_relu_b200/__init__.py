@@ -18,11 +18,12 @@ import torch
 __all__ = ["forward", "step", "forward_workspace_bytes", "step_workspace_bytes", "plan_info",
            "forward_blocks", "forward_blocks_workspace_bytes", "temporal_conv",
            "shard_begin", "shard_end", "shard_workspace_bytes",
-           "LclaError", "LIB_PATH", "lib", "BF16", "F32", "D"]
+           "LclaError", "LIB_PATH", "lib", "BF16", "F32", "D", "HEAD_DIMS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblcla.so")
 BF16, F32 = 0, 1
-D = 32
+D = 32                 # head dim of the tensor-core path
+HEAD_DIMS = (32, 64)   # head dims the library serves
 DEFAULT_EPS = 1e-8
 
 

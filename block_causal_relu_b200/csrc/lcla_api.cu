@@ -15,6 +15,7 @@
 
 #include "lcla.h"
 #include "lcla_ffma.cuh"
+#include "lcla_gen.cuh"
 #include "lcla_plan.h"
 #include "lcla_shard.cuh"
 #include "lcla_tc.cuh"
@@ -30,7 +31,8 @@ int check_shape(int B, int H, int N, int d, int L, int dtype)
     if (B < 1 || H < 1 || N < 0 || d < 1 || L < 1) return LCLA_ERR_INVALID_ARG;
     if (dtype != LCLA_BF16 && dtype != LCLA_F32) return LCLA_ERR_INVALID_ARG;
     if (d & 1) return LCLA_ERR_INVALID_ARG;
-    if (d != LCLA_D) return LCLA_ERR_UNSUPPORTED;
+    if (d != LCLA_D && d != LCLA_D_WIDE) return LCLA_ERR_UNSUPPORTED;
+    if (d == LCLA_D_WIDE && H > 65535) return LCLA_ERR_UNSUPPORTED;   // grid y of the d = 64 kernels
     if (N > (1 << 30)) return LCLA_ERR_UNSUPPORTED;
     if (B > 65535) return LCLA_ERR_UNSUPPORTED;
     if ((long long)B * H > 0x7fffffffLL) return LCLA_ERR_UNSUPPORTED;
@@ -41,20 +43,23 @@ int check_shape(int B, int H, int N, int d, int L, int dtype)
 // [status word, 256 B][part: nseg x B x H x (d+1) x d fp32][pref: npref x B x H x (d+1) x d fp32]
 // [chunk totals of the scan, when it runs in chunks].  nblocks > 0: that many explicit blocks (their
 // offsets are read on the device), always in block mode, sized by their mean length.
-LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0)
+LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0, int d = LCLA_D)
 {
     LclaPlan p;
     memset(&p, 0, sizeof p);
     if (nblocks > 0 && N > 0) L = (int)(((long long)N + nblocks - 1) / nblocks);
     p.B = B; p.H = H; p.N = N; p.L = L; p.dtype = dtype;
+    p.d = d; p.sz = (d + 1) * d;
     p.ngroups = (H + LCLA_HG - 1) / LCLA_HG;
     p.nquads = (H + LCLA_TC_HQ - 1) / LCLA_TC_HQ;
     if (N == 0) return p;
     p.nb = nblocks > 0 ? nblocks : (int)(((long long)N + L - 1) / L);
-    const long long units = (long long)p.ngroups * B;
-    if (nblocks > 0 || L >= LCLA_T) {
+    // CUDA-core CTAs per segment: head pairs at d = 32, single heads at d = 64
+    const long long units = (long long)(d == LCLA_D ? p.ngroups : H) * B;
+    // d = 64 runs in block mode for every block length (its kernels have no chunk mode)
+    if (nblocks > 0 || L >= LCLA_T || d != LCLA_D) {
         p.chunk = 0;
-        p.tc = dtype == LCLA_BF16;
+        p.tc = dtype == LCLA_BF16 && d == LCLA_D;
         p.T = p.tc ? LCLA_TC_T : LCLA_T;
         const long long tpb = ((long long)(L < N ? L : N) + p.T - 1) / p.T;   // tiles per full block
         long long nsb;
@@ -107,7 +112,7 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0)
         p.scs = lcla::SCAN_CHUNK_GROUPS * (p.chunk ? 1 : p.nsb);
         p.nch = (p.nseg + p.scs - 1) / p.scs;
     }
-    const size_t slice = (size_t)B * H * LCLA_SZ * sizeof(float);
+    const size_t slice = (size_t)B * H * p.sz * sizeof(float);
     p.part_off = kAlign;
     p.pref_off = p.part_off + round_up((size_t)p.nseg * slice);
     p.ctot_off = p.pref_off + round_up((size_t)p.npref * slice);
@@ -122,7 +127,10 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0)
 enum Phase { PH_ALL, PH_BEGIN, PH_END };
 
 // The launch grid flattens (segment, head group) into blockIdx.x.
-bool grid_fits(const LclaPlan &p) { return (long long)p.nseg * p.ngroups <= 0x7fffffffLL; }
+bool grid_fits(const LclaPlan &p)
+{
+    return (long long)p.nseg * (p.d == LCLA_D ? p.ngroups : 1) <= 0x7fffffffLL;
+}
 
 bool misaligned(const void *ptr) { return ((uintptr_t)ptr & 15u) != 0; }
 
@@ -154,7 +162,7 @@ void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
 
 unsigned scan_blocks(const LclaPlan &p)
 {
-    const size_t n = (size_t)p.B * p.H * (LCLA_SZ / lcla::SCAN_VEC);
+    const size_t n = (size_t)p.B * p.H * (p.sz / lcla::SCAN_VEC);
     return (unsigned)((n + lcla::SCAN_THREADS - 1) / lcla::SCAN_THREADS);
 }
 
@@ -165,7 +173,7 @@ void launch_scan(const LclaPlan &p, const float *part, float *pref, const float 
 {
     if (p.nch == 0) {
         const int ngroups = p.chunk ? p.nseg : p.nb;
-        const size_t n4 = (size_t)p.B * p.H * (LCLA_SZ / lcla::SCAN_VEC);
+        const size_t n4 = (size_t)p.B * p.H * (p.sz / lcla::SCAN_VEC);
         const int smem = ngroups * 32 * 16;
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(lcla::scan_states_grouped, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -318,11 +326,44 @@ int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const 
     return cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
 }
 
+// Head dim 64: the generic CUDA-core passes (block mode), one CTA per (segment, head, batch entry).
+template <typename Tin>
+int launch_gen(const Tin *q, const Tin *k, const Tin *v, const float *rc, const float *rs, const LclaPlan &p,
+               float eps, Tin *out, const float *state_in, float *state_out, unsigned char *ws, cudaStream_t st,
+               cudaEvent_t const *ev, Phase ph)
+{
+    float *part = reinterpret_cast<float *>(ws + p.part_off);
+    float *pref = reinterpret_cast<float *>(ws + p.pref_off);
+    const dim3 grid(p.nseg, p.H, p.B);
+    if (ph != PH_END) {
+        cudaMemsetAsync(ws, 0, sizeof(int), st);   // status word (no CUDA-core kernel sets it)
+        if (ev) cudaEventRecord(ev[0], st);
+        lcla::gen::pass_a_gen<Tin, LCLA_D_WIDE><<<grid, lcla::gen::THREADS, 0, st>>>(k, v, rc, rs, p, part);
+        if (ev) cudaEventRecord(ev[1], st);
+    }
+    launch_scan(p, part, pref, state_in, state_out, ws, st);
+    if (ph != PH_BEGIN) {
+        if (ev) cudaEventRecord(ev[2], st);
+        launch_pdl(lcla::gen::pass_c_gen<Tin, LCLA_D_WIDE>, grid, dim3(lcla::gen::THREADS), 0, st, q, rc, rs, p,
+                   (const float *)pref, eps, out);
+        if (ev) cudaEventRecord(ev[3], st);
+    }
+    return cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
+}
+
 // Shared body of every entry point once the arguments are checked.
 int run(const void *q, const void *k, const void *v, const float *rc, const float *rs,
         const LclaPlan &p, float eps, void *out, const float *state_in, float *state_out,
         void *ws, cudaStream_t st, cudaEvent_t const *ev = nullptr, Phase ph = PH_ALL)
 {
+    if (p.d != LCLA_D) {
+        if (p.dtype == LCLA_BF16)
+            return launch_gen<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                             (const __nv_bfloat16 *)v, rc, rs, p, eps, (__nv_bfloat16 *)out,
+                                             state_in, state_out, (unsigned char *)ws, st, ev, ph);
+        return launch_gen<float>((const float *)q, (const float *)k, (const float *)v, rc, rs, p, eps,
+                                 (float *)out, state_in, state_out, (unsigned char *)ws, st, ev, ph);
+    }
     if (p.tc) {
         int status = LCLA_OK;
         if (launch_tc(q, k, v, rc, rs, p, eps, out, state_in, state_out, (unsigned char *)ws, st, ev, &status, ph))
@@ -340,7 +381,7 @@ int run(const void *q, const void *k, const void *v, const float *rc, const floa
 // Pointer, alignment, overlap and workspace checks for one call.
 int check_buffers(const void *q, const void *k, const void *v, const float *rc, const float *rs,
                   const void *out, const float *state, bool state_required, int B, int H, int N,
-                  int dtype, float eps, const void *ws, size_t ws_bytes, size_t need)
+                  int d, int dtype, float eps, const void *ws, size_t ws_bytes, size_t need)
 {
     if (!(eps >= 0.f) || !isfinite(eps)) return LCLA_ERR_INVALID_ARG;
     if (state_required && !state) return LCLA_ERR_INVALID_ARG;
@@ -353,9 +394,9 @@ int check_buffers(const void *q, const void *k, const void *v, const float *rc, 
         misaligned(out) || (state && misaligned(state)) || (ws && misaligned(ws)))
         return LCLA_ERR_MISALIGNED;
     const size_t esz = dtype == LCLA_BF16 ? 2 : 4;
-    const size_t nio = (size_t)B * N * H * LCLA_D * esz;
-    const size_t ntab = (size_t)N * (LCLA_D / 2) * sizeof(float);
-    const size_t nst = (size_t)B * H * LCLA_SZ * sizeof(float);
+    const size_t nio = (size_t)B * N * H * d * esz;
+    const size_t ntab = (size_t)N * (d / 2) * sizeof(float);
+    const size_t nst = (size_t)B * H * (d + 1) * d * sizeof(float);
     if (overlaps(out, nio, q, nio) || overlaps(out, nio, k, nio) || overlaps(out, nio, v, nio) ||
         overlaps(out, nio, rc, ntab) || overlaps(out, nio, rs, ntab) ||
         overlaps(out, nio, state, nst) || overlaps(out, nio, ws, ws_bytes))
@@ -377,13 +418,13 @@ int check_buffers(const void *q, const void *k, const void *v, const float *rc, 
 // carried-in state (one [B, H, d+1, d] fp32 slice).
 size_t shard_ws_bytes(const LclaPlan &p)
 {
-    return p.N == 0 ? 0 : p.ws_bytes + round_up((size_t)p.B * p.H * LCLA_SZ * sizeof(float));
+    return p.N == 0 ? 0 : p.ws_bytes + round_up((size_t)p.B * p.H * p.sz * sizeof(float));
 }
 
 void launch_combine(const float *totals, int nranks, int rank, const float *state_in, float *carry,
-                    float *state_final, int B, int H, cudaStream_t st)
+                    float *state_final, int B, int H, int d, cudaStream_t st)
 {
-    const size_t n4 = (size_t)B * H * (LCLA_SZ / lcla::SCAN_VEC);
+    const size_t n4 = (size_t)B * H * ((d + 1) * d / lcla::SCAN_VEC);
     lcla::combine_rank_totals<<<(unsigned)((n4 + lcla::SCAN_THREADS - 1) / lcla::SCAN_THREADS), lcla::SCAN_THREADS,
                                 0, st>>>(totals, nranks, rank, n4, state_in, carry, state_final);
 }
@@ -395,14 +436,14 @@ extern "C" {
 size_t lcla_forward_workspace_bytes(int B, int H, int N, int d, int block_len, int dtype)
 {
     if (check_shape(B, H, N, d, block_len, dtype) != LCLA_OK) return 0;
-    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype, 0, d);
     return grid_fits(p) ? p.ws_bytes : 0;
 }
 
 size_t lcla_step_workspace_bytes(int B, int H, int L, int d, int dtype)
 {
     if (check_shape(B, H, L, d, L < 1 ? 1 : L, dtype) != LCLA_OK) return 0;
-    const LclaPlan p = make_plan(B, H, L, L < 1 ? 1 : L, dtype);
+    const LclaPlan p = make_plan(B, H, L, L < 1 ? 1 : L, dtype, 0, d);
     return grid_fits(p) ? p.ws_bytes : 0;
 }
 
@@ -413,9 +454,9 @@ int lcla_forward_timed(const void *q, const void *k, const void *v, const float 
 {
     int rc = check_shape(B, H, N, d, block_len, dtype);
     if (rc != LCLA_OK) return rc;
-    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype, 0, d);
     if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
-    rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, dtype, eps,
+    rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, d, dtype, eps,
                        workspace, workspace_bytes, p.ws_bytes);
     if (rc != LCLA_OK) return rc;
     if (events && (!events[0] || !events[1] || !events[2] || !events[3])) return LCLA_ERR_INVALID_ARG;
@@ -423,7 +464,7 @@ int lcla_forward_timed(const void *q, const void *k, const void *v, const float 
     cudaEvent_t const *ev = reinterpret_cast<cudaEvent_t const *>(events);
     if (N == 0) {
         if (ev) cudaEventRecord(ev[0], st);
-        if (state_out && cudaMemsetAsync(state_out, 0, (size_t)B * H * LCLA_SZ * sizeof(float), st) != cudaSuccess)
+        if (state_out && cudaMemsetAsync(state_out, 0, (size_t)B * H * (d + 1) * d * sizeof(float), st) != cudaSuccess)
             return LCLA_ERR_CUDA;
         if (ev) { cudaEventRecord(ev[1], st); cudaEventRecord(ev[2], st); cudaEventRecord(ev[3], st); }
         return LCLA_OK;
@@ -444,7 +485,7 @@ size_t lcla_forward_blocks_workspace_bytes(int B, int H, int N, int d, int nbloc
 {
     if (check_shape(B, H, N, d, 1, dtype) != LCLA_OK) return 0;
     if (N > 0 && (nblocks < 1 || nblocks > N)) return 0;
-    const LclaPlan p = make_plan(B, H, N, 1, dtype, nblocks);
+    const LclaPlan p = make_plan(B, H, N, 1, dtype, nblocks, d);
     return grid_fits(p) ? p.ws_bytes : 0;
 }
 
@@ -457,14 +498,14 @@ int lcla_forward_blocks(const void *q, const void *k, const void *v, const float
     if (rc != LCLA_OK) return rc;
     if (N > 0 && (nblocks < 1 || nblocks > N || !block_offsets)) return LCLA_ERR_INVALID_ARG;
     if (N > 0 && ((uintptr_t)block_offsets & 3u)) return LCLA_ERR_MISALIGNED;
-    LclaPlan p = make_plan(B, H, N, 1, dtype, nblocks);
+    LclaPlan p = make_plan(B, H, N, 1, dtype, nblocks, d);
     if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
-    rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, dtype, eps, workspace,
+    rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, d, dtype, eps, workspace,
                        workspace_bytes, p.ws_bytes);
     if (rc != LCLA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (N == 0) {
-        if (state_out && cudaMemsetAsync(state_out, 0, (size_t)B * H * LCLA_SZ * sizeof(float), st) != cudaSuccess)
+        if (state_out && cudaMemsetAsync(state_out, 0, (size_t)B * H * (d + 1) * d * sizeof(float), st) != cudaSuccess)
             return LCLA_ERR_CUDA;
         return LCLA_OK;
     }
@@ -475,7 +516,7 @@ int lcla_forward_blocks(const void *q, const void *k, const void *v, const float
 size_t lcla_shard_workspace_bytes(int B, int H, int N, int d, int block_len, int dtype)
 {
     if (check_shape(B, H, N, d, block_len, dtype) != LCLA_OK) return 0;
-    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype, 0, d);
     return grid_fits(p) ? shard_ws_bytes(p) : 0;
 }
 
@@ -485,11 +526,11 @@ int lcla_shard_begin(const void *k, const void *v, const float *rope_cos, const 
 {
     int rc = check_shape(B, H, N, d, block_len, dtype);
     if (rc != LCLA_OK) return rc;
-    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype, 0, d);
     if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
     if (!total_out) return LCLA_ERR_INVALID_ARG;
     if (misaligned(total_out)) return LCLA_ERR_MISALIGNED;
-    const size_t nst = (size_t)B * H * LCLA_SZ * sizeof(float);
+    const size_t nst = (size_t)B * H * (d + 1) * d * sizeof(float);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (N == 0) return cudaMemsetAsync(total_out, 0, nst, st) == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
     if (!k || !v || !rope_cos || !rope_sin) return LCLA_ERR_INVALID_ARG;
@@ -498,8 +539,8 @@ int lcla_shard_begin(const void *k, const void *v, const float *rope_cos, const 
         return LCLA_ERR_MISALIGNED;
     const size_t need = shard_ws_bytes(p);
     if (!workspace || workspace_bytes < need) return LCLA_ERR_WORKSPACE;
-    const size_t nio = (size_t)B * N * H * LCLA_D * (dtype == LCLA_BF16 ? 2 : 4);
-    const size_t ntab = (size_t)N * (LCLA_D / 2) * sizeof(float);
+    const size_t nio = (size_t)B * N * H * d * (dtype == LCLA_BF16 ? 2 : 4);
+    const size_t ntab = (size_t)N * (d / 2) * sizeof(float);
     const void *reads[4] = {k, v, rope_cos, rope_sin};
     const size_t rlen[4] = {nio, nio, ntab, ntab};
     for (int i = 0; i < 4; ++i)
@@ -517,32 +558,32 @@ int lcla_shard_end(const void *q, const void *k, const void *v, const float *rop
 {
     int rc = check_shape(B, H, N, d, block_len, dtype);
     if (rc != LCLA_OK) return rc;
-    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype, 0, d);
     if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
     if (nranks < 1 || rank < 0 || rank >= nranks || !totals) return LCLA_ERR_INVALID_ARG;
     if (!(eps >= 0.f) || !isfinite(eps)) return LCLA_ERR_INVALID_ARG;
     if (misaligned(totals) || (state_in && misaligned(state_in)) || (state_out && misaligned(state_out)))
         return LCLA_ERR_MISALIGNED;
-    const size_t nst = (size_t)B * H * LCLA_SZ * sizeof(float);
+    const size_t nst = (size_t)B * H * (d + 1) * d * sizeof(float);
     const size_t ntot = nst * (size_t)nranks;
     // state_out may be state_in itself, but no other overlap with the states it is summed from
     if (overlaps(state_out, nst, totals, ntot) || (state_in != state_out && overlaps(state_out, nst, state_in, nst)))
         return LCLA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (N == 0) {
-        if (state_out) launch_combine(totals, nranks, rank, state_in, nullptr, state_out, B, H, st);
+        if (state_out) launch_combine(totals, nranks, rank, state_in, nullptr, state_out, B, H, d, st);
         return cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
     }
     const size_t need = shard_ws_bytes(p);
-    rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, dtype, eps, workspace,
+    rc = check_buffers(q, k, v, rope_cos, rope_sin, out, state_out, false, B, H, N, d, dtype, eps, workspace,
                        workspace_bytes, need);
     if (rc != LCLA_OK) return rc;
-    const size_t nio = (size_t)B * N * H * LCLA_D * (dtype == LCLA_BF16 ? 2 : 4);
+    const size_t nio = (size_t)B * N * H * d * (dtype == LCLA_BF16 ? 2 : 4);
     if (overlaps(out, nio, totals, ntot) || overlaps(workspace, need, totals, ntot) ||
         overlaps(out, nio, state_in, nst) || overlaps(workspace, need, state_in, nst))
         return LCLA_ERR_INVALID_ARG;
     float *carry = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + p.ws_bytes);
-    launch_combine(totals, nranks, rank, state_in, carry, state_out, B, H, st);
+    launch_combine(totals, nranks, rank, state_in, carry, state_out, B, H, d, st);
     return run(q, k, v, rope_cos, rope_sin, p, eps, out, carry, nullptr, workspace, st, nullptr, PH_END);
 }
 
@@ -552,9 +593,9 @@ int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk, const flo
 {
     int rc = check_shape(B, H, L, d, L < 1 ? 1 : L, dtype);
     if (rc != LCLA_OK) return rc;
-    const LclaPlan p = make_plan(B, H, L, L < 1 ? 1 : L, dtype);
+    const LclaPlan p = make_plan(B, H, L, L < 1 ? 1 : L, dtype, 0, d);
     if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
-    rc = check_buffers(q_blk, k_blk, v_blk, cos_blk, sin_blk, out, state, true, B, H, L, dtype, eps,
+    rc = check_buffers(q_blk, k_blk, v_blk, cos_blk, sin_blk, out, state, true, B, H, L, d, dtype, eps,
                        workspace, workspace_bytes, p.ws_bytes);
     if (rc != LCLA_OK) return rc;
     if (L == 0) return LCLA_OK;
@@ -568,7 +609,7 @@ int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,
     const int rc = check_shape(B, H, N, d, block_len, dtype);
     if (rc != LCLA_OK) return rc;
     if (!info) return LCLA_ERR_INVALID_ARG;
-    const LclaPlan p = make_plan(B, H, N, block_len, dtype);
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype, 0, d);
     if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
     info[0] = p.chunk;
     info[1] = p.nseg;
@@ -583,7 +624,7 @@ const char *lcla_status_string(int status)
     switch (status) {
     case LCLA_OK: return "ok";
     case LCLA_ERR_INVALID_ARG: return "invalid argument";
-    case LCLA_ERR_UNSUPPORTED: return "unsupported problem (this build serves d = 32, N <= 2^30)";
+    case LCLA_ERR_UNSUPPORTED: return "unsupported problem (this build serves d = 32 and 64, N <= 2^30)";
     case LCLA_ERR_MISALIGNED: return "array pointer not 16-byte aligned";
     case LCLA_ERR_WORKSPACE: return "workspace missing or too small";
     case LCLA_ERR_CUDA: return "CUDA launch failed";

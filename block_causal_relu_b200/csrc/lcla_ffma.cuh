@@ -638,7 +638,7 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
 // state_out (may equal state_in) receives the total.
 // ---------------------------------------------------------------------------
 constexpr int SCAN_THREADS = 128;
-constexpr int SCAN_VEC = 4;   // elements per thread (LCLA_SZ is a multiple of 4)
+constexpr int SCAN_VEC = 4;   // elements per thread (a state's (d + 1) * d floats are a multiple of 4 for even d)
 
 __device__ __forceinline__ void add4(float4 &a, const float4 &b)
 {
@@ -663,7 +663,7 @@ __global__ void __launch_bounds__(SCAN_THREADS)
 scan_chunk_totals(const LclaPlan p, const float *__restrict__ part, const float *state_in, float *__restrict__ ctot)
 {
     constexpr int BATCH = 16;
-    const size_t n4 = (size_t)p.B * p.H * (LCLA_SZ / SCAN_VEC);
+    const size_t n4 = (size_t)p.B * p.H * (p.sz / SCAN_VEC);
     const size_t x = (size_t)blockIdx.x * SCAN_THREADS + threadIdx.x;
     const int c = blockIdx.y;
     pdl_wait();
@@ -693,7 +693,7 @@ scan_chunk_prefix(const LclaPlan p, const float *__restrict__ part, const float 
                   float *__restrict__ pref, float *state_out)
 {
     constexpr int BATCH = 16;
-    const size_t n4 = (size_t)p.B * p.H * (LCLA_SZ / SCAN_VEC);
+    const size_t n4 = (size_t)p.B * p.H * (p.sz / SCAN_VEC);
     const size_t x = (size_t)blockIdx.x * SCAN_THREADS + threadIdx.x;
     const int c = blockIdx.y;
     pdl_wait();
@@ -754,7 +754,7 @@ scan_states_grouped(const LclaPlan p, const float *__restrict__ part, float *__r
                     const float *state_in, float *state_out)
 {
     extern __shared__ float4 gsum[];   // [groups][32]
-    const size_t n4 = (size_t)p.B * p.H * (LCLA_SZ / SCAN_VEC);
+    const size_t n4 = (size_t)p.B * p.H * (p.sz / SCAN_VEC);
     const int lane = threadIdx.x & 31, wg = threadIdx.x >> 5;
     const size_t x = (size_t)blockIdx.x * 32 + lane;
     const bool live = x < n4;

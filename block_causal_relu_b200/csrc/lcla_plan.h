@@ -5,9 +5,10 @@
 // Attention for Long Video Generation with Sana", section "Chunk-Wise
 // Causality").  The kernels cut the sequence into *segments*, contiguous token
 // ranges that either
-//   - lie inside one block (block mode, block_len >= LCLA_T): every token of
-//     the segment uses the inclusive prefix state of its block; or
-//   - hold whole blocks only (chunk mode, block_len < LCLA_T): tiles of
+//   - lie inside one block (block mode: block_len >= LCLA_T, explicit block
+//     offsets, and every block length at head dim 64): every token of the
+//     segment uses the inclusive prefix state of its block; or
+//   - hold whole blocks only (chunk mode, block_len < LCLA_T at d = 32): tiles of
 //     T = (LCLA_T / block_len) * block_len tokens, where a token uses the
 //     exclusive prefix at the tile start plus a masked term inside the tile.
 // Pass A reduces each segment to a partial state, the scan turns partials
@@ -15,18 +16,20 @@
 #pragma once
 #include <stddef.h>
 
-#define LCLA_D 32                              // head dim served
+#define LCLA_D 32                              // head dim of the tensor-core and tiled CUDA-core kernels
+#define LCLA_D_WIDE 64                         // the other head dim served (generic CUDA-core kernels)
 #define LCLA_HG 2                              // heads per CTA (CUDA-core path)
 #define LCLA_T 64                              // tokens per tile (CUDA-core path)
 #define LCLA_TC_T 64                           // tokens per tile (tensor-core path)
 #define LCLA_TC_HQ 4                           // heads per work unit (tensor-core path)
 #define LCLA_TC_CTAS LCLA_SMS                  // persistent tensor-core CTAs (one per SM)
-#define LCLA_SZ ((LCLA_D + 1) * LCLA_D)        // floats per (S, z) state
+#define LCLA_SZ ((LCLA_D + 1) * LCLA_D)        // floats per (S, z) state at LCLA_D
 #define LCLA_SMS 148                           // B200 streaming multiprocessors
 #define LCLA_TARGET_CTAS (LCLA_SMS * 4)        // CTAs per pass the CUDA-core plan aims for
 
 struct LclaPlan {
     int B, H, N, L, dtype;
+    int d, sz;     // head dim and floats per (S, z) state, (d + 1) * d
     int chunk;     // 0: block mode, 1: chunk mode
     int tc;        // 1: tensor-core kernels (bf16, block mode), 0: CUDA-core kernels
     int T;         // chunk mode: tokens per tile (whole blocks); block mode: tile tokens

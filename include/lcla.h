@@ -35,7 +35,11 @@
  *   - Arguments are validated before anything is enqueued; on any error code
  *     other than LCLA_ERR_CUDA nothing was enqueued and no memory was touched.
  *   - Every array pointer must be 16-byte aligned (LCLA_ERR_MISALIGNED).
- *   - d must be 32 (other head dims: LCLA_ERR_UNSUPPORTED).
+ *   - d must be 32 or 64 (the pages set linear_head_dim to 32 or 64: "Implementing
+ *     Block Causal Linear Attention ...", section "Integration into Sana's
+ *     Video Backbone"); other head dims: LCLA_ERR_UNSUPPORTED.  d = 32 runs
+ *     on tensor cores for bf16 with block_len >= 64; d = 64 runs on CUDA cores
+ *     with one thread block per (segment, head, batch entry), so H <= 65535.
  *   - `out` must not overlap q, k, v, the tables, the state or the workspace
  *     (LCLA_ERR_INVALID_ARG).
  *   - eps must be finite and >= 0.
@@ -61,7 +65,7 @@ extern "C" {
 typedef enum {
     LCLA_OK = 0,
     LCLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad dtype, overlap, bad eps */
-    LCLA_ERR_UNSUPPORTED = 2,   /* valid request this build does not serve (d != 32, N > 2^30) */
+    LCLA_ERR_UNSUPPORTED = 2,   /* valid request this build does not serve (d not 32 or 64, N > 2^30) */
     LCLA_ERR_MISALIGNED = 3,    /* an array pointer is not 16-byte aligned */
     LCLA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the query says */
     LCLA_ERR_CUDA = 5,          /* a CUDA launch failed; see cudaGetLastError */
@@ -272,11 +276,11 @@ LCLA_API int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk,
 
 /*
  * How lcla_forward cuts this problem, for benchmarks and tests: writes
- * info[0] = 1 when tiles hold whole blocks (block_len < 64), else 0;
+ * info[0] = 1 when tiles hold whole blocks (d = 32 and block_len < 64), else 0;
  * info[1] = segments (partial states written by the first pass);
  * info[2] = prefix states (blocks, or segments when info[0] = 1);
  * info[3] = tokens per tile; info[4] = 1 when the tensor-core kernels run
- * (bf16 with block_len >= 64), else 0.  `info` holds 5 ints.  Returns an
+ * (d = 32, bf16, block_len >= 64), else 0.  `info` holds 5 ints.  Returns an
  * lcla_status; touches no device.
  */
 LCLA_API int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,

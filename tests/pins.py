@@ -86,7 +86,8 @@ def pin_masked_equals_recurrence(orc):
     cases = [dict(seed=1, N=37, L=5), dict(seed=2, N=40, L=8), dict(seed=3, N=33, L=1),
              dict(seed=4, N=29, L=29), dict(seed=5, N=31, L=64),
              dict(seed=6, N=50, L=7, dtype="bf16", dist="laplace_negrows"),
-             dict(seed=7, N=24, L=6, d=32)]
+             dict(seed=7, N=24, L=6, d=32), dict(seed=8, N=22, L=6, d=64),
+             dict(seed=9, N=17, L=17, d=64, dtype="bf16", dist="laplace_negrows")]
     for c in cases:
         inp = small(c["seed"], N=c["N"], L=c["L"], d=c.get("d", 8), dtype=c.get("dtype", "f32"),
                     dist=c.get("dist", "normal"))
@@ -98,8 +99,9 @@ def pin_masked_equals_recurrence(orc):
 def pin_single_block_equals_printed_formula(orc):
     """block_len = N is the printed non-causal formula, with the normaliser on
     the unrotated features and vk = v k_rotated^T."""
-    for seed, dtype, dist in [(11, "f32", "normal"), (12, "bf16", "laplace_negrows")]:
-        inp = small(seed, N=23, d=8, dtype=dtype, dist=dist)
+    for seed, dtype, dist, d in [(11, "f32", "normal", 8), (12, "bf16", "laplace_negrows", 8),
+                                 (13, "f32", "normal", 64)]:
+        inp = small(seed, N=23, d=d, dtype=dtype, dist=dist)
         ref = literal(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, 1e-8)
         rec, _, _ = orc.recurrence(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, 23, 1e-8)
         rows_close(rec, ref, 1e-12, "recurrence(block_len=N) vs printed formula")
@@ -113,16 +115,17 @@ def pin_single_block_equals_printed_formula(orc):
 def pin_block_len_one_is_token_causal(orc):
     """block_len = 1 is token-causal linear attention (running sums), and the
     final state is the total sum of v k_rot^T and phi(k)."""
-    inp = small(21, N=41, d=8, dtype="f32")
-    q, k, v = (inp.as_f32(n) for n in ("q", "k", "v"))
-    ref, S, z = causal_cumsum(q, k, v, inp.rope_cos, inp.rope_sin, 1e-8)
-    out, st, _ = orc.recurrence(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, 1, 1e-8)
-    rows_close(out, ref, 1e-12, "block_len=1 vs running sums")
-    msk = orc.masked(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, 1, 1e-8)
-    rows_close(msk, ref, 1e-12, "masked block_len=1 vs running sums")
-    scale = np.abs(S).max()
-    assert np.abs(st[:, :, :-1, :] - S).max() <= 1e-12 * scale, "state S vs running sum"
-    assert np.abs(st[:, :, -1, :] - z).max() <= 1e-12 * np.abs(z).max(), "state z vs running sum"
+    for seed, d in ((21, 8), (22, 64)):
+        inp = small(seed, N=41, d=d, dtype="f32")
+        q, k, v = (inp.as_f32(n) for n in ("q", "k", "v"))
+        ref, S, z = causal_cumsum(q, k, v, inp.rope_cos, inp.rope_sin, 1e-8)
+        out, st, _ = orc.recurrence(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, 1, 1e-8)
+        rows_close(out, ref, 1e-12, f"block_len=1 vs running sums, d={d}")
+        msk = orc.masked(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, 1, 1e-8)
+        rows_close(msk, ref, 1e-12, f"masked block_len=1 vs running sums, d={d}")
+        scale = np.abs(S).max()
+        assert np.abs(st[:, :, :-1, :] - S).max() <= 1e-12 * scale, "state S vs running sum"
+        assert np.abs(st[:, :, -1, :] - z).max() <= 1e-12 * np.abs(z).max(), "state z vs running sum"
 
 
 def pin_step_chain_equals_forward(orc):

@@ -43,7 +43,15 @@ def test_workspace_queries():
     assert f(1, 16, 65536, 32, 1, lcla.F32) > 0
     assert f(1, 1, 0, 32, 4, lcla.BF16) == 0          # empty sequence needs nothing
     assert f(0, 1, 10, 32, 4, lcla.BF16) == 0          # invalid -> 0
-    assert f(1, 1, 10, 64, 4, lcla.BF16) == 0          # unsupported -> 0
+    assert f(1, 1, 10, 128, 4, lcla.BF16) == 0         # unsupported -> 0
+    # head dim 64: block mode at every block length, states of 65 x 64 floats
+    assert f(1, 35, 32760, 64, 4680, lcla.BF16) > 0
+    assert f(1, 35, 32760, 64, 4680, lcla.BF16) % 256 == 0
+    assert f(1, 2, 300, 64, 1, lcla.F32) >= 256 + 2 * 300 * 2 * 65 * 64 * 4   # partials and prefixes per block
+    assert f(1, 70000, 10, 64, 4, lcla.BF16) == 0       # grid y limit of the d = 64 kernels
+    info = lcla.plan_info(1, 35, 32760, 64, 4680, lcla.BF16)
+    assert not info["chunk_mode"] and not info["tensor_cores"]
+    assert not lcla.plan_info(1, 2, 300, 64, 1, lcla.F32)["chunk_mode"]
     assert f(1, 1, 10, 32, 0, lcla.BF16) == 0
     assert f(1, 1, 10, 32, 4, 7) == 0
     # independent of anything but the arguments
@@ -79,7 +87,7 @@ def stp(**kw):
     (dict(c=None), INVALID), (dict(s=None), INVALID), (dict(out=None), INVALID),
     (dict(N=-1), INVALID), (dict(B=0), INVALID), (dict(H=0), INVALID), (dict(B=-3), INVALID),
     (dict(L=0), INVALID), (dict(L=-5), INVALID), (dict(d=0), INVALID), (dict(d=31), INVALID),
-    (dict(d=64), UNSUPPORTED), (dict(d=16), UNSUPPORTED), (dict(N=(1 << 30) + 1), UNSUPPORTED),
+    (dict(d=128), UNSUPPORTED), (dict(d=16), UNSUPPORTED), (dict(N=(1 << 30) + 1), UNSUPPORTED),
     (dict(dtype=2), INVALID), (dict(dtype=-1), INVALID),
     (dict(eps=-1.0), INVALID), (dict(eps=float("nan")), INVALID), (dict(eps=float("inf")), INVALID),
     (dict(q=A + 8), MISALIGNED), (dict(k=2 * A + 4), MISALIGNED), (dict(v=3 * A + 2), MISALIGNED),
@@ -96,7 +104,7 @@ def test_forward_rejects(kw, code):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(st=None), INVALID), (dict(q=None), INVALID), (dict(L=-1), INVALID), (dict(B=0), INVALID),
-    (dict(d=64), UNSUPPORTED), (dict(dtype=5), INVALID), (dict(st=7 * A + 8), MISALIGNED),
+    (dict(d=128), UNSUPPORTED), (dict(dtype=5), INVALID), (dict(st=7 * A + 8), MISALIGNED),
     (dict(ws=None), WORKSPACE), (dict(out=3 * A), INVALID), (dict(st=5 * A), INVALID),
     (dict(eps=-0.5), INVALID),
 ])
@@ -116,7 +124,7 @@ def test_explicit_blocks_workspace_and_arguments():
     assert f(1, 4, 100, 32, 0, lcla.BF16) == 0          # no blocks
     assert f(1, 4, 100, 32, 101, lcla.BF16) == 0        # more blocks than tokens
     assert f(1, 4, 100, 32, 3, lcla.BF16) > 0
-    assert f(1, 4, 100, 64, 3, lcla.BF16) == 0          # d = 64 not served
+    assert f(1, 4, 100, 128, 3, lcla.BF16) == 0         # d = 128 not served
     import ctypes
     a = 1 << 20
     fn = lcla.lib.lcla_forward_blocks
@@ -149,7 +157,7 @@ def test_shard_workspace_and_arguments():
     assert f(1, 70, 18720, 32, 4680, lcla.BF16) == \
         lcla.forward_workspace_bytes(1, 70, 18720, 32, 4680, lcla.BF16) + 70 * 33 * 32 * 4
     assert f(1, 4, 0, 32, 16, lcla.BF16) == 0            # an empty shard needs nothing
-    assert f(1, 4, 100, 64, 16, lcla.BF16) == 0          # d = 64 not served
+    assert f(1, 4, 100, 128, 16, lcla.BF16) == 0         # d = 128 not served
     a = 1 << 20
     begin, end = lcla.lib.lcla_shard_begin, lcla.lib.lcla_shard_end
     # argument errors return before any launch (no device memory is touched)

@@ -29,6 +29,10 @@ def test_page_constants():
     pc = json.load(open(os.path.join(HERE, "page_constants.json")))
     assert pc["eps"]["value"] == 1e-8
     assert pc["head_dim"]["value"] == 32
+    assert pc["head_dims_served"]["value"] == [32, 64]
     for spec in NAMED.values():
         assert spec.eps == pc["eps"]["value"]
-        assert spec.d == pc["head_dim"]["value"]
+        assert spec.d in pc["head_dims_served"]["value"]
+        # the head count follows hidden_size // linear_head_dim at the model width of 2240
+        if spec.d == 64:
+            assert spec.H * spec.d == 2240

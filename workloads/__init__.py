@@ -238,7 +238,8 @@ def _robust(dtype: str, L: int, seed: int) -> Spec:
 
 
 # The named workloads: tiny parity case, 480p-like forward, streaming blocks,
-# minute-scale forward, and the robustness sweep over block lengths.
+# minute-scale forward, the 480p-like forward at head dim 64, and the
+# robustness sweep over block lengths.
 NAMED = {
     "tiny_f32": Spec("tiny_f32", 1, 2, 1024, 32, 256, "f32", 0),
     "fwd480p_bf16": Spec("fwd480p_bf16", 1, 70, 21 * 30 * 52, 32, 3 * 30 * 52, "bf16", 1,
@@ -247,6 +248,9 @@ NAMED = {
                         rope="3d", grid=(41, 30, 52)),
     "minute_bf16": Spec("minute_bf16", 1, 70, 241 * 44 * 80, 32, 3 * 44 * 80, "bf16", 3,
                         rope="3d", grid=(241, 44, 80)),
+    # linear_head_dim 64 at the same model width (35 heads x 64 = 2240)
+    "fwd480p_d64_bf16": Spec("fwd480p_d64_bf16", 1, 35, 21 * 30 * 52, 64, 3 * 30 * 52, "bf16", 12,
+                             rope="3d", grid=(21, 30, 52)),
 }
 for _i, _L in enumerate((1, 64, 1560, 4680, 65536)):
     for _dt in ("f32", "bf16"):
