@@ -2,8 +2,10 @@
 
 Thin binding of the C-ABI library ``liblcla.so`` (declared in
 ``include/lcla.h``): it checks and marshals torch tensors (device memory and
-the current CUDA stream) into the two entry points.  Every step of the
-computation runs in the library's sm_100a kernels; there is no other path.
+the current CUDA stream) into its entry points -- the whole-sequence forward
+(uniform or explicit blocks), the streaming step, the two halves of a
+sequence-sharded forward and the Mix-FFN temporal convolution.  Every step of
+the computation runs in the library's sm_100a kernels; there is no other path.
 Importing this package fails if the library has not been built
 (``python block_causal_relu_b200/build.py``).
 """

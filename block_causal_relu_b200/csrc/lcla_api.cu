@@ -3,7 +3,11 @@
 // Validates every argument on the host before anything is enqueued, builds
 // the work plan, and launches pass A (segment partial states), the scan
 // (prefix states, carried state in/out) and pass C (outputs) on the caller's
-// stream.  Allocates nothing.
+// stream -- all three for a forward or a step, pass A and the scan for the
+// first half of a sharded forward, the carry-in, the scan and pass C for the
+// second.  Kernels: tensor cores for bf16 at d = 32 in block mode, the tiled
+// CUDA-core kernels otherwise at d = 32, the generic CUDA-core kernels at
+// d = 64.  Allocates nothing.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -81,6 +85,26 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0, int d
                 const double balance = (double)n / (double)(rounds * LCLA_TC_CTAS);
                 const double overhead = (4.0 * 4224.0 * nsb) / (256.0 * (double)Lb);
                 const double cost = (1.0 + overhead) / balance;
+                if (cost < best_cost - 1e-9) { best_cost = cost; best = nsb; }
+            }
+            nsb = best;
+        } else if (d != LCLA_D) {
+            // one CTA per (segment, head, batch entry) and pass; pick the split that fills whole waves of
+            // both passes' resident CTAs best, against a segment's partial state (written and read back)
+            // relative to its q, k, v, out bytes
+            const long long Lb = L < N ? L : N;
+            const double io = 4.0 * d * (dtype == LCLA_BF16 ? 2 : 4);   // bytes per token and head
+            long long best = 1;
+            double best_cost = 1e30;
+            for (nsb = 1; nsb <= tpb && nsb <= 64; ++nsb) {
+                const long long n = units * p.nb * nsb;
+                double bal = 0.0;
+                for (int res : {lcla::gen::RES_A, lcla::gen::RES_C}) {
+                    const long long cap = (long long)LCLA_SMS * res;
+                    bal += 0.5 * (double)n / (double)(((n + cap - 1) / cap) * cap);
+                }
+                const double overhead = (2.0 * 4.0 * p.sz * nsb) / (io * (double)Lb);
+                const double cost = (1.0 + overhead) / bal;
                 if (cost < best_cost - 1e-9) { best_cost = cost; best = nsb; }
             }
             nsb = best;
