@@ -55,7 +55,8 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0, int d
     p.B = B; p.H = H; p.N = N; p.L = L; p.dtype = dtype;
     p.d = d; p.sz = (d + 1) * d;
     p.ngroups = (H + LCLA_HG - 1) / LCLA_HG;
-    p.nquads = (H + LCLA_TC_HQ - 1) / LCLA_TC_HQ;
+    // tensor-core work units hold four 32-dim (virtual) heads: four heads at d = 32, two at d = 64
+    p.nquads = (int)(((long long)H * (d / LCLA_D) + LCLA_TC_HQ - 1) / LCLA_TC_HQ);
     if (N == 0) return p;
     p.nb = nblocks > 0 ? nblocks : (int)(((long long)N + L - 1) / L);
     // CUDA-core CTAs per segment: head pairs at d = 32, single heads at d = 64
@@ -63,7 +64,7 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0, int d
     // d = 64 runs in block mode for every block length (its kernels have no chunk mode)
     if (nblocks > 0 || L >= LCLA_T || d != LCLA_D) {
         p.chunk = 0;
-        p.tc = dtype == LCLA_BF16 && d == LCLA_D;
+        p.tc = dtype == LCLA_BF16;
         p.T = p.tc ? LCLA_TC_T : LCLA_T;
         const long long tpb = ((long long)(L < N ? L : N) + p.T - 1) / p.T;   // tiles per full block
         long long nsb;
@@ -83,13 +84,13 @@ LclaPlan make_plan(int B, int H, int N, int L, int dtype, int nblocks = 0, int d
                 const long long ctas = n < LCLA_TC_CTAS ? n : LCLA_TC_CTAS;
                 const long long rounds = (n + ctas - 1) / ctas;
                 const double balance = (double)n / (double)(rounds * LCLA_TC_CTAS);
-                const double overhead = (4.0 * 4224.0 * nsb) / (256.0 * (double)Lb);
+                const double overhead = (4.0 * 4.0 * p.sz * nsb) / (8.0 * d * (double)Lb);
                 const double cost = (1.0 + overhead) / balance;
                 if (cost < best_cost - 1e-9) { best_cost = cost; best = nsb; }
             }
             nsb = best;
         } else if (d != LCLA_D) {
-            // one CTA per (segment, head, batch entry) and pass; pick the split that fills whole waves of
+            // fp32 at d = 64: one CTA per (segment, head, batch entry) and pass; pick the split that fills whole waves of
             // both passes' resident CTAs best, against a segment's partial state (written and read back)
             // relative to its q, k, v, out bytes
             const long long Lb = L < N ? L : N;
@@ -262,13 +263,13 @@ bool map_out_blocks(CUtensorMap *m, const void *base, int B, int N, int H)
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [N, d/2] fp32 rotary table; box = one tile of tokens, 64-byte swizzle.
-bool map_table(CUtensorMap *m, const float *base, int N)
+// [N, d/2] fp32 rotary table; box = 16 columns of one tile of tokens, 64-byte swizzle (d = 64: two boxes).
+bool map_table(CUtensorMap *m, const float *base, int N, int d)
 {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {LCLA_D / 2, (cuuint64_t)N};
-    cuuint64_t strides[1] = {(cuuint64_t)(LCLA_D / 2) * 4};
+    cuuint64_t dims[2] = {(cuuint64_t)d / 2, (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)(d / 2) * 4};
     cuuint32_t box[2] = {LCLA_D / 2, LCLA_TC_T};
     cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, es,
@@ -277,36 +278,40 @@ bool map_table(CUtensorMap *m, const float *base, int N)
 }
 
 // Tensor-core path: returns false (nothing enqueued) when a tensor map cannot
-// be encoded, so that the caller can run the CUDA-core kernels instead.
+// be encoded, so that the caller can run the CUDA-core kernels instead.  At
+// d = 64 the tensors are mapped as 2H virtual heads of 32 dims.
+template <int DW>
 bool launch_tc(const void *q, const void *k, const void *v, const float *rc, const float *rs,
                const LclaPlan &p, float eps, void *out, const float *state_in, float *state_out,
                unsigned char *ws, cudaStream_t st, cudaEvent_t const *ev, int *rc_out, Phase ph = PH_ALL)
 {
     CUtensorMap mq, mk, mv, mo, mc, ms;
     const bool a = ph != PH_END, c = ph != PH_BEGIN;
-    if ((a && (!map_tokens(&mk, k, p.B, p.N, p.H) || !map_tokens(&mv, v, p.B, p.N, p.H))) ||
-        (c && (!map_tokens(&mq, q, p.B, p.N, p.H) || !map_out_blocks(&mo, out, p.B, p.N, p.H))) ||
-        !map_table(&mc, rc, p.N) || !map_table(&ms, rs, p.N))
+    const int HV = p.H * (DW / LCLA_D);
+    if ((a && (!map_tokens(&mk, k, p.B, p.N, HV) || !map_tokens(&mv, v, p.B, p.N, HV))) ||
+        (c && (!map_tokens(&mq, q, p.B, p.N, HV) || !map_out_blocks(&mo, out, p.B, p.N, HV))) ||
+        !map_table(&mc, rc, p.N, DW) || !map_table(&ms, rs, p.N, DW))
         return false;
+    using LA = lcla::tc::LayA<DW>;
+    using LC = lcla::tc::LayC<DW>;
     float *part = reinterpret_cast<float *>(ws + p.part_off);
     float *pref = reinterpret_cast<float *>(ws + p.pref_off);
     int *status = reinterpret_cast<int *>(ws);
     const long long units = (long long)p.nseg * p.nquads * p.B;
     const dim3 grid((unsigned)(units < LCLA_TC_CTAS ? units : LCLA_TC_CTAS));
     if (a) {
-        set_smem(lcla::tc::pass_a_tc, lcla::tc::LayA::BYTES);
+        set_smem(lcla::tc::pass_a_tc<DW>, LA::BYTES);
         cudaMemsetAsync(status, 0, sizeof(int), st);
         if (ev) cudaEventRecord(ev[0], st);
-        lcla::tc::pass_a_tc<<<grid, lcla::tc::LayA::NTHREADS, lcla::tc::LayA::BYTES, st>>>(mk, mv, mc, ms, p,
-                                                                                           part, status);
+        lcla::tc::pass_a_tc<DW><<<grid, LA::NTHREADS, LA::BYTES, st>>>(mk, mv, mc, ms, p, part, status);
         if (ev) cudaEventRecord(ev[1], st);
     }
     launch_scan(p, part, pref, state_in, state_out, ws, st);
     if (c) {
-        set_smem(lcla::tc::pass_c_tc, lcla::tc::LayC::BYTES);
+        set_smem(lcla::tc::pass_c_tc<DW>, LC::BYTES);
         if (ev) cudaEventRecord(ev[2], st);
-        launch_pdl(lcla::tc::pass_c_tc, grid, dim3(lcla::tc::LayC::NTHREADS), lcla::tc::LayC::BYTES, st, mq, mc,
-                   ms, mo, p, (const float *)pref, eps, (__nv_bfloat16 *)out, status);
+        launch_pdl(lcla::tc::pass_c_tc<DW>, grid, dim3(LC::NTHREADS), LC::BYTES, st, mq, mc, ms, mo, p,
+                   (const float *)pref, eps, (__nv_bfloat16 *)out, status);
         if (ev) cudaEventRecord(ev[3], st);
     }
     *rc_out = cudaGetLastError() == cudaSuccess ? LCLA_OK : LCLA_ERR_CUDA;
@@ -380,6 +385,16 @@ int run(const void *q, const void *k, const void *v, const float *rc, const floa
         const LclaPlan &p, float eps, void *out, const float *state_in, float *state_out,
         void *ws, cudaStream_t st, cudaEvent_t const *ev = nullptr, Phase ph = PH_ALL)
 {
+    if (p.tc) {
+        int status = LCLA_OK;
+        const bool launched =
+            p.d == LCLA_D
+                ? launch_tc<LCLA_D>(q, k, v, rc, rs, p, eps, out, state_in, state_out, (unsigned char *)ws, st, ev,
+                                    &status, ph)
+                : launch_tc<LCLA_D_WIDE>(q, k, v, rc, rs, p, eps, out, state_in, state_out, (unsigned char *)ws, st,
+                                         ev, &status, ph);
+        if (launched) return status;
+    }
     if (p.d != LCLA_D) {
         if (p.dtype == LCLA_BF16)
             return launch_gen<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
@@ -387,11 +402,6 @@ int run(const void *q, const void *k, const void *v, const float *rc, const floa
                                              state_in, state_out, (unsigned char *)ws, st, ev, ph);
         return launch_gen<float>((const float *)q, (const float *)k, (const float *)v, rc, rs, p, eps,
                                  (float *)out, state_in, state_out, (unsigned char *)ws, st, ev, ph);
-    }
-    if (p.tc) {
-        int status = LCLA_OK;
-        if (launch_tc(q, k, v, rc, rs, p, eps, out, state_in, state_out, (unsigned char *)ws, st, ev, &status, ph))
-            return status;
     }
     if (p.dtype == LCLA_BF16)
         return launch_all<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,

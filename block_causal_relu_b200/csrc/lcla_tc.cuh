@@ -444,18 +444,30 @@ __device__ __forceinline__ Unit unit_at(const LclaPlan &p, int u)
     return x;
 }
 
-constexpr int NT = 3;             // rotary-table ring slots ([cos 4 KB | sin 4 KB] per tile)
+constexpr int NT = 3;             // rotary-table ring slots
 constexpr int CTRL_BYTES = 512;   // control block: mbarriers (8 B each), tensor-memory slot, abort flag
 constexpr int SMEM_MAX = 232448;  // dynamic shared memory a CTA may opt in to
-constexpr int TAB_BYTES = 8192;
 constexpr int NPRO = 16;          // prologue warps (both passes)
+
+// Head width DW: 32, or 64 seen as two 32-dim "virtual" heads (dims 0-31 and
+// 32-63 of a head are virtual heads 2h and 2h+1 of the same [B, N, H * 64]
+// row).  A table slot holds one tile's rotary rows: [cos | sin] of 4 KB each
+// at DW = 32, [cos 0-15 | cos 16-31 | sin 0-15 | sin 16-31] at DW = 64, the
+// second half rotating the second virtual head.
+template <int DW>
+struct Width {
+    static_assert(DW == 32 || DW == 64, "head widths 32 and 64");
+    static constexpr int VPH = DW / 32;               // virtual heads per head
+    static constexpr int TAB_BYTES = 8192 * VPH;      // one table slot
+    static constexpr int SZ = (DW + 1) * DW;          // floats per (S, z) state
+};
 
 // Producer: per tile, TMA loads of the quad's input boxes into the stage ring
 // (NBOX boxes of [64 token][4 / NBOX heads] per tensor map, heads past H read
 // as zeros)
 // and of the tile's rotary rows into the table ring.  On abort, waits
 // (bounded) for the loads already issued before returning.
-template <int S, int STAGE, int NMAP, int NBOX>
+template <int DW, int S, int STAGE, int NMAP, int NBOX>
 __device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t sb, uint32_t tab0,
                                         uint32_t FULL, uint32_t EMPTY, uint32_t CFULL, uint32_t CEMPTY,
                                         const CUtensorMap *const (&maps)[NMAP], const int (&offs)[NMAP],
@@ -488,10 +500,14 @@ __device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t 
                 ok = false;
                 break;
             }
-            const uint32_t tb = tab0 + cr.idx * TAB_BYTES, cb = CFULL + 8 * cr.idx;
-            bar_expect_tx(cb, (uint32_t)TAB_BYTES);
-            tma_load2(tb, mc, cb, 0, t);
-            tma_load2(tb + TAB_BYTES / 2, ms, cb, 0, t);
+            constexpr int TB = Width<DW>::TAB_BYTES, VPH = Width<DW>::VPH;
+            const uint32_t tb = tab0 + cr.idx * TB, cb = CFULL + 8 * cr.idx;
+            bar_expect_tx(cb, (uint32_t)TB);
+#pragma unroll
+            for (int hh = 0; hh < VPH; ++hh) {   // columns [16 hh, 16 hh + 16) of the [N, DW / 2] tables
+                tma_load2(tb + hh * 4096, mc, cb, 16 * hh, t);
+                tma_load2(tb + TB / 2 + hh * 4096, ms, cb, 16 * hh, t);
+            }
             ring_next<NT>(cr);
             ++tissued;
         }
@@ -507,10 +523,13 @@ __device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t 
 // ---------------------------------------------------------------------------
 // Pass A
 // ---------------------------------------------------------------------------
+template <int DW>
 struct LayA {
-    static constexpr int STAGES = 4;
+    // four stages at DW = 32; three at DW = 64, whose table slots are twice as large
+    static constexpr int STAGES = DW == 32 ? 4 : 3;
     // stage: [k~ operand, 4 atoms of [64 tok][hi 32 | lo 32] (raw k lands in atoms 0-1) | v, 2 boxes]
     static constexpr int K_OFF = 0, V_OFF = 32768, STAGE = 49152;
+    static constexpr int TAB_BYTES = Width<DW>::TAB_BYTES;
     static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
     static constexpr int Z_OFF = C_OFF + NT * TAB_BYTES;            // key-sum parts [16 warps][2 g][4 f][2 heads][8]
     static constexpr int Z_BYTES = NPRO * 2 * 4 * 2 * 8 * 4;
@@ -527,18 +546,23 @@ struct LayA {
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 1, 1);
     static constexpr int TMEM_COLS = NTM * 256;
     static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 3;
+    static_assert(BYTES <= SMEM_MAX, "pass A shared memory");
+    static_assert(8 * NBARS + 8 <= CTRL_BYTES, "pass A control block");
+    static_assert(NTHREADS / 32 - W_PRO0 == NPRO, "pass A prologue warps: barrier counts use NPRO");
 };
-static_assert(LayA::BYTES <= SMEM_MAX, "pass A shared memory");
-static_assert(8 * LayA::NBARS + 8 <= CTRL_BYTES, "pass A control block");
-static_assert(LayA::NTHREADS / 32 - LayA::W_PRO0 == NPRO, "pass A prologue warps: barrier counts use NPRO");
 
-__global__ void __launch_bounds__(LayA::NTHREADS, 1)
+// Pass A over head width DW.  At DW = 64 each quad holds two heads as four
+// virtual heads; the products of the quad already hold the cross blocks
+// (virtual heads 2h', 2h'+1 against 2h, 2h+1) that a 64-dim head's state needs.
+template <int DW>
+__global__ void __launch_bounds__(LayA<DW>::NTHREADS, 1)
 pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
           const __grid_constant__ CUtensorMap mc, const __grid_constant__ CUtensorMap ms, const LclaPlan p,
           float *__restrict__ part, int *__restrict__ status)
 {
-    using L = LayA;
-    constexpr int S = L::STAGES, NTM = L::NTM;
+    using L = LayA<DW>;
+    constexpr int S = L::STAGES, NTM = L::NTM, VPH = Width<DW>::VPH, TB = L::TAB_BYTES;
+    const int HV = p.H * VPH;   // virtual heads
     extern __shared__ __align__(1024) unsigned char smraw[];
     const uint32_t raw = s32(smraw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -588,8 +612,8 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
         if (lane == 0) {
             const CUtensorMap *const maps[2] = {&mk, &mv};
             const int offs[2] = {L::K_OFF, L::V_OFF};
-            produce<S, L::STAGE, 2, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc, &ms,
-                                       abort_flag);
+            produce<DW, S, L::STAGE, 2, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc,
+                                           &ms, abort_flag);
         }
     } else if (w == L::W_MMA) {
         // ---------------- MMA issuer: one accumulator per chunk of CHUNK tiles ----------------
@@ -654,9 +678,13 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                 ring_next<S>(fr);
                 ring_next<NT>(cr);
                 unsigned char *stg = sm + st * L::STAGE;
-                const unsigned char *tab = sm + L::C_OFF + ct * TAB_BYTES;
-                const float4 c4 = ldsf4(tab + o.tab);
-                const float4 s4 = ldsf4(tab + TAB_BYTES / 2 + o.tab);
+                const unsigned char *tab = sm + L::C_OFF + ct * TB;
+                // DW = 64: heads 2g, 2g+1 are the halves of one head and rotate with table halves 0, 1
+                float4 c4[2], s4[2];
+                c4[0] = ldsf4(tab + o.tab);
+                s4[0] = ldsf4(tab + TB / 2 + o.tab);
+                c4[1] = VPH == 2 ? ldsf4(tab + 4096 + o.tab) : c4[0];
+                s4[1] = VPH == 2 ? ldsf4(tab + TB / 2 + 4096 + o.tab) : s4[0];
                 const uint4 k0 = lds128(stg + L::K_OFF + o.in0);   // head 2g
                 const uint4 k1 = lds128(stg + L::K_OFF + o.in1);   // head 2g+1
                 const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
@@ -671,7 +699,7 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                         zacc[hh][2 * j] += bf_lo(fw[j]);
                         zacc[hh][2 * j + 1] += bf_hi(fw[j]);
                     }
-                    rope_split4(fw, c4, s4, hi, lo);
+                    rope_split4(fw, c4[hh], s4[hh], hi, lo);
                     // head 2g -> atom g (over the raw chunks just read), head 2g+1 -> atom 2+g
                     sts128(stg + L::K_OFF + (hh ? o.out2 : o.in0), hi);
                     sts128(stg + L::K_OFF + (hh ? o.out3 : o.in1), lo);
@@ -714,23 +742,31 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
         }
     } else {
         // ---------------- drain: chunk accumulators -> partial state of the unit ----------------
-        const int q = w;   // head of the quad; tensor-memory lanes 32q + c
+        // warp q: virtual head q of the quad, tensor-memory lanes 32q + c.  DW = 32: row c of its own S (the
+        // diagonal block, hi + lo columns).  DW = 64: row 32 a + c of its head's S, a = q & 1, from the blocks
+        // against both halves of the head (virtual heads q & ~1 and q | 1: columns e and 32 + e).
+        const int q = w;
         const float nanv = __int_as_float(0x7fc00000);
         Ring tr = {0, 0u}, zr = {0, 0u};   // accumulator full, key sum ready (1 slot)
         bool ok = true;
         for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
-            const int head = HQ * x.hq + q;
-            float *dst = part + (((size_t)x.s * p.B + x.b) * p.H + (head < p.H ? head : 0)) * LCLA_SZ;
+            const int vh = HQ * x.hq + q;
+            const bool live = vh < HV;
+            float *dst = part + (((size_t)x.s * p.B + x.b) * p.H + (live ? vh / VPH : 0)) * Width<DW>::SZ;
+            float *rows = dst + (size_t)(vh % VPH) * 32 * DW;   // this warp's 32 rows of S
+            float *zdst = dst + DW * DW + (vh % VPH) * 32;       // and its 32 entries of z
             if (ok && x.ntile == 0) {   // empty segment: nothing was loaded or summed
-                if (head < p.H)
-                    for (int e = lane; e < LCLA_SZ; e += 32) dst[e] = 0.f;
+                if (live) {
+                    for (int e = lane; e < 32 * DW; e += 32) rows[e] = 0.f;
+                    zdst[lane] = 0.f;
+                }
                 continue;
             }
             if (ok) {
-                float sacc[32];   // S row c = lane, summed over the unit's chunks
+                float sacc[DW];   // S row (lane) over the unit's chunks
 #pragma unroll
-                for (int j = 0; j < 32; ++j) sacc[j] = 0.f;
+                for (int j = 0; j < DW; ++j) sacc[j] = 0.f;
                 for (int i = 0; i < x.ntile; i += L::CHUNK) {
                     const int tb = tr.idx;
                     if (!__all_sync(ALL, bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag))) {
@@ -739,13 +775,17 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                     }
                     ring_next<NTM>(tr);
                     tc_after();
-                    const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q);
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {   // k~hi columns e = 0-15, 16-31, then k~lo
-                        uint32_t v[16];
-                        tmem_ld16(ta + 16 * c4, v);
+                    for (int hb = 0; hb < VPH; ++hb) {
+                        const int atom = atom_of(VPH == 1 ? q : (q & ~1) + hb);
+                        const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) sacc[16 * (c4 & 1) + j] += __uint_as_float(v[j]);
+                        for (int c4 = 0; c4 < 4; ++c4) {   // k~hi columns e = 0-15, 16-31, then k~lo
+                            uint32_t v[16];
+                            tmem_ld16(ta + 16 * c4, v);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) sacc[32 * hb + 16 * (c4 & 1) + j] += __uint_as_float(v[j]);
+                        }
                     }
                     tc_before();
                     __syncwarp();
@@ -761,19 +801,21 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
                     for (int pw = 0; pw < NPRO; ++pw) zs += zp[pw * 2 * 4 * 16];
                     __syncwarp();
                     if (lane == 0) bar_arrive(ZFREE);
-                    if (head < p.H) {   // row c = lane of S, then z; kept in L2 for the scan
+                    if (live) {   // row of S, then z; kept in L2 for the scan
                         const uint64_t keep = policy_evict_last();
-                        float4 *row = reinterpret_cast<float4 *>(dst + lane * LCLA_D);
+                        float4 *row = reinterpret_cast<float4 *>(rows + lane * DW);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
+                        for (int j = 0; j < DW / 4; ++j)
                             st_v4_hint(row + j, make_float4(sacc[4 * j], sacc[4 * j + 1], sacc[4 * j + 2], sacc[4 * j + 3]),
                                        keep);
-                        st_f32_hint(dst + LCLA_D * LCLA_D + lane, zs, keep);
+                        st_f32_hint(zdst + lane, zs, keep);
                     }
                 }
             }
-            if (!ok && head < p.H)   // aborted: this and every later partial of the head reads NaN
-                for (int e = lane; e < LCLA_SZ; e += 32) dst[e] = nanv;
+            if (!ok && live) {   // aborted: this and every later partial of the head reads NaN
+                for (int e = lane; e < 32 * DW; e += 32) rows[e] = nanv;
+                zdst[lane] = nanv;
+            }
         }
     }
 
@@ -790,12 +832,18 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
 // ---------------------------------------------------------------------------
 // Pass C
 // ---------------------------------------------------------------------------
+template <int DW>
 struct LayC {
-    static constexpr int STAGES = 4;
+    // four stages at DW = 32; three at DW = 64, whose table slots are twice as large
+    static constexpr int STAGES = DW == 32 ? 4 : 3;
     // stage: q~ operand, 4 blocks of [64 rows (tok)][q~hi 32 | q~lo 32] (raw q lands in blocks 0-1)
     static constexpr int STAGE = 32768;
+    static constexpr int TAB_BYTES = Width<DW>::TAB_BYTES;
     static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
-    static constexpr int P_OFF = C_OFF + NT * TAB_BYTES, P_BYTES = 16384;   // 2 x [128 rows (head, c)][P hi | P lo]
+    // prefix operands [128 rows (virtual head, c)][P hi | P lo]: DW = 32, one per unit, double-buffered;
+    // DW = 64, the unit's two key halves (e < 32, e >= 32) in one buffer
+    static constexpr int P_BYTES = 16384, NPB = DW == 32 ? 2 : 1;
+    static constexpr int P_OFF = C_OFF + NT * TAB_BYTES;
     static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 8 warps x 2 x [32 tok][32 c] bf16
     static constexpr int OBUF = 2048;
     static constexpr int CTRL = O_OFF + 8 * 2 * OBUF;               // mbarriers, tensor-memory slot, abort flag
@@ -806,19 +854,28 @@ struct LayC {
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
     static constexpr int TMEM_COLS = NTM * 256;
     static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 2;
+    static_assert(NPB * Width<DW>::VPH == 2, "two prefix operands of P_BYTES");
+    static_assert(BYTES <= SMEM_MAX, "pass C shared memory");
+    static_assert(8 * NBARS + 8 <= CTRL_BYTES, "pass C control block");
+    static_assert(NTHREADS / 32 - W_PRO0 == NPRO, "pass C prologue warps: barrier counts use NPRO");
+    static_assert(O_OFF % 1024 == 0 && OBUF % 512 == 0, "64-byte-swizzled output boxes need 512-byte alignment");
 };
-static_assert(LayC::BYTES <= SMEM_MAX, "pass C shared memory");
-static_assert(8 * LayC::NBARS + 8 <= CTRL_BYTES, "pass C control block");
-static_assert(LayC::NTHREADS / 32 - LayC::W_PRO0 == NPRO, "pass C prologue warps: barrier counts use NPRO");
-static_assert(LayC::O_OFF % 1024 == 0 && LayC::OBUF % 512 == 0, "64-byte-swizzled output boxes need 512-byte alignment");
 
-__global__ void __launch_bounds__(LayC::NTHREADS, 1)
+// Pass C over head width DW.  At DW = 64 the quad holds two heads as four
+// virtual heads; the output of head R, half a, is sum over the key halves b of
+// P_R[32 a + c][32 b + e] q~_{R, b}[e]: one set of MMAs with the first key half
+// of P against the stage's operand, one with the second half against the
+// operand two atoms on (atoms hold virtual heads 0, 2, 1, 3, so the window from
+// atom 2 holds 1, 3), which lands both sums in column block R.
+template <int DW>
+__global__ void __launch_bounds__(LayC<DW>::NTHREADS, 1)
 pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mc,
           const __grid_constant__ CUtensorMap ms, const __grid_constant__ CUtensorMap mo, const LclaPlan p,
           const float *__restrict__ pref, const float eps, __nv_bfloat16 *__restrict__ out, int *__restrict__ status)
 {
-    using L = LayC;
-    constexpr int S = L::STAGES, NTM = L::NTM;
+    using L = LayC<DW>;
+    constexpr int S = L::STAGES, NTM = L::NTM, VPH = Width<DW>::VPH, TB = L::TAB_BYTES, SZ = Width<DW>::SZ;
+    const int HV = p.H * VPH;   // virtual heads
     extern __shared__ __align__(1024) unsigned char smraw[];
     const uint32_t raw = s32(smraw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -865,8 +922,8 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         if (lane == 0) {
             const CUtensorMap *const maps[1] = {&mq};
             const int offs[1] = {0};
-            produce<S, L::STAGE, 1, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc, &ms,
-                                       abort_flag);
+            produce<DW, S, L::STAGE, 1, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc,
+                                           &ms, abort_flag);
         }
     } else if (w == L::W_MMA) {
         // ---------------- MMA issuer ----------------
@@ -889,14 +946,19 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     }
                     tc_after();
                     const uint32_t d = tmem + tr.idx * 256;
-                    const uint64_t bd = qdesc0 + (uint64_t)((sr.idx * L::STAGE) >> 4);
-                    // K steps of 16 elements = 32 B = 2 descriptor units; hi at +0, lo at +64 B
-                    mma_bf16(d, pd + 0, bd + 0, L::IDESC, 0);   // P hi . q~hi
-                    mma_bf16(d, pd + 2, bd + 2, L::IDESC, 1);
-                    mma_bf16(d, pd + 4, bd + 0, L::IDESC, 1);   // P lo . q~hi
-                    mma_bf16(d, pd + 6, bd + 2, L::IDESC, 1);
-                    mma_bf16(d, pd + 0, bd + 4, L::IDESC, 1);   // P hi . q~lo
-                    mma_bf16(d, pd + 2, bd + 6, L::IDESC, 1);
+                    const uint64_t bd0 = qdesc0 + (uint64_t)((sr.idx * L::STAGE) >> 4);
+#pragma unroll
+                    for (int kh = 0; kh < VPH; ++kh) {   // DW = 64: key half kh of P against the operand from atom 2 kh
+                        const uint64_t pk = pd + (uint64_t)((kh * L::P_BYTES) >> 4);
+                        const uint64_t bd = bd0 + (uint64_t)((kh * 2 * 8192) >> 4);
+                        // K steps of 16 elements = 32 B = 2 descriptor units; hi at +0, lo at +64 B
+                        mma_bf16(d, pk + 0, bd + 0, L::IDESC, kh);   // P hi . q~hi
+                        mma_bf16(d, pk + 2, bd + 2, L::IDESC, 1);
+                        mma_bf16(d, pk + 4, bd + 0, L::IDESC, 1);    // P lo . q~hi
+                        mma_bf16(d, pk + 6, bd + 2, L::IDESC, 1);
+                        mma_bf16(d, pk + 0, bd + 4, L::IDESC, 1);    // P hi . q~lo
+                        mma_bf16(d, pk + 2, bd + 6, L::IDESC, 1);
+                    }
                     mma_commit(TFULL + 8 * tr.idx);
                     mma_commit(EMPTY + 8 * sr.idx);
                     if (i == x.ntile - 1) mma_commit(PFREE + 8 * ub);
@@ -906,7 +968,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     ring_next<NTM>(tr);
                     ++issued;
                 }
-                ub ^= 1;
+                ub = (ub + 1) % L::NPB;
             }
             if (!ok && issued > 0) bar_wait_quiet(TFULL + 8 * last_tb, last_phase);
         }
@@ -926,35 +988,39 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 ok = false;
                 break;
             }
-            ring_next<2>(br);
-            {   // the quad's prefix state -> A operand rows m = (head, c): [P hi | P lo]; thread = (m, quarter of e)
-                const int m = pt >> 2, qq = pt & 3, head = HQ * x.hq + (m >> 5);
-                float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
-                if (head < p.H) {
-                    const float4 *src =
-                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + (m & 31) * LCLA_D + 8 * qq);
-                    a4 = src[0];
-                    b4 = src[1];
-                }
-                const float y[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
-                uint32_t hw[4], lw[4];
+            ring_next<L::NPB>(br);
+            {   // the quad's prefix -> A operand rows m = (virtual head, c): [P hi | P lo]; thread = (m, quarter
+                // qq of the 32 keys of key half kh); DW = 64: row 32 (vh % 2) + c of head vh / 2, one operand per kh
+                const int m = pt >> 2, qq = pt & 3, vh = HQ * x.hq + (m >> 5);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
-                    const float2 hf = __bfloat1622float2(h2);
-                    hw[j] = bf2_bits(h2);
-                    lw[j] = pack_bf2(y[2 * j] - hf.x, y[2 * j + 1] - hf.y);
+                for (int kh = 0; kh < VPH; ++kh) {
+                    float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
+                    if (vh < HV) {
+                        const float4 *src = reinterpret_cast<const float4 *>(
+                            pref + (pbase + vh / VPH) * SZ + (size_t)(32 * (vh % VPH) + (m & 31)) * DW + 32 * kh + 8 * qq);
+                        a4 = src[0];
+                        b4 = src[1];
+                    }
+                    const float y[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
+                        const float2 hf = __bfloat1622float2(h2);
+                        hw[j] = bf2_bits(h2);
+                        lw[j] = pack_bf2(y[2 * j] - hf.x, y[2 * j + 1] - hf.y);
+                    }
+                    store_quarter_hi_lo(sm + L::P_OFF + (ub + kh) * L::P_BYTES, m, qq, hw, lw);
                 }
-                store_quarter_hi_lo(sm + L::P_OFF + ub * L::P_BYTES, m, qq, hw, lw);
             }
-            float zq[2][8];   // z[8f, 8f+8) of heads 2g, 2g+1
+            float zq[2][8];   // z[8f, 8f+8) of virtual heads 2g, 2g+1
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const int head = HQ * x.hq + 2 * o.g + hh;
+                const int vh = HQ * x.hq + 2 * o.g + hh;
                 float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
-                if (head < p.H) {
-                    const float4 *src =
-                        reinterpret_cast<const float4 *>(pref + (pbase + head) * LCLA_SZ + LCLA_D * LCLA_D + 8 * o.f);
+                if (vh < HV) {
+                    const float4 *src = reinterpret_cast<const float4 *>(pref + (pbase + vh / VPH) * SZ + DW * DW +
+                                                                         32 * (vh % VPH) + 8 * o.f);
                     a4 = src[0];
                     b4 = src[1];
                 }
@@ -972,9 +1038,13 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 ring_next<S>(fr);
                 ring_next<NT>(cr);
                 unsigned char *stg = sm + st * L::STAGE;
-                const unsigned char *tab = sm + L::C_OFF + ct * TAB_BYTES;
-                const float4 c4 = ldsf4(tab + o.tab);
-                const float4 s4 = ldsf4(tab + TAB_BYTES / 2 + o.tab);
+                const unsigned char *tab = sm + L::C_OFF + ct * TB;
+                // DW = 64: virtual heads 2g, 2g+1 are the halves of one head and rotate with table halves 0, 1
+                float4 c4[2], s4[2];
+                c4[0] = ldsf4(tab + o.tab);
+                s4[0] = ldsf4(tab + TB / 2 + o.tab);
+                c4[1] = VPH == 2 ? ldsf4(tab + 4096 + o.tab) : c4[0];
+                s4[1] = VPH == 2 ? ldsf4(tab + TB / 2 + 4096 + o.tab) : s4[0];
                 const uint4 q0 = lds128(stg + o.in0);   // head 2g
                 const uint4 q1 = lds128(stg + o.in1);   // head 2g+1
                 uint32_t fw[2][4] = {{q0.x, q0.y, q0.z, q0.w}, {q1.x, q1.y, q1.z, q1.w}};
@@ -996,6 +1066,10 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     den[hh] += __shfl_xor_sync(ALL, den[hh], 1);
                     den[hh] += __shfl_xor_sync(ALL, den[hh], 2);
                 }
+                if (VPH == 2) {   // one 64-dim head: z . phi(q) over both halves
+                    const float both = den[0] + den[1];
+                    den[0] = den[1] = both;
+                }
                 // 1 / (z . phi(q) + eps): quarters with even f divide for head 2g, odd f for head 2g+1,
                 // and trade the results (lane bit 0 is bit 0 of f)
                 const float mine = 1.0f / (((o.f & 1) ? den[1] : den[0]) + eps);
@@ -1004,7 +1078,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t hi[4], lo[4];
-                    rope_split4_scaled(fw[hh], c4, s4, hh ? g1 : g0, hi, lo);
+                    rope_split4_scaled(fw[hh], c4[hh], s4[hh], hh ? g1 : g0, hi, lo);
                     // head 2g -> atom g (over the raw chunks just read), head 2g+1 -> atom 2+g
                     sts128(stg + (hh ? o.out2 : o.in0), hi);
                     sts128(stg + (hh ? o.out3 : o.in1), lo);
@@ -1022,7 +1096,10 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         // warp e: head q = e & 3 (tensor-memory lanes 32q + c), tokens [32 hf, 32 hf + 32), hf = e >> 2.
         // The accumulator already carries 1 / (z . phi(q) + eps): the epilogue only converts and moves.
         const int q = w & 3, hf = w >> 2;
-        const size_t tstride = (size_t)p.H * LCLA_D;   // elements per token
+        const size_t tstride = (size_t)p.H * DW;   // elements per token
+        // the accumulator block of this warp's rows: its own head's (DW = 32), or column block R of head R's
+        // two virtual heads (DW = 64)
+        const int ocol = 64 * (VPH == 1 ? atom_of(q) : (q >> 1));
         const uint32_t obs0 = sb + L::O_OFF + w * 2 * L::OBUF;
         const unsigned char *obp0 = sm + L::O_OFF + w * 2 * L::OBUF;
         // stmatrix row of this lane: c group m = lane >> 3 (c in [8m, 8m + 8)), token 8j + k, k = lane & 7;
@@ -1046,7 +1123,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 if (lane == 0) bulk_wait_read1();   // this buffer's previous store has read it
                 __syncwarp();
                 uint32_t v[32];
-                const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + 64 * atom_of(q) + 32 * hf;
+                const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + ocol + 32 * hf;
                 tmem_ld16x256_x4x2(ta, ta + (16u << 16), v);
                 tc_before();
                 __syncwarp();
@@ -1065,11 +1142,11 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 if (nt == T) {
                     fence_async_smem();
                     __syncwarp();
-                    if (lane == 0 && head < p.H) tma_store3_hint(&mo, obs, LCLA_D * head, t + 32 * hf, x.b, policy_evict_first());
+                    if (lane == 0 && head < HV) tma_store3_hint(&mo, obs, LCLA_D * head, t + 32 * hf, x.b, policy_evict_first());
                 } else {   // ragged tile: lane = token, its 64-byte row back from the box to global memory
                     __syncwarp();
                     const int tok = lane;
-                    if (head < p.H && 32 * hf + tok < nt) {
+                    if (head < HV && 32 * hf + tok < nt) {
                         const unsigned char *row = obp0 + ob * L::OBUF + tok * 64;
                         uint4 *g = reinterpret_cast<uint4 *>(out + ((size_t)x.b * p.N + t + 32 * hf + tok) * tstride +
                                                              (size_t)head * LCLA_D);

@@ -50,7 +50,8 @@ def test_workspace_queries():
     assert f(1, 2, 300, 64, 1, lcla.F32) >= 256 + 2 * 300 * 2 * 65 * 64 * 4   # partials and prefixes per block
     assert f(1, 70000, 10, 64, 4, lcla.BF16) == 0       # grid y limit of the d = 64 kernels
     info = lcla.plan_info(1, 35, 32760, 64, 4680, lcla.BF16)
-    assert not info["chunk_mode"] and not info["tensor_cores"]
+    assert not info["chunk_mode"] and info["tensor_cores"]          # bf16: two heads per tensor-core unit
+    assert not lcla.plan_info(1, 35, 32760, 64, 4680, lcla.F32)["tensor_cores"]   # fp32: CUDA cores
     assert not lcla.plan_info(1, 2, 300, 64, 1, lcla.F32)["chunk_mode"]
     assert f(1, 1, 10, 32, 0, lcla.BF16) == 0
     assert f(1, 1, 10, 32, 4, 7) == 0

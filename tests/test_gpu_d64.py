@@ -1,7 +1,8 @@
 """Head dim 64 on the GPU against the fp64 oracle.
 
-d = 64 runs on the generic CUDA-core passes in block mode for every block
-length.  Small cases span several 32-token tiles, ragged tails, blocks shorter
+d = 64 runs in block mode for every block length: bf16 on the tensor-core
+passes (each 64-dim head as two 32-dim virtual heads), fp32 on the generic
+CUDA-core passes.  Small cases span several 32-token tiles, ragged tails, blocks shorter
 than a tile and more than 256 blocks (the chunked scan); the 480p-like latent
 at head dim 64 (35 heads x 64 = the same 2240 width) runs at full size and is
 compared on sampled rows plus the full state.  The other entry points
