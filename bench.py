@@ -56,9 +56,10 @@ def parse():
                     help="N > 1: replicas = one independent copy of the workload per rank (weak scaling); "
                          "seq = one sequence cut into runs of whole blocks, one per rank, with one "
                          "all-gather of state totals per step (strong scaling)")
-    ap.add_argument("--op", choices=["attention", "tconv"], default="attention",
+    ap.add_argument("--op", choices=["attention", "tconv", "step"], default="attention",
                     help="attention: the block-causal attention forward (the headline); "
-                         "tconv: the causal temporal convolution with a cached last frame")
+                         "tconv: the causal temporal convolution with a cached last frame; "
+                         "step: the streaming workload block by block through lcla_step")
     return ap.parse_args()
 
 
@@ -98,18 +99,18 @@ def source_digest():
 
 
 def ncu_traffic(kernel, workload):
-    """DRAM bytes per launch from the committed ncu summary, when it was taken
-    on the current kernel sources; else None."""
+    """DRAM bytes per launch of ``kernel`` on ``workload`` from the committed
+    ncu summary, when it was taken on the current kernel sources; else None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)
     except Exception:
         return None
-    ent = rec.get("kernels", {}).get(kernel)
-    if not ent or rec.get("source_digest") != source_digest() or ent.get("workload") != workload:
+    if rec.get("source_digest") != source_digest():
         return None
-    return ent.get("traffic_bytes_per_launch")
+    ent = rec.get("workloads", {}).get(workload, {}).get(kernel)
+    return ent.get("traffic_bytes_per_launch") if ent else None
 
 
 class ClockSampler:
@@ -397,6 +398,104 @@ def run_tconv(args):
     print(json.dumps(line), flush=True)
 
 
+def run_step(args):
+    """One GPU: the streaming workload (B=2, H=70, 41 latent frames of 30 x 52
+    tokens) fed block by block through lcla_step with save=1 -- 13 blocks of
+    4680 tokens and one of 3120 -- against the carried state, the blocks'
+    inputs resident in HBM.  A step is the whole 14-block sequence; the line
+    reports the mean device time per full block, eager (one call per block,
+    events around each) and as a CUDA graph of the whole sequence."""
+    import torch
+    import block_causal_relu_b200 as lcla
+    spec = NAMED["stream_bf16"]
+    dev = torch.device("cuda", 0)
+    inp = make_inputs(spec)
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    L = spec.block_len
+    bounds = [(t, min(spec.N, t + L)) for t in range(0, spec.N, L)]
+    blocks = [[to_dev(a[:, t0:t1]) for a in (inp.q, inp.k, inp.v)] + [to_dev(inp.rope_cos[t0:t1]),
+                                                                      to_dev(inp.rope_sin[t0:t1])]
+              for t0, t1 in bounds]
+    outs = [torch.empty_like(b[0]) for b in blocks]
+    state = torch.zeros((spec.B, spec.H, spec.d + 1, spec.d), dtype=torch.float32, device=dev)
+    ws = torch.empty(lcla.step_workspace_bytes(spec.B, spec.H, L, spec.d, lcla.BF16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def sequence(events=None):
+        state.zero_()
+        for i, b in enumerate(blocks):
+            if events is not None:
+                events[i][0].record(stream)
+            lcla.step(*b, state, True, spec.eps, out=outs[i], workspace=ws, stream=stream)
+            if events is not None:
+                events[i][1].record(stream)
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        sequence()
+    torch.cuda.synchronize(dev)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in blocks] for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        e0.record(stream)
+        for r in range(K):
+            sequence(evs[r])
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms_seq = e0.elapsed_time(e1) / K
+    full = [i for i, (t0, t1) in enumerate(bounds) if t1 - t0 == L]
+    per_block = statistics.mean(evs[r][i][0].elapsed_time(evs[r][i][1]) for r in range(K) for i in full)
+    # the same sequence replayed as one CUDA graph
+    graph_ms = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            sequence()                                   # warm up on the capture stream
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(g):
+            cap = torch.cuda.current_stream(dev)
+            state.zero_()
+            for i, b in enumerate(blocks):
+                lcla.step(*b, state, True, spec.eps, out=outs[i], workspace=ws, stream=cap)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(K):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        graph_ms = g0.elapsed_time(g1) / K
+    except Exception as e:  # report, do not hide: the eager numbers stand on their own
+        graph_ms = f"capture failed: {type(e).__name__}: {e}"
+    tok_heads = spec.B * spec.N * spec.H
+    blk_bytes = 4 * spec.B * L * spec.H * spec.d * 2 + 2 * L * (spec.d // 2) * 4 + 2 * spec.B * spec.H * 33 * 32 * 4
+    peak, peak_kind = measured_peak()
+    achieved = blk_bytes / (per_block / 1e3) / 1e9
+    line = {"metric": "streaming blocks: attended tokens*heads/s and ms per full block, 1 GPU", "op": "step",
+            "value": tok_heads / (ms_seq / 1e3), "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": W,
+            "ms_per_step": ms_seq, "ms_per_block": per_block,
+            "graph_ms_per_step": graph_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded)",
+            "config": {"workload": f"{spec.name}: B={spec.B} H={spec.H} N={spec.N}, {len(blocks)} blocks of "
+                                   f"{L} tokens (last {bounds[-1][1] - bounds[-1][0]}), save=1 each",
+                       "l2": f"a full block moves {blk_bytes / 1e6:.0f} MB"},
+            "roofline": {"bound": "hbm", "kernel": "one full block (pass A + scan + pass C)", "achieved": achieved,
+                         "peak": peak, "peak_source": f"{peak_kind} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": None, "algorithmic_bytes": blk_bytes},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": K * len(blocks) * 3, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def run_seq(args):
     """Sequence-sharded forward: every rank holds the whole-block run
     ``shard_bounds(N, block_len, world)[rank]`` of one sequence; a step is
@@ -489,6 +588,8 @@ def main():
         return run_reference(args)
     if args.op == "tconv":
         return run_tconv(args)
+    if args.op == "step":
+        return run_step(args)
     if args.parallel == "seq":
         return run_seq(args)
 
