@@ -31,6 +31,9 @@ SMALL = [  # (B, H, N, block_len, dtype, dist)
     (2, 1, 65, 64, "f32", "normal"),
     (1, 5, 2000, 33, "bf16", "normal"),
     (1, 2, 1, 1, "f32", "normal"),
+    (1, 1, 300, 100, "bf16", "normal"),            # one head: its quad's last two virtual heads are past H
+    (3, 2, 129, 64, "bf16", "laplace_negrows"),    # batch 3, ragged last tile
+    (1, 3, 70, 5, "bf16", "normal"),               # 14 blocks shorter than a tile
 ]
 
 
@@ -123,3 +126,14 @@ def test_sharded_d64():
     check_outputs(host(torch.cat([o for o, _ in res], dim=1)), ref, "bf16", "d64 sharded")
     check_state(host(res[0][1]), ref_st, "d64 sharded state")
     assert all(torch.equal(st, res[0][1]) for _, st in res)
+
+
+def test_d64_repeated_calls_bit_identical():
+    spec = Spec("d64det", 2, 5, 3000, D, 700, "bf16", 2401, qk_dist="laplace_negrows", v_sigma=2.0)
+    inp = make_inputs(spec, threads=2)
+    q, k, v, c, s = inputs_to_dev(inp)
+    ref_out, ref_st = lcla.forward(q, k, v, c, s, spec.block_len, spec.eps)
+    for _ in range(5):
+        out, st = lcla.forward(q, k, v, c, s, spec.block_len, spec.eps)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref_out) and torch.equal(st, ref_st)
