@@ -19,7 +19,7 @@ import torch
 
 __all__ = ["forward", "step", "forward_workspace_bytes", "step_workspace_bytes", "plan_info",
            "forward_blocks", "forward_blocks_workspace_bytes", "temporal_conv",
-           "shard_begin", "shard_end", "shard_workspace_bytes",
+           "shard_begin", "shard_end", "shard_workspace_bytes", "device_status", "selftest_bounded_wait",
            "LclaError", "LIB_PATH", "lib", "BF16", "F32", "D", "HEAD_DIMS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblcla.so")
@@ -63,6 +63,8 @@ def _load() -> ctypes.CDLL:
     L.lcla_shard_begin.restype = I
     L.lcla_shard_end.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P, I, I, P, P, P, I, P, Z, P]
     L.lcla_shard_end.restype = I
+    L.lcla_selftest_bounded_wait.argtypes = [I, P, P]
+    L.lcla_selftest_bounded_wait.restype = I
     L.lcla_forward_plan_info.argtypes = [I, I, I, I, I, I, P]
     L.lcla_forward_plan_info.restype = I
     L.lcla_status_string.argtypes = [I]
@@ -256,6 +258,23 @@ def shard_end(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rope_cos: torch
                               _ptr(out), _ptr(state_out), code, _ptr(workspace),
                               0 if workspace is None else workspace.numel(), _stream(stream, q.device)))
     return out, state_out
+
+
+def device_status(workspace: Optional[torch.Tensor]) -> int:
+    """The device status word a call left in ``workspace`` (0: every bounded
+    wait completed; bit 0 / bit 1: pass A / pass C gave up).  Synchronises on
+    the copy."""
+    if workspace is None or workspace.numel() < 4:
+        return 0
+    return int(workspace[:4].view(torch.int32).item())
+
+
+def selftest_bounded_wait(arrive_first: bool, stream=None) -> Tuple[bool, int, int]:
+    """``lcla_selftest_bounded_wait``: (gave_up, nanoseconds waited, abort flag)."""
+    res = torch.zeros(3, dtype=torch.int64, device="cuda")
+    _check(lib.lcla_selftest_bounded_wait(int(bool(arrive_first)), _ptr(res), _stream(stream, res.device)))
+    r = res.cpu().tolist()
+    return bool(r[0]), int(r[1]), int(r[2])
 
 
 def step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cos: torch.Tensor,

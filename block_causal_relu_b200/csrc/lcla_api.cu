@@ -21,6 +21,7 @@
 #include "lcla_ffma.cuh"
 #include "lcla_gen.cuh"
 #include "lcla_plan.h"
+#include "lcla_selftest.cuh"
 #include "lcla_shard.cuh"
 #include "lcla_tc.cuh"
 

@@ -317,6 +317,30 @@ LCLA_API int lcla_forward_noalloc(const void *q, const void *k, const void *v,
                  int B, int H, int N, int d, int block_len, float eps,
                  void *out, float *state_out, int dtype, void *stream);
 
+/*
+ * Device status of a call.  The first 4 bytes of the workspace of
+ * lcla_forward, lcla_forward_blocks, lcla_step and the shard calls hold an int
+ * that the call zeroes first (lcla_shard_end keeps lcla_shard_begin's) and
+ * that its tensor-core kernels OR bits into when one of their bounded waits
+ * (1 s) gives up: bit 0 pass A, bit 1 pass C.  A CTA that gives up lets its
+ * copies and MMAs in flight land, frees its tensor memory, writes NaN partial
+ * states and returns, so the outputs are NaN instead of the GPU hanging; the
+ * status is read once the stream has reached the call.
+ */
+#define LCLA_DEVICE_STATUS_PASS_A 1
+#define LCLA_DEVICE_STATUS_PASS_C 2
+
+/*
+ * Self-test of that bounded wait: one thread waits on an mbarrier phase with
+ * the kernels' wait.  arrive_first != 0: the phase is completed first and the
+ * wait must return at once; 0: nothing arrives and the wait must give up after
+ * its limit (about 1 s).  Writes result[0] = 1 if the wait gave up (else 0),
+ * result[1] = nanoseconds spent waiting, result[2] = the abort flag it left.
+ *   result   3 x uint64 device array, 8-byte aligned.
+ * Returns an lcla_status; the kernel runs on `stream`.
+ */
+LCLA_API int lcla_selftest_bounded_wait(int arrive_first, unsigned long long *result, void *stream);
+
 /* Static, human-readable name of a status code. */
 LCLA_API const char *lcla_status_string(int status);
 

@@ -69,6 +69,10 @@ def check_state(st, ref, what: str = "") -> tuple:
     with np.errstate(divide="ignore", invalid="ignore"):
         z_rel = np.where(zr > 0, np.abs(z - zr) / np.where(zr > 0, zr, 1.0), np.abs(z - zr))
     ws, wz = float(s_rel.max()), float(z_rel.max())
+    # also the per-(b, h) relative Frobenius error of S (reported, not a bar)
+    fden = np.sqrt((Sr ** 2).sum(axis=(-2, -1)))
+    fro = float((np.sqrt(((S - Sr) ** 2).sum(axis=(-2, -1))) / np.where(fden > 0, fden, 1.0)).max())
     if ws > STATE_TOL or wz > STATE_TOL:
-        raise AssertionError(f"{what}: state error S {ws:.3e}, z {wz:.3e} > {STATE_TOL:.0e}")
-    return ws, wz
+        raise AssertionError(f"{what}: state error S {ws:.3e}, z {wz:.3e} > {STATE_TOL:.0e} "
+                             f"(relative Frobenius {fro:.3e})")
+    return ws, wz, fro

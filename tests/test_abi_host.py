@@ -23,7 +23,8 @@ def test_every_declared_symbol_is_exported():
     assert {"lcla_forward", "lcla_step", "lcla_forward_workspace_bytes",
             "lcla_step_workspace_bytes", "lcla_status_string", "lcla_version",
             "lcla_forward_blocks", "lcla_forward_blocks_workspace_bytes", "lcla_temporal_conv",
-            "lcla_shard_begin", "lcla_shard_end", "lcla_shard_workspace_bytes"} <= set(names)
+            "lcla_shard_begin", "lcla_shard_end", "lcla_shard_workspace_bytes",
+            "lcla_selftest_bounded_wait"} <= set(names)
     lib = ctypes.CDLL(lcla.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -184,3 +185,9 @@ def test_shard_workspace_and_arguments():
     assert e(sin=9 * a, sout=9 * a + 128) == INVALID     # partial overlap of state_in and state_out
     assert e(ws=None, wsb=0) == WORKSPACE
     assert e(out=6 * a) == INVALID                       # out over the totals
+
+
+def test_selftest_arguments():
+    fn = lcla.lib.lcla_selftest_bounded_wait
+    assert fn(1, None, None) == INVALID
+    assert fn(1, (1 << 20) + 4, None) == MISALIGNED
