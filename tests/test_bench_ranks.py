@@ -83,3 +83,24 @@ def test_reference_arm_non_zero_rank_does_no_work(monkeypatch, capsys):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"])
     assert bench.run_reference(bench.parse()) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_rank0_prints_the_contract_line(monkeypatch, capsys):
+    """Rank 0 times the fp64 oracle on the tiny workload and prints one JSON line
+    with the keys the driver reads."""
+    import json
+    bench = load_bench()
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "tiny_f32",
+                                      "--steps", "2", "--warmup", "1"])
+    bench.run_reference(bench.parse())
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 1
+    assert d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
