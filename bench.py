@@ -85,7 +85,7 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-KERNEL_SOURCES = ("lcla_tc.cuh", "lcla_ffma.cuh", "lcla_plan.h")
+KERNEL_SOURCES = ("lcla_tc.cuh", "lcla_ffma.cuh", "lcla_plan.h", "lcla_tconv.cu")
 
 
 def source_digest():
@@ -386,7 +386,8 @@ def run_tconv(args):
             "config": {"workload": f"{w['name']}: B={B} F={F} S={S} C={C}", "cache": "previous frame, saved",
                        "l2": f"x and y {2 * units * 2 / 1e6:.0f} MB per step > 126 MB"},
             "roofline": {"bound": "hbm", "kernel": "temporal_conv_k2", "achieved": achieved, "peak": peak,
-                         "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": ncu_traffic("temporal_conv_k2", w["name"]),
                          "algorithmic_bytes": bytes_step},
             "cpu_baseline": {"value": n * units / el, "unit": "token*channels/s", "cores": 1, "kind": "oracle",
                              "sample": f"{n} whole call(s) of the numpy fp64 oracle, {el:.1f} s"},
