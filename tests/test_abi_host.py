@@ -191,3 +191,28 @@ def test_selftest_arguments():
     fn = lcla.lib.lcla_selftest_bounded_wait
     assert fn(1, None, None) == INVALID
     assert fn(1, (1 << 20) + 4, None) == MISALIGNED
+
+
+def test_header_compiles_as_c_and_a_c_program_links(tmp_path):
+    """The boundary is plain C: the header compiles as pedantic C99 and a C
+    program links against the library and calls it (the planner touches no
+    device)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text('#include "lcla.h"\n'
+                   "int main(void) {\n"
+                   "    int info[5];\n"
+                   "    if (lcla_forward_plan_info(1, 70, 32760, 32, 4680, LCLA_BF16, info) != LCLA_OK) return 1;\n"
+                   "    if (info[0] != 0 || info[4] != 1) return 2;\n"
+                   "    if (lcla_forward_workspace_bytes(1, 70, 32760, 64, 4680, LCLA_BF16) == 0) return 3;\n"
+                   "    return lcla_version() >= 100 ? 0 : 4;\n"
+                   "}\n")
+    libdir = os.path.dirname(lcla.LIB_PATH)
+    exe = tmp_path / "abi"
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           str(src), "-L", libdir, "-llcla", f"-Wl,-rpath,{libdir}", "-o", str(exe)])
+    assert subprocess.run([str(exe)]).returncode == 0
