@@ -347,9 +347,10 @@ int launch_all(const Tin *q, const Tin *k, const Tin *v, const float *rc, const 
         launch_pdl(lcla::pass_c_ffma<Tin>, grid, dim3(256), smem_c, st, q, rc, rs, p, (const float *)pref, eps, out);
     } else {
         const int smem_c = 3 * G::TILE_IN + 2 * G::TILE_TAB + 4 * G::TILE_F +
-                           (LCLA_HG * LCLA_T * LCLA_T + LCLA_HG * LCLA_D * LCLA_D + LCLA_HG * LCLA_D) * 4;
+                           (LCLA_HG * LCLA_T * LCLA_T + LCLA_HG * LCLA_D * LCLA_D + LCLA_HG * LCLA_D) * 4 +
+                           lcla::chunk_smem_extra<Tin>();
         set_smem(lcla::pass_c_chunk_ffma<Tin>, smem_c);
-        launch_pdl(lcla::pass_c_chunk_ffma<Tin>, grid, dim3(256), smem_c, st, q, k, v, rc, rs, p,
+        launch_pdl(lcla::pass_c_chunk_ffma<Tin>, grid, dim3(lcla::CHUNK_THREADS), smem_c, st, q, k, v, rc, rs, p,
                    (const float *)pref, eps, out);
     }
     if (ev) cudaEventRecord(ev[3], st);

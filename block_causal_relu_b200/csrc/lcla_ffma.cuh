@@ -397,10 +397,22 @@ pass_c_ffma(const Tin *__restrict__ q, const float *__restrict__ rcos, const flo
 // at the tile start):
 //   num_i = R_S q~_i + sum_{j in tile, blk(j) <= blk(i)} v_j (k~_j . q~_i)
 //   den_i = (R_z + sum_{same j} phi(k_j)) . phi(q_i) + eps
-// then R += the tile's (S, z).  grid (nseg, ngroups, B), 256 threads.
+// then R += the tile's (S, z).  grid (nseg * ngroups, B), CHUNK_THREADS threads.
 // ---------------------------------------------------------------------------
+constexpr int CHUNK_THREADS = 512;   // 16 warps: one CTA fills an SM's shared memory, so the warps are the latency hiding
+// Rows of the rotated features (token stride) and of the score matrix are padded by 4 floats: a
+// 128-bit shared access is served eight lanes at a time, and with 17 16-byte chunks per row the
+// rows of consecutive tokens fall on different bank groups.
+constexpr int CHUNK_QK_TS = LCLA_HG * LCLA_D + 4;   // floats per token row of qt / kt
+constexpr int CHUNK_SC_TS = LCLA_T + 4;             // floats per score row
+constexpr int CHUNK_RED_TS = LCLA_D + 1;           // floats per row of the per-token-group state partials
+// bytes beyond the unpadded layout: row padding, a second v tile (the next tile's v lands while this one's is
+// in use) and the key-sum run totals
 template <typename Tin>
-__global__ void __launch_bounds__(256)
+constexpr int chunk_smem_extra() { return (2 * LCLA_T * 4 + LCLA_HG * LCLA_T * 4 + 8 * LCLA_HG * LCLA_D) * 4 + Geo<Tin>::TILE_IN; }
+
+template <typename Tin>
+__global__ void __launch_bounds__(CHUNK_THREADS)
 pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                   const float *__restrict__ rcos, const float *__restrict__ rsin, const LclaPlan p,
                   const float *__restrict__ pref, const float eps, Tin *__restrict__ out)
@@ -409,16 +421,17 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
     extern __shared__ __align__(128) unsigned char sm[];
     unsigned char *qraw_b = sm;
     unsigned char *kraw_b = qraw_b + G::TILE_IN;
-    unsigned char *vraw_b = kraw_b + G::TILE_IN;
-    unsigned char *ct_b = vraw_b + G::TILE_IN;
+    unsigned char *vraw_b = kraw_b + G::TILE_IN;                       // two v tiles: this one, the next
+    unsigned char *ct_b = vraw_b + 2 * G::TILE_IN;
     unsigned char *st_b = ct_b + G::TILE_TAB;
-    float *qt = reinterpret_cast<float *>(st_b + G::TILE_TAB);        // [T][HG][D] rotated q
-    float *kt = qt + LCLA_T * LCLA_HG * LCLA_D;                       // rotated k
-    float *fq = kt + LCLA_T * LCLA_HG * LCLA_D;                       // phi(q)
+    float *qt = reinterpret_cast<float *>(st_b + G::TILE_TAB);        // [T][CHUNK_QK_TS] rotated q: [HG][D] + pad
+    float *kt = qt + LCLA_T * CHUNK_QK_TS;                            // rotated k, same rows
+    float *fq = kt + LCLA_T * CHUNK_QK_TS;                            // [T][HG][D] phi(q)
     float *fk = fq + LCLA_T * LCLA_HG * LCLA_D;                       // phi(k), then its running sum
-    float *sc = fk + LCLA_T * LCLA_HG * LCLA_D;                       // [HG][T j][T i] scores / reduction
-    float *RT = sc + LCLA_HG * LCLA_T * LCLA_T;                       // [HG][D e][D c]
+    float *sc = fk + LCLA_T * LCLA_HG * LCLA_D;                       // [HG][T j][CHUNK_SC_TS] scores / reduction
+    float *RT = sc + LCLA_HG * LCLA_T * CHUNK_SC_TS;                  // [HG][D e][D c]
     float *Rz = RT + LCLA_HG * LCLA_D * LCLA_D;                       // [HG][D]
+    float *ktot = Rz + LCLA_HG * LCLA_D;                              // [8 runs][HG][D] key-sum run totals
 
     const int s = blockIdx.x / p.ngroups, h0 = (blockIdx.x % p.ngroups) * LCLA_HG, b = blockIdx.y;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -428,7 +441,7 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
     if (ntile <= 0) return;
     pdl_wait();
 
-    for (int x = tid; x < LCLA_HG * LCLA_SZ; x += 256) {
+    for (int x = tid; x < LCLA_HG * LCLA_SZ; x += CHUNK_THREADS) {
         const int hh = x / LCLA_SZ, e = x - hh * LCLA_SZ;
         float val = 0.f;
         if (h0 + hh < p.H) val = pref[(((size_t)s * p.B + b) * p.H + (h0 + hh)) * LCLA_SZ + e];
@@ -436,45 +449,55 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
         else Rz[hh * LCLA_D + (e - LCLA_D * LCLA_D)] = val;
     }
 
-    const int ohh = w >> 2, otq = (w & 3) * 16 + (lane >> 3) * 4;
+    // outputs: warp w -> head w / 8 and tokens [8 (w % 8), +8); lane -> 2 tokens (lane / 8) and 4 channels
+    const int ohh = w >> 3, otq = (w & 7) * 8 + (lane >> 3) * 2;
     const int c0 = (lane & 7) * 4;
 
+    // one cp.async group per tile: q, k and the tables (free once the tile's prologue is done) and v into
+    // the v tile the tile before last used
+    auto issue_tile = [&](int ii) {
+        const int tt = g.t0 + ii * T, ntt = min(T, g.t1 - tt);
+        issue_rows<Tin>(qraw_b, q, p, b, tt, ntt, h0, tid, CHUNK_THREADS);
+        issue_rows<Tin>(kraw_b, k, p, b, tt, ntt, h0, tid, CHUNK_THREADS);
+        issue_rows<Tin>(vraw_b + (ii & 1) * G::TILE_IN, v, p, b, tt, ntt, h0, tid, CHUNK_THREADS);
+        issue_table(ct_b, rcos, tt, ntt, tid, CHUNK_THREADS);
+        issue_table(st_b, rsin, tt, ntt, tid, CHUNK_THREADS);
+        cp_async_commit();
+    };
+    issue_tile(0);
     for (int i = 0; i < ntile; ++i) {
         const int t = g.t0 + i * T, nt = min(T, g.t1 - t);
-        issue_rows<Tin>(qraw_b, q, p, b, t, nt, h0, tid, 256);
-        issue_rows<Tin>(kraw_b, k, p, b, t, nt, h0, tid, 256);
-        issue_rows<Tin>(vraw_b, v, p, b, t, nt, h0, tid, 256);
-        issue_table(ct_b, rcos, t, nt, tid, 256);
-        issue_table(st_b, rsin, t, nt, tid, 256);
-        cp_async_commit();
         cp_async_wait<0>();
         __syncthreads();
         const Tin *qraw = reinterpret_cast<const Tin *>(qraw_b);
         const Tin *kraw = reinterpret_cast<const Tin *>(kraw_b);
-        const Tin *vraw = reinterpret_cast<const Tin *>(vraw_b);
+        const Tin *vraw = reinterpret_cast<const Tin *>(vraw_b + (i & 1) * G::TILE_IN);
         const float *ct = reinterpret_cast<const float *>(ct_b);
         const float *st = reinterpret_cast<const float *>(st_b);
 
         // prologue for q and k (rows past nt are zero-filled, so they give zeros)
-        for (int it = tid; it < LCLA_T * LCLA_HG * 4; it += 256) {
+        for (int it = tid; it < LCLA_T * LCLA_HG * 4; it += CHUNK_THREADS) {
             const int tok = it >> 3, hh = (it >> 2) & 1, qtr = it & 3;
             const float4 c4 = reinterpret_cast<const float4 *>(ct + tok * (LCLA_D / 2))[qtr];
             const float4 s4 = reinterpret_cast<const float4 *>(st + tok * (LCLA_D / 2))[qtr];
             const int o = (tok * LCLA_HG + hh) * LCLA_D + qtr * 8;
+            const int ot = tok * CHUNK_QK_TS + hh * LCLA_D + qtr * 8;
             float x[8], f[8], y[8];
             load8(qraw + o, x);
             relu_rope8(x, c4, s4, f, y);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) { fq[o + j] = f[j]; qt[o + j] = y[j]; }
+            for (int j = 0; j < 8; ++j) { fq[o + j] = f[j]; qt[ot + j] = y[j]; }
             load8(kraw + o, x);
             relu_rope8(x, c4, s4, f, y);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) { fk[o + j] = f[j]; kt[o + j] = y[j]; }
+            for (int j = 0; j < 8; ++j) { fk[o + j] = f[j]; kt[ot + j] = y[j]; }
         }
         __syncthreads();
+        if (i + 1 < ntile) issue_tile(i + 1);   // the prologue has consumed q, k and the tables
 
-        // scores sc[hh][j][i] = [blk(j) <= blk(i)] (k~_j . q~_i), 4x4 blocks
-        for (int blkid = tid; blkid < LCLA_HG * 16 * 16; blkid += 256) {
+        // scores sc[hh][j][i] = [blk(j) <= blk(i)] (k~_j . q~_i); a thread takes queries ib*4..+3 and keys
+        // jb, jb+16, jb+32, jb+48, so that the lanes of a warp read consecutive key rows
+        for (int blkid = tid; blkid < LCLA_HG * 16 * 16; blkid += CHUNK_THREADS) {
             const int hh = blkid >> 8, ib = (blkid >> 4) & 15, jb = blkid & 15;
             float a[4][4];
 #pragma unroll
@@ -486,8 +509,8 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
                 float4 qv[4], kv[4];
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
-                    qv[x] = *reinterpret_cast<const float4 *>(qt + ((ib * 4 + x) * LCLA_HG + hh) * LCLA_D + e4 * 4);
-                    kv[x] = *reinterpret_cast<const float4 *>(kt + ((jb * 4 + x) * LCLA_HG + hh) * LCLA_D + e4 * 4);
+                    qv[x] = *reinterpret_cast<const float4 *>(qt + (ib * 4 + x) * CHUNK_QK_TS + hh * LCLA_D + e4 * 4);
+                    kv[x] = *reinterpret_cast<const float4 *>(kt + (jb + 16 * x) * CHUNK_QK_TS + hh * LCLA_D + e4 * 4);
                 }
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii)
@@ -498,44 +521,53 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
             }
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
-                const int j = jb * 4 + jj;
+                const int j = jb + 16 * jj;
                 float o4[4];
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii) {
                     const int i2 = ib * 4 + ii;
                     o4[ii] = (j < nt && (j / L) <= (i2 / L)) ? a[ii][jj] : 0.f;
                 }
-                *reinterpret_cast<float4 *>(sc + (hh * LCLA_T + j) * LCLA_T + ib * 4) =
+                *reinterpret_cast<float4 *>(sc + (hh * LCLA_T + j) * CHUNK_SC_TS + ib * 4) =
                     make_float4(o4[0], o4[1], o4[2], o4[3]);
             }
         }
-        // running key sum over the tile, in token order, one thread per (head, dim)
-        if (tid < LCLA_HG * LCLA_D) {
-            const int hh = tid >> 5, e = tid & 31;
-            float run = 0.f;
-            for (int j = 0; j < nt; ++j) {
-                run += fk[(j * LCLA_HG + hh) * LCLA_D + e];
-                fk[(j * LCLA_HG + hh) * LCLA_D + e] = run;
+        // running key sum over the tile in token order: 8 runs of 8 tokens per (head, dim) column, run r in
+        // warps 2r, 2r+1 (consecutive lanes take consecutive columns), then each run adds the earlier runs' totals
+        {
+            const int col = tid & (LCLA_HG * LCLA_D - 1), r = tid / (LCLA_HG * LCLA_D);
+            const int hh = col / LCLA_D, e = col % LCLA_D;
+            float run[8], acc = 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                acc += fk[((r * 8 + u) * LCLA_HG + hh) * LCLA_D + e];
+                run[u] = acc;
             }
+            ktot[r * LCLA_HG * LCLA_D + col] = acc;
+            __syncthreads();
+            float off = 0.f;
+            for (int r2 = 0; r2 < r; ++r2) off += ktot[r2 * LCLA_HG * LCLA_D + col];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) fk[((r * 8 + u) * LCLA_HG + hh) * LCLA_D + e] = run[u] + off;
         }
         __syncthreads();
 
         // outputs
-        float acc[4][4];
+        float acc[2][4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
         for (int e4 = 0; e4 < LCLA_D / 4; ++e4) {      // carried state
-            float4 qv[4], pv[4];
+            float4 qv[2], pv[4];
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
-                qv[a] = *reinterpret_cast<const float4 *>(qt + ((otq + a) * LCLA_HG + ohh) * LCLA_D + e4 * 4);
+            for (int a = 0; a < 2; ++a)
+                qv[a] = *reinterpret_cast<const float4 *>(qt + (otq + a) * CHUNK_QK_TS + ohh * LCLA_D + e4 * 4);
 #pragma unroll
             for (int m = 0; m < 4; ++m)
                 pv[m] = *reinterpret_cast<const float4 *>(RT + ohh * LCLA_D * LCLA_D + (e4 * 4 + m) * LCLA_D + c0);
 #pragma unroll
-            for (int a = 0; a < 4; ++a) {
+            for (int a = 0; a < 2; ++a) {
                 const float qq[4] = {qv[a].x, qv[a].y, qv[a].z, qv[a].w};
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
@@ -547,19 +579,19 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
             }
         }
         for (int j = 0; j < nt; ++j) {                 // masked in-tile term
-            const float4 sv = *reinterpret_cast<const float4 *>(sc + (ohh * LCLA_T + j) * LCLA_T + otq);
+            const float2 sv = *reinterpret_cast<const float2 *>(sc + (ohh * LCLA_T + j) * CHUNK_SC_TS + otq);
             float vv[4];
             load4(vraw + (j * LCLA_HG + ohh) * LCLA_D + c0, vv);
-            const float ss[4] = {sv.x, sv.y, sv.z, sv.w};
+            const float ss[2] = {sv.x, sv.y};
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 2; ++a)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(ss[a], vv[c], acc[a][c]);
         }
-        // denominators: the 8 lanes sharing these 4 tokens split the key dims
-        float den[4];
+        // denominators: the 8 lanes sharing these 2 tokens split the key dims
+        float den[2];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
+        for (int a = 0; a < 2; ++a) {
             const int tok = otq + a;
             const int last = min(nt, (tok / L + 1) * L) - 1;   // last in-tile token of tok's block
             const int lc = last < 0 ? 0 : last;
@@ -577,7 +609,7 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
         }
         if (h0 + ohh < p.H) {
 #pragma unroll
-            for (int a = 0; a < 4; ++a) {
+            for (int a = 0; a < 2; ++a) {
                 const int tok = otq + a;
                 if (tok < nt) {
                     const float r = 1.0f / den[a];
@@ -588,37 +620,50 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
         }
         __syncthreads();
 
-        // R += tile state: per-warp partial over 16 tokens, fixed-order sum
+        // R += tile state: warp w -> head w / 8, tokens [16 ((w / 2) % 4), +16), value dims [16 (w % 2), +16);
+        // lane -> 2 value dims x 8 key dims; the four token groups of a head are summed in a fixed order
         {
-            const int rc0 = (lane >> 2) * 4, re0 = (lane & 3) * 8, rtq = (w & 3) * 16;
-            float ra[4][8];
+            const int shh = w >> 3, tg = (w >> 1) & 3, half = w & 1;
+            const int rc0 = half * 16 + (lane >> 2) * 2, re0 = (lane & 3) * 8, rtq = tg * 16;
+            float ra[2][8];
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii)
+            for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) ra[ii][j] = 0.f;
             for (int tt = 0; tt < 16; ++tt) {
                 const int tok = rtq + tt;
-                float vv[4];
-                load4(vraw + (tok * LCLA_HG + ohh) * LCLA_D + rc0, vv);
-                const float4 ka = *reinterpret_cast<const float4 *>(kt + (tok * LCLA_HG + ohh) * LCLA_D + re0);
-                const float4 kb = *reinterpret_cast<const float4 *>(kt + (tok * LCLA_HG + ohh) * LCLA_D + re0 + 4);
+                const Tin *vp = vraw + (tok * LCLA_HG + shh) * LCLA_D + rc0;
+                float vv[2];
+                if constexpr (sizeof(Tin) == 2) {
+                    const uint32_t u = *reinterpret_cast<const uint32_t *>(vp);
+                    vv[0] = bf_lo(u);
+                    vv[1] = bf_hi(u);
+                } else {
+                    const float2 f2 = *reinterpret_cast<const float2 *>(vp);
+                    vv[0] = f2.x;
+                    vv[1] = f2.y;
+                }
+                const float4 ka = *reinterpret_cast<const float4 *>(kt + tok * CHUNK_QK_TS + shh * LCLA_D + re0);
+                const float4 kb = *reinterpret_cast<const float4 *>(kt + tok * CHUNK_QK_TS + shh * LCLA_D + re0 + 4);
                 const float kk[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-                for (int ii = 0; ii < 4; ++ii)
+                for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
                     for (int j = 0; j < 8; ++j) ra[ii][j] = fmaf(vv[ii], kk[j], ra[ii][j]);
             }
-            float *red = sc;                                 // [8 warps][D c][D e]
+            float *red = sc;                                 // [2 heads][4 token groups][D c][CHUNK_RED_TS]
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii)
+            for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) red[w * LCLA_D * LCLA_D + (rc0 + ii) * LCLA_D + re0 + j] = ra[ii][j];
+                for (int j = 0; j < 8; ++j)
+                    red[((shh * 4 + tg) * LCLA_D + rc0 + ii) * CHUNK_RED_TS + re0 + j] = ra[ii][j];
         }
         __syncthreads();
-        for (int x = tid; x < LCLA_HG * LCLA_D * LCLA_D; x += 256) {
-            const int hh = x >> 10, ce = x & 1023, c = ce >> 5, e = ce & 31;
-            const float *r = sc + (hh * 4) * LCLA_D * LCLA_D + ce;
-            const float add = ((r[0] + r[LCLA_D * LCLA_D]) + r[2 * LCLA_D * LCLA_D]) + r[3 * LCLA_D * LCLA_D];
+        for (int x = tid; x < LCLA_HG * LCLA_D * LCLA_D; x += CHUNK_THREADS) {   // lanes: consecutive c
+            const int hh = x >> 10, ec = x & 1023, e = ec >> 5, c = ec & 31;
+            constexpr int G4 = LCLA_D * CHUNK_RED_TS;    // one token group's partial
+            const float *r = sc + (hh * 4) * G4 + c * CHUNK_RED_TS + e;
+            const float add = ((r[0] + r[G4]) + r[2 * G4]) + r[3 * G4];
             RT[hh * LCLA_D * LCLA_D + e * LCLA_D + c] += add;
         }
         if (tid < LCLA_HG * LCLA_D && nt > 0) {
