@@ -85,7 +85,9 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-KERNEL_SOURCES = ("lcla_tc.cuh", "lcla_ffma.cuh", "lcla_plan.h", "lcla_tconv.cu")
+# the files the profiled kernels are built from (tensor-core passes, the scans, the temporal convolution);
+# the CUDA-core passes in lcla_ffma.cuh and lcla_gen.cuh have no traffic record
+KERNEL_SOURCES = ("lcla_common.cuh", "lcla_scan.cuh", "lcla_tc.cuh", "lcla_plan.h", "lcla_tconv.cu")
 
 
 def source_digest():

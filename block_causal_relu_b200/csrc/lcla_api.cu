@@ -19,6 +19,7 @@
 
 #include "lcla.h"
 #include "lcla_ffma.cuh"
+#include "lcla_scan.cuh"
 #include "lcla_gen.cuh"
 #include "lcla_plan.h"
 #include "lcla_selftest.cuh"

@@ -19,136 +19,10 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "lcla_common.cuh"
 #include "lcla_plan.h"
 
 namespace lcla {
-
-// ---------------------------------------------------------------------------
-// small device helpers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid)
-{
-    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-    const int n = valid ? 16 : 0;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
-
-// Programmatic dependent launch: wait until the preceding kernel of the
-// stream has completed (no-op when launched without the attribute), and let
-// the next kernel of the stream start its launch.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-// ReLU written as a comparison so that NaN passes through.
-__device__ __forceinline__ float relu(float x) { return x < 0.f ? 0.f : x; }
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-// 8 consecutive elements -> fp32
-__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float *x)
-{
-    const uint4 u = *reinterpret_cast<const uint4 *>(p);
-    x[0] = bf_lo(u.x); x[1] = bf_hi(u.x); x[2] = bf_lo(u.y); x[3] = bf_hi(u.y);
-    x[4] = bf_lo(u.z); x[5] = bf_hi(u.z); x[6] = bf_lo(u.w); x[7] = bf_hi(u.w);
-}
-__device__ __forceinline__ void load8(const float *p, float *x)
-{
-    const float4 a = reinterpret_cast<const float4 *>(p)[0];
-    const float4 b = reinterpret_cast<const float4 *>(p)[1];
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-// 4 consecutive elements -> fp32
-__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float *x)
-{
-    const uint2 u = *reinterpret_cast<const uint2 *>(p);
-    x[0] = bf_lo(u.x); x[1] = bf_hi(u.x); x[2] = bf_lo(u.y); x[3] = bf_hi(u.y);
-}
-__device__ __forceinline__ void load4(const float *p, float *x)
-{
-    const float4 a = *reinterpret_cast<const float4 *>(p);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-}
-// 4 fp32 -> 4 consecutive outputs (bf16 round-to-nearest-even)
-__device__ __forceinline__ void store4(__nv_bfloat16 *p, const float *x)
-{
-    __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]);
-    __nv_bfloat162 b = __floats2bfloat162_rn(x[2], x[3]);
-    uint2 u;
-    u.x = *reinterpret_cast<uint32_t *>(&a);
-    u.y = *reinterpret_cast<uint32_t *>(&b);
-    *reinterpret_cast<uint2 *>(p) = u;
-}
-__device__ __forceinline__ void store4(float *p, const float *x)
-{
-    *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
-}
-
-// phi then the rotary embedding on 8 consecutive elements (4 pairs) of a head
-// row; x holds the raw values on entry, f the ReLU features and y the rotated
-// features on exit.  c4/s4 are the 4 table entries of these pairs.
-__device__ __forceinline__ void relu_rope8(const float *x, const float4 &c4, const float4 &s4,
-                                           float *f, float *y)
-{
-#pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] = relu(x[i]);
-    const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
-    const float ss[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const float a = f[2 * p], b = f[2 * p + 1];
-        y[2 * p] = a * cc[p] - b * ss[p];
-        y[2 * p + 1] = a * ss[p] + b * cc[p];
-    }
-}
-
-// Tile geometry for one input type.
-template <typename Tin>
-struct Geo {
-    static constexpr int EB = (int)sizeof(Tin);
-    static constexpr int ROWB = LCLA_D * EB;                  // bytes of one head row
-    static constexpr int CPR = ROWB / 16;                     // 16-byte chunks per head row
-    static constexpr int TILE_IN = LCLA_T * LCLA_HG * ROWB;   // one input tile [T][HG][D]
-    static constexpr int TILE_TAB = LCLA_T * (LCLA_D / 2) * 4; // one table tile [T][D/2] fp32
-    static constexpr int TILE_F = LCLA_T * LCLA_HG * LCLA_D * 4; // fp32 tile [T][HG][D]
-};
-
-// Queue cp.async copies of rows [t, t + nt) of an input tensor for heads
-// h0, h0+1 into buf ([T][HG][D] elements); rows and heads outside the valid
-// range are zero-filled without reading global memory.
-template <typename Tin>
-__device__ __forceinline__ void issue_rows(unsigned char *buf, const Tin *src, const LclaPlan &p,
-                                           int b, int t, int nt, int h0, int tid, int nthr)
-{
-    using G = Geo<Tin>;
-    for (int c = tid; c < LCLA_T * LCLA_HG * G::CPR; c += nthr) {
-        const int tok = c / (LCLA_HG * G::CPR);
-        const int rem = c - tok * (LCLA_HG * G::CPR);
-        const int hh = rem / G::CPR;
-        const int part = rem - hh * G::CPR;
-        const bool ok = tok < nt && h0 + hh < p.H;
-        const size_t off = ok ? ((((size_t)b * p.N + (size_t)(t + tok)) * p.H + (size_t)(h0 + hh)) *
-                                     LCLA_D) * G::EB + (size_t)part * 16
-                              : 0;
-        cp_async16(buf + (size_t)c * 16, reinterpret_cast<const unsigned char *>(src) + off, ok);
-    }
-}
-
-// Same for the [N, D/2] fp32 tables.
-__device__ __forceinline__ void issue_table(unsigned char *buf, const float *tab, int t, int nt,
-                                            int tid, int nthr)
-{
-    for (int c = tid; c < LCLA_T * 4; c += nthr) {
-        const int tok = c >> 2, part = c & 3;
-        const bool ok = tok < nt;
-        const size_t off = ok ? (size_t)(t + tok) * (LCLA_D / 2) * 4 + (size_t)part * 16 : 0;
-        cp_async16(buf + (size_t)c * 16, reinterpret_cast<const unsigned char *>(tab) + off, ok);
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Pass A: segment partial states.  grid (nseg, ngroups, B), 256 threads.
@@ -671,171 +545,6 @@ pass_c_chunk_ffma(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
             Rz[hh * LCLA_D + e] += fk[((nt - 1) * LCLA_HG + hh) * LCLA_D + e];
         }
         __syncthreads();
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Scan: partials -> prefixes, one thread per 4 consecutive state elements
-// (b, h, x..x+3) with x < (D+1)*D; the segment partials are loaded as float4
-// in batches of independent loads and summed in a fixed order.
-// Block mode: pref[blk] = state_in + sum of all segments of blocks <= blk.
-// Chunk mode: pref[s]   = state_in + sum of segments < s.
-// state_out (may equal state_in) receives the total.
-// ---------------------------------------------------------------------------
-constexpr int SCAN_THREADS = 128;
-constexpr int SCAN_VEC = 4;   // elements per thread (a state's (d + 1) * d floats are a multiple of 4 for even d)
-
-__device__ __forceinline__ void add4(float4 &a, const float4 &b)
-{
-    a.x += b.x;
-    a.y += b.y;
-    a.z += b.z;
-    a.w += b.w;
-}
-
-// Chunked scan, for more groups than the grouped scan holds: the segments are
-// cut into chunks of p.scs segments (whole groups).  scan_chunk_totals sums
-// each chunk in segment order (grid: column blocks x chunks) and copies
-// state_in after the chunk totals; scan_chunk_prefix starts each chunk from
-// state_in plus the totals of the chunks before it, walks the chunk's
-// segments and writes the same prefixes as the one-pass scans, and the last
-// chunk writes the total.  Only the first kernel reads state_in, so state_out
-// may alias it.
-// ---------------------------------------------------------------------------
-constexpr int SCAN_CHUNK_GROUPS = 32;
-
-__global__ void __launch_bounds__(SCAN_THREADS)
-scan_chunk_totals(const LclaPlan p, const float *__restrict__ part, const float *state_in, float *__restrict__ ctot)
-{
-    constexpr int BATCH = 16;
-    const size_t n4 = (size_t)p.B * p.H * (p.sz / SCAN_VEC);
-    const size_t x = (size_t)blockIdx.x * SCAN_THREADS + threadIdx.x;
-    const int c = blockIdx.y;
-    pdl_wait();
-    pdl_trigger();
-    if (x >= n4) return;
-    const float4 *part4 = reinterpret_cast<const float4 *>(part);
-    float4 *ctot4 = reinterpret_cast<float4 *>(ctot);
-    const int s0 = c * p.scs, s1 = min(s0 + p.scs, p.nseg);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sb = s0; sb < s1; sb += BATCH) {
-        float4 v[BATCH];
-#pragma unroll
-        for (int j = 0; j < BATCH; ++j)
-            if (sb + j < s1) v[j] = __ldcg(part4 + (size_t)(sb + j) * n4 + x);
-#pragma unroll
-        for (int j = 0; j < BATCH; ++j)
-            if (sb + j < s1) add4(acc, v[j]);
-    }
-    ctot4[(size_t)c * n4 + x] = acc;
-    if (c == 0)
-        ctot4[(size_t)p.nch * n4 + x] = state_in ? reinterpret_cast<const float4 *>(state_in)[x]
-                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-}
-
-__global__ void __launch_bounds__(SCAN_THREADS)
-scan_chunk_prefix(const LclaPlan p, const float *__restrict__ part, const float *__restrict__ ctot,
-                  float *__restrict__ pref, float *state_out)
-{
-    constexpr int BATCH = 16;
-    const size_t n4 = (size_t)p.B * p.H * (p.sz / SCAN_VEC);
-    const size_t x = (size_t)blockIdx.x * SCAN_THREADS + threadIdx.x;
-    const int c = blockIdx.y;
-    pdl_wait();
-    pdl_trigger();
-    if (x >= n4) return;
-    const float4 *part4 = reinterpret_cast<const float4 *>(part);
-    const float4 *ctot4 = reinterpret_cast<const float4 *>(ctot);
-    float4 *pref4 = reinterpret_cast<float4 *>(pref);
-    float4 acc = __ldcg(ctot4 + (size_t)p.nch * n4 + x);   // state_in
-    for (int cb = 0; cb < c; cb += BATCH) {
-        float4 v[BATCH];
-#pragma unroll
-        for (int j = 0; j < BATCH; ++j)
-            if (cb + j < c) v[j] = __ldcg(ctot4 + (size_t)(cb + j) * n4 + x);
-#pragma unroll
-        for (int j = 0; j < BATCH; ++j)
-            if (cb + j < c) add4(acc, v[j]);
-    }
-    const int s0 = c * p.scs, s1 = min(s0 + p.scs, p.nseg);
-    for (int sb = s0; sb < s1; sb += BATCH) {
-        float4 v[BATCH];
-#pragma unroll
-        for (int j = 0; j < BATCH; ++j)
-            if (sb + j < s1) v[j] = __ldcg(part4 + (size_t)(sb + j) * n4 + x);
-#pragma unroll
-        for (int j = 0; j < BATCH; ++j) {
-            const int sg = sb + j;
-            if (sg < s1) {
-                if (p.chunk) pref4[(size_t)sg * n4 + x] = acc;
-                add4(acc, v[j]);
-                if (!p.chunk && (sg + 1) % p.nsb == 0) pref4[(size_t)(sg / p.nsb) * n4 + x] = acc;
-            }
-        }
-    }
-    if (state_out && c == p.nch - 1) reinterpret_cast<float4 *>(state_out)[x] = acc;
-}
-
-// Grouped scan: the same prefixes in two phases, for up to SCANG_MAX_GROUPS
-// groups (block mode: a block's nsb segments; chunk mode: one segment).  A
-// CTA owns 32 float4 columns of the state slice; phase 1 has its 8 warps sum
-// the groups' segment partials in parallel (all loads of a group in flight)
-// into shared memory; phase 2 has one warp run the prefix over the group sums
-// in group order and write pref (inclusive per block in block mode,
-// exclusive per segment in chunk mode) and the total.
-// ---------------------------------------------------------------------------
-constexpr int SCANG_WARPS = 8;
-constexpr int SCANG_MAX_GROUPS = 256;   // shared memory: groups x 32 x 16 B
-
-__device__ __forceinline__ void st_v4_keep(float4 *p, float4 v, uint64_t pol)
-{
-    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;"
-                 ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
-                 : "memory");
-}
-
-__global__ void __launch_bounds__(32 * SCANG_WARPS)
-scan_states_grouped(const LclaPlan p, const float *__restrict__ part, float *__restrict__ pref,
-                    const float *state_in, float *state_out)
-{
-    extern __shared__ float4 gsum[];   // [groups][32]
-    const size_t n4 = (size_t)p.B * p.H * (p.sz / SCAN_VEC);
-    const int lane = threadIdx.x & 31, wg = threadIdx.x >> 5;
-    const size_t x = (size_t)blockIdx.x * 32 + lane;
-    const bool live = x < n4;
-    const int ngroups = p.chunk ? p.nseg : p.nb, per = p.chunk ? 1 : p.nsb;
-    const float4 *part4 = reinterpret_cast<const float4 *>(part);
-    pdl_wait();
-    pdl_trigger();
-    for (int gi = wg; gi < ngroups; gi += SCANG_WARPS) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (live) {
-            constexpr int BATCH = 8;
-            for (int s0 = 0; s0 < per; s0 += BATCH) {
-                float4 v[BATCH];
-#pragma unroll
-                for (int j = 0; j < BATCH; ++j)
-                    if (s0 + j < per) v[j] = __ldcg(part4 + ((size_t)gi * per + s0 + j) * n4 + x);
-#pragma unroll
-                for (int j = 0; j < BATCH; ++j)
-                    if (s0 + j < per) add4(acc, v[j]);
-            }
-        }
-        gsum[gi * 32 + lane] = acc;
-    }
-    __syncthreads();
-    if (wg == 0 && live) {
-        float4 *pref4 = reinterpret_cast<float4 *>(pref);
-        float4 acc = state_in ? reinterpret_cast<const float4 *>(state_in)[x] : make_float4(0.f, 0.f, 0.f, 0.f);
-        uint64_t keep;   // the prefixes are read back by the next kernel: keep them in L2
-        asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
-        for (int gi = 0; gi < ngroups; ++gi) {
-            const float4 v = gsum[gi * 32 + lane];
-            if (p.chunk) st_v4_keep(pref4 + (size_t)gi * n4 + x, acc, keep);
-            add4(acc, v);
-            if (!p.chunk) st_v4_keep(pref4 + (size_t)gi * n4 + x, acc, keep);
-        }
-        if (state_out) reinterpret_cast<float4 *>(state_out)[x] = acc;
     }
 }
 

@@ -20,7 +20,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "lcla_ffma.cuh"
+#include "lcla_common.cuh"
 #include "lcla_plan.h"
 
 namespace lcla {

@@ -2,7 +2,7 @@
 // unsharded forward does not have (lcla_shard_end in include/lcla.h).
 #pragma once
 
-#include "lcla_ffma.cuh"
+#include "lcla_scan.cuh"
 
 namespace lcla {
 

@@ -61,7 +61,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "lcla_ffma.cuh"
+#include "lcla_common.cuh"
 #include "lcla_plan.h"
 
 #define LCLA_TC_WAIT_NS 1000000000ull   // 1 s: far above any legitimate wait
