@@ -66,6 +66,8 @@ def _load() -> ctypes.CDLL:
     L.lcla_selftest_bounded_wait.argtypes = [I, P, P]
     L.lcla_selftest_bounded_wait.restype = I
     L.lcla_forward_plan_info.argtypes = [I, I, I, I, I, I, P]
+    L.lcla_forward_plan_segments.argtypes = [I, I, I, I, I, I, P, P, P, I]
+    L.lcla_forward_plan_segments.restype = I
     L.lcla_forward_plan_info.restype = I
     L.lcla_status_string.argtypes = [I]
     L.lcla_status_string.restype = ctypes.c_char_p
@@ -129,6 +131,14 @@ def plan_info(B: int, H: int, N: int, d: int, block_len: int, dtype: int) -> dic
     _check(lib.lcla_forward_plan_info(B, H, N, d, block_len, dtype, info))
     return {"chunk_mode": bool(info[0]), "segments": info[1], "prefixes": info[2],
             "tile_tokens": info[3], "tensor_cores": bool(info[4])}
+
+
+def plan_segments(B: int, H: int, N: int, d: int, block_len: int, dtype: int) -> list:
+    """``lcla_forward_plan_segments``: [(t0, t1, block or -1), ...] per segment."""
+    n = plan_info(B, H, N, d, block_len, dtype)["segments"]
+    arr = [(ctypes.c_int * max(n, 1))() for _ in range(3)]
+    _check(lib.lcla_forward_plan_segments(B, H, N, d, block_len, dtype, arr[0], arr[1], arr[2], n))
+    return [(arr[0][i], arr[1][i], arr[2][i]) for i in range(n)]
 
 
 def _stream(stream, device) -> int:

@@ -656,6 +656,24 @@ int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,
     return LCLA_OK;
 }
 
+int lcla_forward_plan_segments(int B, int H, int N, int d, int block_len, int dtype, int *seg_t0, int *seg_t1,
+                               int *seg_blk, int capacity)
+{
+    const int rc = check_shape(B, H, N, d, block_len, dtype);
+    if (rc != LCLA_OK) return rc;
+    if (!seg_t0 || !seg_t1 || !seg_blk) return LCLA_ERR_INVALID_ARG;
+    const LclaPlan p = make_plan(B, H, N, block_len, dtype, 0, d);
+    if (!grid_fits(p)) return LCLA_ERR_UNSUPPORTED;
+    if (capacity < p.nseg) return LCLA_ERR_INVALID_ARG;
+    for (int s = 0; s < p.nseg; ++s) {   // the segment map the kernels evaluate, here on the host
+        const LclaSeg g = lcla_segment(p, s);
+        seg_t0[s] = g.t0;
+        seg_t1[s] = g.t1;
+        seg_blk[s] = g.blk;
+    }
+    return LCLA_OK;
+}
+
 const char *lcla_status_string(int status)
 {
     switch (status) {

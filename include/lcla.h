@@ -287,6 +287,17 @@ LCLA_API int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, i
                                     int *info);
 
 /*
+ * The segments lcla_forward cuts this problem into (uniform blocks), from the
+ * same segment map the kernels evaluate: segment s covers tokens
+ * [seg_t0[s], seg_t1[s]) (possibly empty) and, in block mode, lies in block
+ * seg_blk[s] (-1 in chunk mode).  The three int arrays are HOST memory of at
+ * least `capacity` entries; capacity must be >= info[1] of
+ * lcla_forward_plan_info.  Returns an lcla_status; touches no device.
+ */
+LCLA_API int lcla_forward_plan_segments(int B, int H, int N, int d, int block_len, int dtype,
+                                        int *seg_t0, int *seg_t1, int *seg_blk, int capacity);
+
+/*
  * lcla_forward for callers that cannot allocate device memory.  (The paper
  * has no counterpart: this is a packaging choice of this library.)
  *
