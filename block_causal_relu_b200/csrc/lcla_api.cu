@@ -679,7 +679,7 @@ const char *lcla_status_string(int status)
     switch (status) {
     case LCLA_OK: return "ok";
     case LCLA_ERR_INVALID_ARG: return "invalid argument";
-    case LCLA_ERR_UNSUPPORTED: return "unsupported problem (this build serves d = 32 and 64, N <= 2^30)";
+    case LCLA_ERR_UNSUPPORTED: return "unsupported problem (the library serves d = 32 and 64, N <= 2^30)";
     case LCLA_ERR_MISALIGNED: return "array pointer not 16-byte aligned";
     case LCLA_ERR_WORKSPACE: return "workspace missing or too small";
     case LCLA_ERR_CUDA: return "CUDA launch failed";

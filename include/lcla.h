@@ -65,7 +65,7 @@ extern "C" {
 typedef enum {
     LCLA_OK = 0,
     LCLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad dtype, overlap, bad eps */
-    LCLA_ERR_UNSUPPORTED = 2,   /* valid request this build does not serve (d not 32 or 64, N > 2^30) */
+    LCLA_ERR_UNSUPPORTED = 2,   /* valid request the library does not serve (d not 32 or 64, N > 2^30) */
     LCLA_ERR_MISALIGNED = 3,    /* an array pointer is not 16-byte aligned */
     LCLA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the query says */
     LCLA_ERR_CUDA = 5,          /* a CUDA launch failed; see cudaGetLastError */
