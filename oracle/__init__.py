@@ -75,7 +75,7 @@ class Oracle:
         """Outputs [B, nrows, H, d] from the pair-by-pair definition."""
         q, k, v, c, s, code, (B, N, H, d) = _prep(q, k, v, rope_cos, rope_sin)
         r, nrows = _rows(rows, N)
-        out = np.empty((B, nrows, H, d), np.float64)
+        out = np.full((B, nrows, H, d), np.nan)     # a slot left unwritten stays NaN
         rc = self.lib.lcla_oracle_masked(_ptr(q), _ptr(k), _ptr(v), code, _ptr(c), _ptr(s),
                                          B, H, N, d, int(block_len), float(eps),
                                          _ptr(r), nrows, _ptr(out))
@@ -96,7 +96,7 @@ class Oracle:
         if int(block_len) <= 0:
             raise ValueError("block_len must be positive")
         nb = -(-N // int(block_len))
-        out = np.empty((B, nrows, H, d), np.float64) if want_out else None
+        out = np.full((B, nrows, H, d), np.nan) if want_out else None   # unwritten slots stay NaN
         st = np.empty((B, H, d + 1, d), np.float64)
         pre = np.empty((B, H, nb, d + 1, d), np.float64) if want_prefix else None
         sin_ = None

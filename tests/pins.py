@@ -410,7 +410,43 @@ def pin_explicit_blocks(orc):
     rows_close(a, b, 1e-12, "uniform offsets vs recurrence")
 
 
+def pin_row_subset(orc):
+    """Both routes evaluate a requested subset of rows (an unsorted list that
+    spans several blocks, holds the first and last token and one repeat) into
+    the slots in the order the rows were asked for.  Each row equals the same
+    row of the full evaluation bit for bit, and the pair-by-pair definition
+    written in numpy (explicit block ids, complex rotary) to 1e-12."""
+    cases = [dict(seed=51, N=37, L=5, d=8, dtype="f32"),
+             dict(seed=52, N=37, L=1, d=8, dtype="bf16", dist="laplace_negrows"),
+             dict(seed=53, N=37, L=37, d=8, dtype="f32"),
+             dict(seed=54, N=30, L=5, d=32, dtype="bf16"),
+             dict(seed=55, N=26, L=1, d=32, dtype="f32"),
+             dict(seed=56, N=22, L=22, d=64, dtype="bf16", dist="laplace_negrows"),
+             dict(seed=57, N=22, L=5, d=64, dtype="f32")]
+    for c in cases:
+        N, L = c["N"], c["L"]
+        inp = small(c["seed"], B=2, H=2, N=N, L=L, d=c["d"], dtype=c["dtype"],
+                    dist=c.get("dist", "normal"))
+        rng = np.random.default_rng(c["seed"])
+        mid = rng.permutation(np.arange(1, N - 1))[: N // 3]
+        rows = np.concatenate([[N - 1], mid[:2], [0], mid[2:], mid[:1]]).astype(np.int64)
+        assert rows[0] > rows[1] or rows[1] > rows[2], "rows must be unsorted"
+        args = (inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, L, 1e-8)
+        full_m = orc.masked(*args)
+        full_r, st_full, _ = orc.recurrence(*args)
+        sub_m = orc.masked(*args, rows=rows)
+        sub_r, st_sub, _ = orc.recurrence(*args, rows=rows)
+        assert np.array_equal(sub_m, full_m[:, rows]), f"masked rows= vs full rows {c}"
+        assert np.array_equal(sub_r, full_r[:, rows]), f"recurrence rows= vs full rows {c}"
+        assert np.array_equal(st_sub, st_full), f"recurrence rows= changed the state {c}"
+        offs = list(range(0, N, L)) + [N]
+        ref = masked_blocks_numpy(inp.as_f32("q"), inp.as_f32("k"), inp.as_f32("v"),
+                                  inp.rope_cos, inp.rope_sin, offs, 1e-8)[:, rows]
+        rows_close(sub_m, ref, 1e-12, f"masked rows= vs definition {c}")
+        rows_close(sub_r, ref, 1e-12, f"recurrence rows= vs definition {c}")
+
+
 ALL_PINS = [pin_masked_equals_recurrence, pin_single_block_equals_printed_formula,
             pin_block_len_one_is_token_causal, pin_step_chain_equals_forward,
             pin_exact_rational, pin_closed_forms, pin_symmetries, pin_bf16_widening,
-            pin_explicit_blocks]
+            pin_explicit_blocks, pin_row_subset]

@@ -48,6 +48,12 @@ MUTANTS = {
     "recurrence_exclusive_prefix": [("order[next].tok < j1;", "order[next].tok < j0;")],
     "recurrence_unrotated_query": [("    rotate(qf, cs, sn, i, d, qr);\n    double den = dot(P",
                                     "    rotate(qf, cs, sn, 0, d, qr);\n    double den = dot(P")],
+    # row subsets (rows=): each requested row goes to its own slot, in token order
+    "recurrence_rows_slot_is_visit_order": [
+        ("out + (((size_t)b * nrows + (size_t)order[next].slot) * H + h)",
+         "out + (((size_t)b * nrows + (size_t)next) * H + h)")],
+    "recurrence_rows_not_sorted": [("    if (rows) qsort(order,", "    if (0) qsort(order,")],
+    "masked_rows_ignored": [("long i = rows ? (long)rows[r] : (long)r;", "long i = (long)r;")],
     # step route
     "step_ignores_carried_state": [("S[x] += st[x];", "S[x] += 0.0 * st[x];")],
     "step_save_inverted": [("if (save) memcpy(st, S,", "if (!save) memcpy(st, S,")],
