@@ -2,36 +2,25 @@
 //
 // For callers that cannot allocate device memory (see lcla_forward_noalloc in
 // include/lcla.h).  The scratch is a file-scope device array; host code only
-// knows a host-side stand-in for it under that name, so its device address is
-// looked up once per device, with that device current, and that address is
-// what the kernels receive.
+// knows a host-side stand-in for it under that name, so every call looks up
+// its device address in the current context, and that address is what the
+// kernels receive.  The lookup is not cached: a cached address would go stale
+// after a device reset, or belong to another context's copy of the module when
+// the caller switches contexts.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "lcla.h"
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-
 static __device__ __align__(256) unsigned char g_scratch[LCLA_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_lock;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_scratch on the current device (looked up on first use).
-int scratch_on_current_device(void **ptr)
+// Device address of g_scratch in the context current on this thread.
+int scratch_in_current_context(void **ptr)
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LCLA_ERR_CUDA;
-    std::lock_guard<std::mutex> guard(g_lock);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return LCLA_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *ptr = g_scratch_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return LCLA_ERR_CUDA;
+    *ptr = p;
     return LCLA_OK;
 }
 
@@ -45,7 +34,7 @@ extern "C" int lcla_forward_noalloc(const void *q, const void *k, const void *v,
     if (need > LCLA_NOALLOC_SCRATCH_BYTES) return LCLA_ERR_TOO_LARGE;
     void *scratch = nullptr;
     if (need > 0) {
-        const int rc = scratch_on_current_device(&scratch);
+        const int rc = scratch_in_current_context(&scratch);
         if (rc != LCLA_OK) return rc;
     }
     return lcla_forward(q, k, v, rope_cos, rope_sin, B, H, N, d, block_len, eps, out, state_out, dtype,

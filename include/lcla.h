@@ -28,7 +28,8 @@
  * Conventions for every entry point:
  *   - All array pointers are DEVICE pointers owned by the caller; the library
  *     allocates nothing, keeps no per-call state between calls, and never
- *     frees caller memory.
+ *     frees caller memory.  The one exception is lcla_forward_noalloc, which
+ *     uses a scratch array compiled into the library (see its comment).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and the call returns without synchronising.  Results are valid
  *     once the stream has reached the work.
@@ -37,9 +38,11 @@
  *   - Every array pointer must be 16-byte aligned (LCLA_ERR_MISALIGNED).
  *   - d must be 32 or 64 (the pages set linear_head_dim to 32 or 64: "Implementing
  *     Block Causal Linear Attention ...", section "Integration into Sana's
- *     Video Backbone"); other head dims: LCLA_ERR_UNSUPPORTED.  d = 32 runs
- *     on tensor cores for bf16 with block_len >= 64; d = 64 runs on CUDA cores
- *     with one thread block per (segment, head, batch entry), so H <= 65535.
+ *     Video Backbone"); other head dims: LCLA_ERR_UNSUPPORTED.  bf16 runs on
+ *     tensor cores at both head dims (at d = 32 for block_len >= 64; shorter
+ *     blocks take a CUDA-core kernel whose tiles hold whole blocks).  float32
+ *     runs on CUDA cores; at d = 64 with one thread block per (segment, head,
+ *     batch entry), so H <= 65535 at d = 64.
  *   - `out` must not overlap q, k, v, the tables, the state or the workspace
  *     (LCLA_ERR_INVALID_ARG).
  *   - eps must be finite and >= 0.
@@ -280,8 +283,9 @@ LCLA_API int lcla_step(const void *q_blk, const void *k_blk, const void *v_blk,
  * info[1] = segments (partial states written by the first pass);
  * info[2] = prefix states (blocks, or segments when info[0] = 1);
  * info[3] = tokens per tile; info[4] = 1 when the tensor-core kernels run
- * (d = 32, bf16, block_len >= 64), else 0.  `info` holds 5 ints.  Returns an
- * lcla_status; touches no device.
+ * (bf16 in block mode: d = 32 with block_len >= 64, or d = 64 at any block
+ * length), else 0.  `info` holds 5 ints.  Returns an lcla_status; touches no
+ * device.
  */
 LCLA_API int lcla_forward_plan_info(int B, int H, int N, int d, int block_len, int dtype,
                                     int *info);
@@ -314,9 +318,15 @@ LCLA_API int lcla_forward_plan_segments(int B, int H, int N, int d, int block_le
  *     needs more scratch than the array holds, i.e. when
  *     lcla_forward_workspace_bytes(B, H, N, d, block_len, dtype) >
  *     LCLA_NOALLOC_SCRATCH_BYTES.  Other errors are those of lcla_forward.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.  `stream` must belong to the current device.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *     in the context current on the calling thread, so it follows the device
+ *     that is current, a context the caller created and made current, and a
+ *     device reset.  The first call in a context loads the library's device
+ *     code into it; make that first call before any stream capture.
+ *     `stream` must belong to the current context.
+ *   - The workspace's device status word (LCLA_DEVICE_STATUS_*) lives in the
+ *     library's array, which the caller cannot read: on this entry point a
+ *     bounded wait that gives up shows only as NaN outputs and state.
  *   - All calls on a device share the one array, and it keeps the previous
  *     call's contents (each call re-initialises what it reads).  Calls whose
  *     GPU work overlaps -- on different streams, or from different host
