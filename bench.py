@@ -2,11 +2,14 @@
 
 One step = one lcla_forward over the whole workload (pass A partial states,
 scan, pass C outputs) with the inputs resident in HBM.  Default workload: the
-480p-like forward (B=1, H=70, d=32, 21 frames x 30x52 tokens = 32760 tokens,
-blocks of 3 frames = 4680 tokens, bf16, 3D rotary tables).  Prints one JSON
-line with the whole-job throughput in attended token-heads per second, the
-end-to-end number through the same call with host buffers, the roofline of
-the dominant kernel, and the fp64 CPU oracle timed on the host as a baseline.
+minute-scale forward, the largest single-GPU workload (B=1, H=70, d=32, 241
+frames x 44x80 tokens = 848320 tokens, blocks of 3 frames = 10560 tokens,
+bf16, 3D rotary tables); the 480p-like forward (21 frames x 30x52 tokens,
+blocks of 4680) is timed beside it and reported under "also".  Prints one
+JSON line with the whole-job throughput in attended token-heads per second,
+the end-to-end number through the same call with host buffers, the roofline
+of the dominant kernel, and the fp64 CPU oracle timed on the host as a
+baseline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-e2e] [--cpu-seconds S] [--parallel replicas|seq]
@@ -48,7 +51,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="fwd480p_bf16", choices=sorted(NAMED))
+    ap.add_argument("--workload", default="minute_bf16", choices=sorted(NAMED))
+    ap.add_argument("--also", default="fwd480p_bf16",
+                    help="comma-separated workloads timed after the main one (device time and per-pass "
+                         "roofline only), reported under 'also'; 'none' for none")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -180,24 +186,45 @@ class ClockSampler:
                 "power_w_max": max(s[1] for s in self.samples), "source": "NVML"}
 
 
+def head_subset(inp, nh):
+    """q, k, v restricted to the first ``nh`` heads (contiguous copies)."""
+    sub = lambda a: np.ascontiguousarray(a[:, :, :nh])
+    return sub(inp.q), sub(inp.k), sub(inp.v)
+
+
 def cpu_baseline(inp, seconds):
     """The fp64 oracle (block-recurrence route, every output) on the host cores,
-    on a bounded sample: whole passes over the workload until ``seconds``."""
+    on a bounded sample: passes over the workload, or over a subset of its
+    heads when one whole pass would not fit in ``seconds``, until ``seconds``."""
     import oracle
     orc = oracle.default()
     spec = inp.spec
     threads = orc.max_threads()
+    # one pass over as many heads as there are threads (the oracle runs one (b, h) per thread)
+    nh = min(spec.H, threads)
+    q, k, v = head_subset(inp, nh)
+    t0 = time.perf_counter()
+    orc.recurrence(q, k, v, inp.rope_cos, inp.rope_sin, spec.block_len, spec.eps)
+    per_group = time.perf_counter() - t0
+    groups = max(1, int(seconds / 2 / max(per_group, 1e-6)))
+    nh = min(spec.H, nh * groups)
+    if nh < spec.H:
+        q, k, v = head_subset(inp, nh)
+    else:
+        q, k, v = inp.q, inp.k, inp.v
     n = 0
     t0 = time.perf_counter()
     while True:
-        orc.recurrence(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, spec.block_len, spec.eps)
+        orc.recurrence(q, k, v, inp.rope_cos, inp.rope_sin, spec.block_len, spec.eps)
         n += 1
         el = time.perf_counter() - t0
         if el >= seconds or n >= 50:
             break
-    return {"value": n * spec.token_heads / el, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n} full pass(es) of the recurrence route over the whole {spec.name} "
-                      f"workload ({spec.token_heads} token-heads each, every output and the final "
+    units = spec.B * spec.N * nh
+    what = "the whole" if nh == spec.H else f"the first {nh} of {spec.H} heads of the"
+    return {"value": n * units / el, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} pass(es) of the recurrence route over {what} {spec.name} "
+                      f"workload ({units} token-heads each, every output and the final "
                       f"state), fp64, {threads} OpenMP threads, {el:.1f} s"}
 
 
@@ -255,15 +282,15 @@ def run_reference(args):
     spec = NAMED[args.workload]
     inp = make_inputs(spec)
     orc = oracle.default()
-    # calibrate: time of one head
+    # calibrate: one pass over as many heads as there are threads (one (b, h) per thread)
+    nh = min(spec.H, orc.max_threads())
+    q, k, v = head_subset(inp, nh)
     t0 = time.perf_counter()
-    sub = lambda a, nh: np.ascontiguousarray(a[:, :, :nh])
-    orc.recurrence(sub(inp.q, 1), sub(inp.k, 1), sub(inp.v, 1), inp.rope_cos, inp.rope_sin,
-                   spec.block_len, spec.eps)
-    per_head = max(time.perf_counter() - t0, 1e-4)
+    orc.recurrence(q, k, v, inp.rope_cos, inp.rope_sin, spec.block_len, spec.eps)
+    per_group = max(time.perf_counter() - t0, 1e-4)
     budget = 120.0 / max(1, args.steps + args.warmup)
-    nh = int(max(1, min(spec.H, budget / per_head)))
-    q, k, v = sub(inp.q, nh), sub(inp.k, nh), sub(inp.v, nh)
+    nh = int(min(spec.H, nh * max(1, int(budget / per_group))))
+    q, k, v = head_subset(inp, nh)
     for _ in range(args.warmup):
         orc.recurrence(q, k, v, inp.rope_cos, inp.rope_sin, spec.block_len, spec.eps)
     t0 = time.perf_counter()
@@ -585,54 +612,38 @@ def run_seq(args):
     ranks.close()
 
 
-def main():
-    args = parse()
-    if args.impl == "reference":
-        return run_reference(args)
-    if args.op == "tconv":
-        return run_tconv(args)
-    if args.op == "step":
-        return run_step(args)
-    if args.parallel == "seq":
-        return run_seq(args)
-
+def to_dev(a, device):
+    """numpy array (bf16 as uint16 bits, or float32) -> torch tensor on ``device``."""
     import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(a).to(device)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    ranks = Ranks(world, rank, "nccl", device)
 
-    def barrier():
-        ranks.barrier()
-        torch.cuda.synchronize(device)
-
-    max_over_ranks = ranks.max
-
-    import block_causal_relu_b200 as lcla
-
-    spec = rank_spec(NAMED[args.workload], rank)             # independent problem per rank
+def forward_buffers(lcla, spec, device):
+    """Device inputs, outputs and workspace of one forward of ``spec``."""
+    import torch
     inp = make_inputs(spec)
-
-    def to_dev(a):
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
-        return torch.from_numpy(a).to(device)
-
-    q, k, v, c, s = (to_dev(a) for a in (inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin))
+    ins = tuple(to_dev(a, device) for a in (inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin))
     code = lcla.BF16 if spec.dtype == "bf16" else lcla.F32
-    out = torch.empty_like(q)
+    out = torch.empty_like(ins[0])
     st = torch.empty((spec.B, spec.H, spec.d + 1, spec.d), dtype=torch.float32, device=device)
-    ws = torch.empty(max(1, lcla.forward_workspace_bytes(spec.B, spec.H, spec.N, spec.d,
-                                                         spec.block_len, code)),
+    ws = torch.empty(max(1, lcla.forward_workspace_bytes(spec.B, spec.H, spec.N, spec.d, spec.block_len, code)),
                      dtype=torch.uint8, device=device)
-    stream = torch.cuda.current_stream(device)
+    return inp, ins, out, st, ws
 
-    K, W = args.steps, args.warmup
+
+def time_forward(lcla, spec, inputs, out, st, ws, stream, device, K, W, ranks, clocks=False):
+    """W warm-up forwards, then two timed regions of K forwards each on
+    ``stream``: plain calls back to back (the step time; NVML clocks sampled
+    when ``clocks``), then lcla_forward_timed with events between the passes
+    (the per-pass times of the roofline; events between the passes would
+    defeat the programmatic-launch overlap, so they stay out of the first
+    region).  Device times are the max over ranks."""
+    import torch
+    q, k, v, c, s = inputs
+    code = lcla.BF16 if spec.dtype == "bf16" else lcla.F32
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     for row in evs:                       # materialise the event handles
         for e in row:
@@ -642,30 +653,30 @@ def main():
         lcla.forward(q, k, v, c, s, spec.block_len, spec.eps, out=out, state_out=st,
                      workspace=ws, stream=stream, events=events)
 
+    def barrier():
+        ranks.barrier()
+        torch.cuda.synchronize(device)
+
     for _ in range(W):
         step()
     barrier()
-    # timed region 1: the headline number, plain calls back to back
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(device) as clk:
-        e0.record(stream)
-        for i in range(K):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
+    clk = ClockSampler(device) if clocks else None
+    if clk:
+        clk.__enter__()
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    if clk:
+        clk.__exit__(None, None, None)
     barrier()
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
-    ms = ms_total / K
-    units = spec.token_heads
-    value = whole_job_rate(world, units, K, ms_total)
-    # timed region 2: the same steps with events recorded between the passes
-    # (lcla_forward_timed) for the per-kernel durations of the roofline
+    ms_total = ranks.max(e0.elapsed_time(e1))
     for i in range(K):
         step(evs[i])
     torch.cuda.synchronize(device)
     barrier()
-
-    # per-pass device times over the timed region
     pa = [r[0].elapsed_time(r[1]) for r in evs]
     sc = [r[1].elapsed_time(r[2]) for r in evs]
     pc = [r[2].elapsed_time(r[3]) for r in evs]
@@ -699,7 +710,54 @@ def main():
                 "peak_source": f"{peak_kind} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
                 "traffic": ncu_traffic(dname, spec.name), "algorithmic_bytes": dbytes}
     path_bytes = 4 * tok_bytes + 2 * tab_bytes + sl      # q,k,v in + out + tables + state
-    pass_ms = {kk: vv[0] for kk, vv in passes.items()}
+    ms = ms_total / K
+    launches = 2 + (1 if scan_name == "scan_states_grouped" else 2)
+    return {"ms_per_step": ms, "ms_total": ms_total, "clocks": clk.summary() if clk else None,
+            "launches_per_step": launches,
+            "pass_ms": {kk: vv[0] for kk, vv in passes.items()},
+            "pass_frac_of_peak": {kk: vv[1] / (vv[0] / 1e3) / 1e9 / peak for kk, vv in passes.items()},
+            "roofline": roofline, "path_bytes": path_bytes, "tok_bytes": tok_bytes,
+            "tab_bytes": tab_bytes, "state_bytes": sl,
+            "hbm_frac_of_peak": path_bytes / (ms / 1e3) / 1e9 / peak}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.op == "tconv":
+        return run_tconv(args)
+    if args.op == "step":
+        return run_step(args)
+    if args.parallel == "seq":
+        return run_seq(args)
+
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    ranks = Ranks(world, rank, "nccl", device)
+
+    def barrier():
+        ranks.barrier()
+        torch.cuda.synchronize(device)
+
+    import block_causal_relu_b200 as lcla
+
+    stream = torch.cuda.current_stream(device)
+    K, W = args.steps, args.warmup
+    spec = rank_spec(NAMED[args.workload], rank)             # independent problem per rank
+    inp, (q, k, v, c, s), out, st, ws = forward_buffers(lcla, spec, device)
+    res = time_forward(lcla, spec, (q, k, v, c, s), out, st, ws, stream, device, K, W, ranks, clocks=True)
+    ms, ms_total = res["ms_per_step"], res["ms_total"]
+    units = spec.token_heads
+    value = whole_job_rate(world, units, K, ms_total)
+    tok_bytes, tab_bytes, sl = res["tok_bytes"], res["tab_bytes"], res["state_bytes"]
 
     # end to end through the same call with host buffers
     e2e = None
@@ -721,8 +779,8 @@ def main():
 
         e2e_pipelined(device, 2, [hq, hk, hv, hc, hs], ins, [hout, hst], outs, e2e_launch)   # warm the streams
         barrier()
-        ems = max_over_ranks(KE * e2e_pipelined(device, KE, [hq, hk, hv, hc, hs], ins, [hout, hst], outs,
-                                                e2e_launch))
+        ems = ranks.max(KE * e2e_pipelined(device, KE, [hq, hk, hv, hc, hs], ins, [hout, hst], outs,
+                                           e2e_launch))
         barrier()
         h2d = 3 * tok_bytes + tab_bytes
         d2h = tok_bytes + sl
@@ -730,20 +788,37 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ems / KE, "steps": KE,
                "overlap": "step i's upload, step i-1's forward and step i-2's download run on three streams"}
+        del hq, hk, hv, hc, hs, hout, hst, ins, outs
 
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_baseline(inp, args.cpu_seconds)
+    del inp, q, k, v, c, s, out, st, ws
+    torch.cuda.empty_cache()
+
+    # the other workloads of --also: device time and per-pass roofline each
+    also = {}
+    for name in [n for n in args.also.split(",") if n and n != "none" and n != args.workload]:
+        aspec = rank_spec(NAMED[name], rank)
+        _, ains, aout, ast, aws = forward_buffers(lcla, aspec, device)
+        r = time_forward(lcla, aspec, ains, aout, ast, aws, stream, device, K, W, ranks)
+        also[name] = {"workload": workload_config(aspec, world)["workload"], "ms_per_step": r["ms_per_step"],
+                      "value": whole_job_rate(world, aspec.token_heads, K, r["ms_total"]),
+                      "hbm_frac_of_peak": r["hbm_frac_of_peak"], "pass_ms": r["pass_ms"],
+                      "pass_frac_of_peak": r["pass_frac_of_peak"], "roofline": r["roofline"]}
+        del ains, aout, ast, aws
+        torch.cuda.empty_cache()
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
                 "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic (seeded)",
                 "config": workload_config(spec, world),
-                "achieved_hbm_gbs": world * path_bytes / (ms / 1e3) / 1e9 / world,
-                "hbm_frac_of_peak": path_bytes / (ms / 1e3) / 1e9 / peak,
-                "pass_ms": pass_ms, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": 3 * K, "clocks": clk.summary()}
+                "achieved_hbm_gbs": res["path_bytes"] / (ms / 1e3) / 1e9,
+                "hbm_frac_of_peak": res["hbm_frac_of_peak"],
+                "pass_ms": res["pass_ms"], "pass_frac_of_peak": res["pass_frac_of_peak"],
+                "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": res["launches_per_step"] * K, "clocks": res["clocks"], "also": also}
         print(json.dumps(line), flush=True)
     ranks.close()
 

@@ -104,3 +104,20 @@ def test_reference_arm_rank0_prints_the_contract_line(monkeypatch, capsys):
     assert d["value"] > 0 and d["higher_is_better"] is True
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_default_workload_is_minute_scale_and_cpu_baseline_takes_a_head_subset(monkeypatch):
+    """The headline is the largest single-GPU workload; the CPU baseline of a
+    workload too large for its time budget times a labelled subset of heads."""
+    bench = load_bench()
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    a = bench.parse()
+    assert a.workload == "minute_bf16" and "fwd480p_bf16" in a.also.split(",")
+    sys.path.insert(0, ROOT)
+    from dataclasses import replace
+    from workloads import NAMED, make_inputs
+    spec = replace(NAMED["tiny_f32"], H=40, N=4096, block_len=512)
+    inp = make_inputs(spec, threads=1)
+    cb = bench.cpu_baseline(inp, 1e-9)          # a budget too small for any whole pass
+    assert cb["kind"] == "oracle" and cb["value"] > 0
+    assert "heads of the" in cb["sample"] and f"of {spec.H} heads" in cb["sample"]

@@ -24,6 +24,7 @@ Distributions (one row = the d values of one (b, n, h)):
 from __future__ import annotations
 
 import os
+import threading
 from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field, replace
 from typing import Optional, Tuple
@@ -161,23 +162,63 @@ def _seed_seq(seed: int, tensor_id: int, chunk: int) -> np.random.SeedSequence:
     return np.random.SeedSequence(entropy=seed, spawn_key=(tensor_id, chunk))
 
 
+_scratch = threading.local()
+
+
+def _buffers(n: int):
+    """This thread's reusable chunk buffers (float64, uint64, float32, uint32).
+    Reusing them keeps the threads off the allocator: fresh chunk-sized
+    arrays are mapped and unmapped per call, and the page faults and
+    unmappings serialise the threads."""
+    bufs = getattr(_scratch, "bufs", None)
+    if bufs is None or bufs[0].size < n:
+        bufs = (np.empty(n, np.float64), np.empty(n, np.uint64), np.empty(n, np.float32),
+                np.empty(n, np.uint32))
+        _scratch.bufs = bufs
+    return tuple(b[:n] for b in bufs)
+
+
+def _round_bf16_into(x: np.ndarray, t64: np.ndarray, f32: np.ndarray, u32: np.ndarray,
+                     out: np.ndarray):
+    """``f64_to_bf16_bits(x)`` written into ``out`` (uint16) through the
+    caller's buffers; ``x`` is overwritten.  The same checks and bits."""
+    ax = np.abs(x, out=t64.view(np.float64))
+    if not np.isfinite(ax.max()):
+        raise ValueError("non-finite sample")
+    if np.count_nonzero(ax < 2.0 ** -126) != np.count_nonzero(ax == 0.0):
+        raise ValueError("sample in the bf16 subnormal range")
+    b = x.view(np.uint64)
+    np.right_shift(b, np.uint64(45), out=t64)
+    np.bitwise_and(t64, np.uint64(1), out=t64)
+    np.add(t64, np.uint64((1 << 44) - 1), out=t64)
+    np.add(b, t64, out=b)
+    np.bitwise_and(b, ~np.uint64((1 << 45) - 1), out=b)
+    f32[:] = x
+    if not np.isfinite(np.abs(f32).max()):
+        raise ValueError("sample overflows bf16")
+    np.right_shift(f32.view(np.uint32), np.uint32(16), out=u32)
+    out[:] = u32
+
+
 def _fill_chunk(out: np.ndarray, lo: int, hi: int, d: int, seed: int,
                 tensor_id: int, chunk: int, dist: str, sigma: float, dtype: str):
     rng = np.random.Generator(np.random.PCG64(_seed_seq(seed, tensor_id, chunk)))
     n = hi - lo
+    x, t64, f32, u32 = _buffers(n)
     if dist == "normal":
-        x = rng.standard_normal(n) * sigma
+        rng.standard_normal(out=x)
+        x *= sigma
     elif dist == "laplace_negrows":
-        x = rng.laplace(0.0, 1.0, n)
+        x[:] = rng.laplace(0.0, 1.0, n)
         rows = x.reshape(-1, d)
         neg = rng.random(rows.shape[0]) < _NEG_ROW_P
         rows[neg] = -np.abs(rows[neg])
     else:
         raise ValueError(dist)
     if dtype == "bf16":
-        out[lo:hi] = f64_to_bf16_bits(x)
+        _round_bf16_into(x, t64, f32, u32, out[lo:hi])
     else:
-        out[lo:hi] = x.astype(np.float32)
+        out[lo:hi] = x
 
 
 def _draw_tensor(shape, d: int, seed: int, tensor_id: int, dist: str,
