@@ -791,7 +791,7 @@ def main():
         del hq, hk, hv, hc, hs, hout, hst, ins, outs
 
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
         cpu = cpu_baseline(inp, args.cpu_seconds)
     del inp, q, k, v, c, s, out, st, ws
     torch.cuda.empty_cache()

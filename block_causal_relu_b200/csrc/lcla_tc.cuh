@@ -221,6 +221,7 @@ __device__ __forceinline__ void tma_store3(const CUtensorMap *map, uint32_t src,
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols)
@@ -366,6 +367,70 @@ __device__ __forceinline__ void rope_split4_scaled(const uint32_t *fw, const flo
         lo[p] = pack_bf2(y0 - hf.x, y1 - hf.y);
     }
 }
+// Arrive on an mbarrier only once `dep` is known.  A warp that releases a
+// shared buffer for a TMA refill passes a value computed from its loads out of
+// that buffer (lane 0's, which returns with the whole warp's instruction) and
+// `zero`, a register holding 0 that the compiler cannot see through: the
+// barrier address then depends on the loaded data, so the arrive cannot issue
+// before the loads have returned (see release_after_use).
+__device__ __forceinline__ void bar_arrive_dep(uint32_t bar, uint32_t dep, uint32_t zero)
+{
+    bar_arrive(bar + (dep & zero));
+}
+
+// Packed bf16 -> fp32: the element in the low half, and the one in the high half.
+__device__ __forceinline__ float bf_low(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_high(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Rotate, scale and split one quarter (4 pairs) of a head on the paired fp32
+// pipes (fma/mul .f32x2, two lanes per instruction).  fw[j]: packed bf16
+// features of pair j (element 2j low, 2j+1 high); (c, s) of pairs 0-1 and
+// 2-3; g: the factor applied after the rotation.  hi[j], lo[j]: packed bf16
+// hi + lo of the rotated pair j, hi = RNE(y), lo = RNE(y - hi).
+__device__ __forceinline__ void rope_split4_x2(const uint32_t *fw, float2 c01, float2 c23, float2 s01, float2 s23,
+                                               float2 ns01, float2 ns23, float g, uint32_t *hi, uint32_t *lo)
+{
+    const float2 a01 = make_float2(bf_low(fw[0]), bf_low(fw[1])), a23 = make_float2(bf_low(fw[2]), bf_low(fw[3]));
+    const float2 b01 = make_float2(bf_high(fw[0]), bf_high(fw[1])), b23 = make_float2(bf_high(fw[2]), bf_high(fw[3]));
+    const float2 g2 = make_float2(g, g), m1 = make_float2(-1.f, -1.f);
+    // y0 = a c - b s, y1 = a s + b c, then times g
+    const float2 y0_01 = __fmul2_rn(__ffma2_rn(a01, c01, __fmul2_rn(b01, ns01)), g2);
+    const float2 y0_23 = __fmul2_rn(__ffma2_rn(a23, c23, __fmul2_rn(b23, ns23)), g2);
+    const float2 y1_01 = __fmul2_rn(__ffma2_rn(b01, c01, __fmul2_rn(a01, s01)), g2);
+    const float2 y1_23 = __fmul2_rn(__ffma2_rn(b23, c23, __fmul2_rn(a23, s23)), g2);
+    const uint32_t h0 = pack_bf2(y0_01.x, y1_01.x), h1 = pack_bf2(y0_01.y, y1_01.y);
+    const uint32_t h2 = pack_bf2(y0_23.x, y1_23.x), h3 = pack_bf2(y0_23.y, y1_23.y);
+    // y - hi, exact in fp32
+    const float2 l0_01 = __ffma2_rn(make_float2(bf_low(h0), bf_low(h1)), m1, y0_01);
+    const float2 l1_01 = __ffma2_rn(make_float2(bf_high(h0), bf_high(h1)), m1, y1_01);
+    const float2 l0_23 = __ffma2_rn(make_float2(bf_low(h2), bf_low(h3)), m1, y0_23);
+    const float2 l1_23 = __ffma2_rn(make_float2(bf_high(h2), bf_high(h3)), m1, y1_23);
+    hi[0] = h0; hi[1] = h1; hi[2] = h2; hi[3] = h3;
+    lo[0] = pack_bf2(l0_01.x, l1_01.x);
+    lo[1] = pack_bf2(l0_01.y, l1_01.y);
+    lo[2] = pack_bf2(l0_23.x, l1_23.x);
+    lo[3] = pack_bf2(l0_23.y, l1_23.y);
+}
+
+// 1 / x from the hardware approximation (relative error of a few ulp; the
+// products it scales carry bf16 operands, far coarser).
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// z . phi for one quarter: za = z of the even elements (pairs 0-1, 2-3), zb = of the odd ones.
+__device__ __forceinline__ float zdot4_x2(const uint32_t *fw, float2 za01, float2 za23, float2 zb01, float2 zb23)
+{
+    float2 d = __fmul2_rn(make_float2(bf_low(fw[0]), bf_low(fw[1])), za01);
+    d = __ffma2_rn(make_float2(bf_low(fw[2]), bf_low(fw[3])), za23, d);
+    d = __ffma2_rn(make_float2(bf_high(fw[0]), bf_high(fw[1])), zb01, d);
+    d = __ffma2_rn(make_float2(bf_high(fw[2]), bf_high(fw[3])), zb23, d);
+    return d.x + d.y;
+}
+
 // Quarter f of operand row r (128 B, 128-byte swizzle): hi -> chunk f, lo -> chunk 4+f.
 __device__ __forceinline__ void store_quarter_hi_lo(unsigned char *tile, int r, int f, const uint32_t *hi,
                                                     const uint32_t *lo)
@@ -444,7 +509,6 @@ __device__ __forceinline__ Unit unit_at(const LclaPlan &p, int u)
     return x;
 }
 
-constexpr int NT = 3;             // rotary-table ring slots
 constexpr int CTRL_BYTES = 512;   // control block: mbarriers (8 B each), tensor-memory slot, abort flag
 constexpr int SMEM_MAX = 232448;  // dynamic shared memory a CTA may opt in to
 constexpr int NPRO = 16;          // prologue warps (both passes)
@@ -462,19 +526,21 @@ struct Width {
     static constexpr int SZ = (DW + 1) * DW;          // floats per (S, z) state
 };
 
-// Producer: per tile, TMA loads of the quad's input boxes into the stage ring
+// Producers.  The tile's input boxes and its rotary rows come from two
+// threads of two different warps, each running ahead through its own ring:
+// a producer that waited for a slot of one ring before filling the other
+// would hold the deeper ring to the depth of the shallower one.
+//
+// Input boxes: per tile, TMA loads of the quad's boxes into the stage ring
 // (NBOX boxes of [64 token][4 / NBOX heads] per tensor map, heads past H read
-// as zeros)
-// and of the tile's rotary rows into the table ring.  On abort, waits
-// (bounded) for the loads already issued before returning.
-template <int DW, int S, int STAGE, int NMAP, int NBOX>
-__device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t sb, uint32_t tab0,
-                                        uint32_t FULL, uint32_t EMPTY, uint32_t CFULL, uint32_t CEMPTY,
-                                        const CUtensorMap *const (&maps)[NMAP], const int (&offs)[NMAP],
-                                        const CUtensorMap *mc, const CUtensorMap *ms, volatile int *abort_flag)
+// as zeros).  On abort, waits (bounded) for the loads already issued.
+template <int S, int STAGE, int NMAP, int NBOX>
+__device__ __forceinline__ void produce_boxes(const LclaPlan &p, int nunits, uint32_t sb, uint32_t FULL, uint32_t EMPTY,
+                                              const CUtensorMap *const (&maps)[NMAP], const int (&offs)[NMAP],
+                                              volatile int *abort_flag)
 {
-    Ring er = {0, 1u}, cr = {0, 1u};
-    int issued = 0, tissued = 0;
+    Ring er = {0, 1u};
+    int issued = 0;
     bool ok = true;
     const uint64_t stream_pol = policy_evict_first();
     for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
@@ -496,11 +562,32 @@ __device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t 
                                    x0 + j * (HQ * LCLA_D / NBOX), t, x.b, stream_pol);
             ring_next<S>(er);
             ++issued;
+        }
+    }
+    if (!ok)   // let the copies already issued land before the CTA releases its memory
+        for (int j = issued > S ? issued - S : 0; j < issued; ++j)
+            bar_wait_quiet(FULL + 8 * (j % S), (uint32_t)((j / S) & 1));
+}
+
+// Rotary rows: per tile, the tile's rows of the cos and sin tables into the
+// table ring (DW = 64: columns 0-15 and 16-31 of each, one box per half).
+template <int DW, int NTS>
+__device__ __forceinline__ void produce_tables(const LclaPlan &p, int nunits, uint32_t tab0, uint32_t CFULL,
+                                               uint32_t CEMPTY, const CUtensorMap *mc, const CUtensorMap *ms,
+                                               volatile int *abort_flag)
+{
+    constexpr int TB = Width<DW>::TAB_BYTES, VPH = Width<DW>::VPH;
+    Ring cr = {0, 1u};
+    int issued = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+        const Unit x = unit_at(p, u);
+        for (int i = 0; i < x.ntile; ++i) {
+            const int t = x.t0 + i * T;
             if (!bar_wait(CEMPTY + 8 * cr.idx, cr.phase, abort_flag)) {
                 ok = false;
                 break;
             }
-            constexpr int TB = Width<DW>::TAB_BYTES, VPH = Width<DW>::VPH;
             const uint32_t tb = tab0 + cr.idx * TB, cb = CFULL + 8 * cr.idx;
             bar_expect_tx(cb, (uint32_t)TB);
 #pragma unroll
@@ -508,16 +595,13 @@ __device__ __forceinline__ void produce(const LclaPlan &p, int nunits, uint32_t 
                 tma_load2(tb + hh * 4096, mc, cb, 16 * hh, t);
                 tma_load2(tb + TB / 2 + hh * 4096, ms, cb, 16 * hh, t);
             }
-            ring_next<NT>(cr);
-            ++tissued;
+            ring_next<NTS>(cr);
+            ++issued;
         }
     }
-    if (!ok) {   // let the copies already issued land before the CTA releases its memory
-        for (int j = issued > S ? issued - S : 0; j < issued; ++j)
-            bar_wait_quiet(FULL + 8 * (j % S), (uint32_t)((j / S) & 1));
-        for (int j = tissued > NT ? tissued - NT : 0; j < tissued; ++j)
-            bar_wait_quiet(CFULL + 8 * (j % NT), (uint32_t)((j / NT) & 1));
-    }
+    if (!ok)
+        for (int j = issued > NTS ? issued - NTS : 0; j < issued; ++j)
+            bar_wait_quiet(CFULL + 8 * (j % NTS), (uint32_t)((j / NTS) & 1));
 }
 
 // ---------------------------------------------------------------------------
@@ -530,6 +614,7 @@ struct LayA {
     // stage: [k~ operand, 4 atoms of [64 tok][hi 32 | lo 32] (raw k lands in atoms 0-1) | v, 2 boxes]
     static constexpr int K_OFF = 0, V_OFF = 32768, STAGE = 49152;
     static constexpr int TAB_BYTES = Width<DW>::TAB_BYTES;
+    static constexpr int NT = 3;                                    // rotary-table ring slots
     static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
     static constexpr int Z_OFF = C_OFF + NT * TAB_BYTES;            // key-sum parts [16 warps][2 g][4 f][2 heads][8]
     static constexpr int Z_BYTES = NPRO * 2 * 4 * 2 * 8 * 4;
@@ -541,14 +626,14 @@ struct LayA {
     // about 1.6e-5 of max |S| against fp32 sums; 4 tiles (16 K-steps) keep the
     // state well inside 1e-5, the rest is summed in registers
     static constexpr int CHUNK = 4;
-    static constexpr int NTHREADS = 704;                            // drain 0-3, producer 4, MMA 5, prologue 6-21
-    static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6;
+    static constexpr int NTHREADS = 736;                            // drain 0-3, producer 4, MMA 5, prologue 6-21, tables 22
+    static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6, W_TAB = 22;
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 1, 1);
     static constexpr int TMEM_COLS = NTM * 256;
     static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 3;
     static_assert(BYTES <= SMEM_MAX, "pass A shared memory");
     static_assert(8 * NBARS + 8 <= CTRL_BYTES, "pass A control block");
-    static_assert(NTHREADS / 32 - W_PRO0 == NPRO, "pass A prologue warps: barrier counts use NPRO");
+    static_assert(W_TAB - W_PRO0 == NPRO && NTHREADS / 32 == W_TAB + 1, "pass A prologue warps: barrier counts use NPRO");
 };
 
 // Pass A over head width DW.  At DW = 64 each quad holds two heads as four
@@ -561,7 +646,7 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
           float *__restrict__ part, int *__restrict__ status)
 {
     using L = LayA<DW>;
-    constexpr int S = L::STAGES, NTM = L::NTM, VPH = Width<DW>::VPH, TB = L::TAB_BYTES;
+    constexpr int S = L::STAGES, NTM = L::NTM, VPH = Width<DW>::VPH, TB = L::TAB_BYTES, NT = L::NT;
     const int HV = p.H * VPH;   // virtual heads
     extern __shared__ __align__(1024) unsigned char smraw[];
     const uint32_t raw = s32(smraw);
@@ -608,13 +693,15 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
     const uint32_t tmem = *tslot;
 
     if (w == L::W_PROD) {
-        // ---------------- producer: k, v and rotary rows of each tile ----------------
+        // ---------------- producer: k and v boxes of each tile ----------------
         if (lane == 0) {
             const CUtensorMap *const maps[2] = {&mk, &mv};
             const int offs[2] = {L::K_OFF, L::V_OFF};
-            produce<DW, S, L::STAGE, 2, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc,
-                                           &ms, abort_flag);
+            produce_boxes<S, L::STAGE, 2, 2>(p, nunits, sb, FULL, EMPTY, maps, offs, abort_flag);
         }
+    } else if (w == L::W_TAB) {
+        // ---------------- producer: rotary rows of each tile ----------------
+        if (lane == 0) produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag);
     } else if (w == L::W_MMA) {
         // ---------------- MMA issuer: one accumulator per chunk of CHUNK tiles ----------------
         if (lane == 0) {
@@ -834,30 +921,40 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
 // ---------------------------------------------------------------------------
 template <int DW>
 struct LayC {
-    // four stages at DW = 32; three at DW = 64, whose table slots are twice as large
-    static constexpr int STAGES = DW == 32 ? 4 : 3;
-    // stage: q~ operand, 4 blocks of [64 rows (tok)][q~hi 32 | q~lo 32] (raw q lands in blocks 0-1)
-    static constexpr int STAGE = 32768;
+    // raw q ring: one tile's two TMA boxes [64 tok][2 heads x 32] bf16 (16 KB) per slot, released as soon as
+    // the prologue has read it; operand ring: the tile's q~ operand, 4 atoms of [64 rows (tok)][q~hi 32 |
+    // q~lo 32] (32 KB), held until the tile's MMAs complete.  DW = 64 has table slots twice as large.
+    static constexpr int RAW = DW == 32 ? 5 : 4, RAW_BYTES = 16384;
+    static constexpr int OPS = 2, OP_BYTES = 32768;
+    static constexpr int RAW_OFF = 0, OP_OFF = RAW * RAW_BYTES;
     static constexpr int TAB_BYTES = Width<DW>::TAB_BYTES;
-    static constexpr int C_OFF = STAGES * STAGE;                    // rotary-table ring
+    static constexpr int NT = DW == 32 ? 4 : 3;                     // rotary-table ring slots
+    static constexpr int C_OFF = OP_OFF + OPS * OP_BYTES;           // rotary-table ring
     // prefix operands [128 rows (virtual head, c)][P hi | P lo]: DW = 32, one per unit, double-buffered;
     // DW = 64, the unit's two key halves (e < 32, e >= 32) in one buffer
     static constexpr int P_BYTES = 16384, NPB = DW == 32 ? 2 : 1;
     static constexpr int P_OFF = C_OFF + NT * TAB_BYTES;
-    static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 8 warps x 2 x [32 tok][32 c] bf16
+    static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 4 warps x 2 x [32 tok][32 c] bf16
     static constexpr int OBUF = 2048;
-    static constexpr int CTRL = O_OFF + 8 * 2 * OBUF;               // mbarriers, tensor-memory slot, abort flag
+    static constexpr int CTRL = O_OFF + 4 * 2 * OBUF;               // mbarriers, tensor-memory slot, abort flag
     static constexpr int BYTES = CTRL + CTRL_BYTES + 1024;          // + worst-case 1024-byte alignment pad
-    static constexpr int NTHREADS = 832;                            // epilogue 0-7, producer 8, MMA 9, prologue 10-25
-    static constexpr int W_PROD = 8, W_MMA = 9, W_PRO0 = 10, NEPI = 8;
+    // prologue: 8 warps in two groups of 4 that take alternate tiles, so that one group's waits, fences and
+    // load latencies overlap the other's arithmetic; a thread does four token rows of its group's tiles (the
+    // row sets that pair_offsets gives warps 4 gw .. 4 gw + 3)
+    static constexpr int NPC = 16, NGRP = 2, GW = NPC / NGRP, RPT = NPRO / GW;
+    static constexpr int NTHREADS = 736;                            // epilogue 0-3, producer 4, MMA 5, prologue 6-21,
+                                                                    // tables 22
+    static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6, W_TAB = 22, NEPI = 4;
     static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
     static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
     static constexpr int TMEM_COLS = NTM * 256;
-    static constexpr int NBARS = 3 * STAGES + 2 * NT + 2 * NTM + 2;
+    static constexpr int NBARS = 2 * RAW + 2 * OPS + 2 * NT + 2 * NTM + 4;
     static_assert(NPB * Width<DW>::VPH == 2, "two prefix operands of P_BYTES");
     static_assert(BYTES <= SMEM_MAX, "pass C shared memory");
-    static_assert(8 * NBARS + 8 <= CTRL_BYTES, "pass C control block");
-    static_assert(NTHREADS / 32 - W_PRO0 == NPRO, "pass C prologue warps: barrier counts use NPRO");
+    static_assert(8 * NBARS + 12 <= CTRL_BYTES, "pass C control block: barriers, TMEM slot, abort flag, zero word");
+    static_assert(W_TAB - W_PRO0 == NPC && NTHREADS / 32 == W_TAB + 1, "pass C prologue warps: barrier counts use NPC");
+    static_assert(GW * RPT == NPRO && OPS == NGRP, "a group's rows cover the 16 row sets; one operand slot per group");
+    static_assert(OP_OFF % 1024 == 0 && OP_BYTES % 1024 == 0, "128-byte-swizzled operand atoms need 1024-byte alignment");
     static_assert(O_OFF % 1024 == 0 && OBUF % 512 == 0, "64-byte-swizzled output boxes need 512-byte alignment");
 };
 
@@ -874,38 +971,49 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
           const float *__restrict__ pref, const float eps, __nv_bfloat16 *__restrict__ out, int *__restrict__ status)
 {
     using L = LayC<DW>;
-    constexpr int S = L::STAGES, NTM = L::NTM, VPH = Width<DW>::VPH, TB = L::TAB_BYTES, SZ = Width<DW>::SZ;
+    constexpr int R = L::RAW, O = L::OPS, NTM = L::NTM, VPH = Width<DW>::VPH, TB = L::TAB_BYTES, SZ = Width<DW>::SZ;
+    constexpr int NT = L::NT;
     const int HV = p.H * VPH;   // virtual heads
     extern __shared__ __align__(1024) unsigned char smraw[];
     const uint32_t raw = s32(smraw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     unsigned char *sm = smraw + pad;
     const uint32_t sb = raw + pad;
-    const uint32_t FULL = sb + L::CTRL, EMPTY = FULL + 8 * S, KREADY = EMPTY + 8 * S, CFULL = KREADY + 8 * S,
-                   CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
-                   PFREE = TFREE + 8 * NTM;
+    // FULL / RAWFREE: raw q slots (TMA landed / read by every prologue warp); OPREADY / OPFREE: operand slots
+    // (written by every prologue warp / the tile's MMAs complete)
+    const uint32_t FULL = sb + L::CTRL, RAWFREE = FULL + 8 * R, OPREADY = RAWFREE + 8 * R, OPFREE = OPREADY + 8 * O,
+                   CFULL = OPFREE + 8 * O, CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
+                   PFREE = TFREE + 8 * NTM, PREADY = PFREE + 16;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * L::NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
+    volatile uint32_t *zero_word = tslot + 2;
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int nunits = p.nseg * p.nquads * p.B;
 
     if (tid == 0) {
-        for (int i = 0; i < S; ++i) {
+        for (int i = 0; i < R; ++i) {
             bar_init(FULL + 8 * i, 1);
-            bar_init(EMPTY + 8 * i, 1);
-            bar_init(KREADY + 8 * i, NPRO);
+            bar_init(RAWFREE + 8 * i, L::GW);
+        }
+        for (int i = 0; i < O; ++i) {
+            bar_init(OPREADY + 8 * i, L::GW);
+            bar_init(OPFREE + 8 * i, 1);
         }
         for (int i = 0; i < NT; ++i) {
             bar_init(CFULL + 8 * i, 1);
-            bar_init(CEMPTY + 8 * i, NPRO);
+            bar_init(CEMPTY + 8 * i, L::GW);
         }
         for (int i = 0; i < NTM; ++i) {
             bar_init(TFULL + 8 * i, 1);
             bar_init(TFREE + 8 * i, L::NEPI);
         }
-        for (int i = 0; i < 2; ++i) bar_init(PFREE + 8 * i, 1);
+        for (int i = 0; i < 2; ++i) {
+            bar_init(PFREE + 8 * i, 1);
+            bar_init(PREADY + 8 * i, L::NPC);
+        }
         *abort_flag = 0;
+        *zero_word = 0u;
         bar_fence_init();
     }
     if (w == L::W_MMA) {
@@ -922,31 +1030,39 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         if (lane == 0) {
             const CUtensorMap *const maps[1] = {&mq};
             const int offs[1] = {0};
-            produce<DW, S, L::STAGE, 1, 2>(p, nunits, sb, sb + L::C_OFF, FULL, EMPTY, CFULL, CEMPTY, maps, offs, &mc,
-                                           &ms, abort_flag);
+            produce_boxes<R, L::RAW_BYTES, 1, 2>(p, nunits, sb + L::RAW_OFF, FULL, RAWFREE, maps, offs, abort_flag);
         }
+    } else if (w == L::W_TAB) {
+        // ---------------- producer: rotary rows of each tile ----------------
+        if (lane == 0) produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag);
     } else if (w == L::W_MMA) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            Ring sr = {0, 0u}, tr = {0, 1u};   // stage (q~ ready), TMEM free
+            Ring sr = {0, 0u}, tr = {0, 1u};   // operand ready, TMEM free
             const uint64_t pdesc0 = desc_sw128(sb + L::P_OFF, 16, 1024);
-            const uint64_t qdesc0 = desc_sw128(sb, 16, 1024);
+            const uint64_t qdesc0 = desc_sw128(sb + L::OP_OFF, 16, 1024);
             int ub = 0, issued = 0, last_tb = 0;
             uint32_t last_phase = 0;
+            Ring pr = {0, 0u};   // prefix operand staged
             bool ok = true;
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const Unit x = unit_at(p, u);
                 if (x.ntile == 0) continue;
+                if (!bar_wait(PREADY + 8 * pr.idx, pr.phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                ring_next<L::NPB>(pr);
                 const uint64_t pd = pdesc0 + (uint64_t)((ub * L::P_BYTES) >> 4);
                 for (int i = 0; i < x.ntile; ++i) {
-                    if (!bar_wait(KREADY + 8 * sr.idx, sr.phase, abort_flag) ||
+                    if (!bar_wait(OPREADY + 8 * sr.idx, sr.phase, abort_flag) ||
                         !bar_wait(TFREE + 8 * tr.idx, tr.phase, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_after();
                     const uint32_t d = tmem + tr.idx * 256;
-                    const uint64_t bd0 = qdesc0 + (uint64_t)((sr.idx * L::STAGE) >> 4);
+                    const uint64_t bd0 = qdesc0 + (uint64_t)((sr.idx * L::OP_BYTES) >> 4);
 #pragma unroll
                     for (int kh = 0; kh < VPH; ++kh) {   // DW = 64: key half kh of P against the operand from atom 2 kh
                         const uint64_t pk = pd + (uint64_t)((kh * L::P_BYTES) >> 4);
@@ -960,11 +1076,11 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                         mma_bf16(d, pk + 2, bd + 6, L::IDESC, 1);
                     }
                     mma_commit(TFULL + 8 * tr.idx);
-                    mma_commit(EMPTY + 8 * sr.idx);
+                    mma_commit(OPFREE + 8 * sr.idx);
                     if (i == x.ntile - 1) mma_commit(PFREE + 8 * ub);
                     last_tb = tr.idx;
                     last_phase = tr.phase ^ 1u;   // TFULL runs one phase behind TFREE's producer-side parity
-                    ring_next<S>(sr);
+                    ring_next<O>(sr);
                     ring_next<NTM>(tr);
                     ++issued;
                 }
@@ -974,10 +1090,19 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         }
     } else if (w >= L::W_PRO0) {
         // ---------------- prologue: prefix staging, phi, normaliser, rotary, hi/lo split ----------------
+        // Group grp of GW warps takes the tiles whose sequence number (over this CTA's units) has parity grp and
+        // writes operand slot grp.  Thread: RPT token rows (row sets RPT gw .. RPT gw + RPT - 1 of pair_offsets),
+        // one quarter f of the 32 dims of head pair g; all its rows share g and f (lane bits).
         const int pw = w - L::W_PRO0, pt = tid - 32 * L::W_PRO0;
-        const PairOffs o = pair_offsets(pw, lane);
+        const int grp = pw / L::GW, gw = pw % L::GW;
+        PairOffs orow[L::RPT];
+#pragma unroll
+        for (int k = 0; k < L::RPT; ++k) orow[k] = pair_offsets(L::RPT * gw + k, lane);
+        const int f = orow[0].f, g = orow[0].g;
         pdl_wait();   // the prefix states come from the previous kernel
-        Ring fr = {0, 0u}, cr = {0, 0u}, br = {0, 1u};   // stage full, table full, P free
+        Ring fr = {0, 0u}, cr = {0, 0u}, br = {0, 1u};   // raw full, table full, P free
+        uint32_t op_phase = 1u;                           // operand slot grp free
+        int tseq = 0;                                     // tile sequence number
         bool ok = true;
         for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
@@ -989,9 +1114,12 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 break;
             }
             ring_next<L::NPB>(br);
-            {   // the quad's prefix -> A operand rows m = (virtual head, c): [P hi | P lo]; thread = (m, quarter
-                // qq of the 32 keys of key half kh); DW = 64: row 32 (vh % 2) + c of head vh / 2, one operand per kh
-                const int m = pt >> 2, qq = pt & 3, vh = HQ * x.hq + (m >> 5);
+#pragma unroll
+            for (int rep = 0; rep < 512 / (32 * L::NPC); ++rep) {
+                // the quad's prefix -> A operand rows m = (virtual head, c): [P hi | P lo]; (m, quarter qq of the
+                // 32 keys of key half kh); DW = 64: row 32 (vh % 2) + c of head vh / 2, one operand per kh
+                const int ptt = pt + 32 * L::NPC * rep;
+                const int m = ptt >> 2, qq = ptt & 3, vh = HQ * x.hq + (m >> 5);
 #pragma unroll
                 for (int kh = 0; kh < VPH; ++kh) {
                     float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
@@ -1013,99 +1141,121 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     store_quarter_hi_lo(sm + L::P_OFF + (ub + kh) * L::P_BYTES, m, qq, hw, lw);
                 }
             }
-            float zq[2][8];   // z[8f, 8f+8) of virtual heads 2g, 2g+1
+            fence_async_smem();   // the MMAs read the prefix operand
+            __syncwarp();
+            if (lane == 0) bar_arrive(PREADY + 8 * ub);
+            // z[8f, 8f+8) of virtual heads 2g, 2g+1, as (even, odd) element vectors over pairs 0-1 and 2-3
+            float2 za01[2], za23[2], zb01[2], zb23[2];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const int vh = HQ * x.hq + 2 * o.g + hh;
+                const int vh = HQ * x.hq + 2 * g + hh;
                 float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
                 if (vh < HV) {
                     const float4 *src = reinterpret_cast<const float4 *>(pref + (pbase + vh / VPH) * SZ + DW * DW +
-                                                                         32 * (vh % VPH) + 8 * o.f);
+                                                                         32 * (vh % VPH) + 8 * f);
                     a4 = src[0];
                     b4 = src[1];
                 }
-                zq[hh][0] = a4.x; zq[hh][1] = a4.y; zq[hh][2] = a4.z; zq[hh][3] = a4.w;
-                zq[hh][4] = b4.x; zq[hh][5] = b4.y; zq[hh][6] = b4.z; zq[hh][7] = b4.w;
+                za01[hh] = make_float2(a4.x, a4.z);
+                zb01[hh] = make_float2(a4.y, a4.w);
+                za23[hh] = make_float2(b4.x, b4.z);
+                zb23[hh] = make_float2(b4.y, b4.w);
             }
             for (int i = 0; i < x.ntile; ++i) {
-                const int st = fr.idx, ct = cr.idx;
-                bool fine = bar_wait(FULL + 8 * fr.idx, fr.phase, abort_flag);
-                fine = bar_wait(CFULL + 8 * cr.idx, cr.phase, abort_flag) && fine;
+                const int rt = fr.idx, ct = cr.idx;
+                const uint32_t rph = fr.phase, cph = cr.phase;
+                ring_next<R>(fr);
+                ring_next<NT>(cr);
+                if (((tseq++) & 1) != grp) continue;   // the other group's tile
+                bool fine = bar_wait(FULL + 8 * rt, rph, abort_flag);
+                fine = bar_wait(CFULL + 8 * ct, cph, abort_flag) && fine;
+                fine = bar_wait(OPFREE + 8 * grp, op_phase, abort_flag) && fine;
                 if (!__all_sync(ALL, fine)) {
                     ok = false;
                     break;
                 }
-                ring_next<S>(fr);
-                ring_next<NT>(cr);
-                unsigned char *stg = sm + st * L::STAGE;
+                op_phase ^= 1u;
+                const unsigned char *rq = sm + L::RAW_OFF + rt * L::RAW_BYTES;
                 const unsigned char *tab = sm + L::C_OFF + ct * TB;
-                // DW = 64: virtual heads 2g, 2g+1 are the halves of one head and rotate with table halves 0, 1
-                float4 c4[2], s4[2];
-                c4[0] = ldsf4(tab + o.tab);
-                s4[0] = ldsf4(tab + TB / 2 + o.tab);
-                c4[1] = VPH == 2 ? ldsf4(tab + 4096 + o.tab) : c4[0];
-                s4[1] = VPH == 2 ? ldsf4(tab + TB / 2 + 4096 + o.tab) : s4[0];
-                const uint4 q0 = lds128(stg + o.in0);   // head 2g
-                const uint4 q1 = lds128(stg + o.in1);   // head 2g+1
-                uint32_t fw[2][4] = {{q0.x, q0.y, q0.z, q0.w}, {q1.x, q1.y, q1.z, q1.w}};
-                float den[2];
+                unsigned char *op = sm + L::OP_OFF + grp * L::OP_BYTES;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float dd = 0.f;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        fw[hh][j] = relu2(fw[hh][j]);
-                        dd = fmaf(bf_lo(fw[hh][j]), zq[hh][2 * j], dd);
-                        dd = fmaf(bf_hi(fw[hh][j]), zq[hh][2 * j + 1], dd);
+                for (int k = 0; k < L::RPT; ++k) {
+                    const PairOffs &o = orow[k];
+                    // the raw features of heads 2g, 2g+1 of this row, phi applied
+                    uint32_t fw[2][4];   // [head of the pair][pair j]
+                    const uint4 q0 = lds128(rq + o.in0);   // head 2g
+                    const uint4 q1 = lds128(rq + o.in1);   // head 2g+1
+                    fw[0][0] = relu2(q0.x); fw[0][1] = relu2(q0.y); fw[0][2] = relu2(q0.z); fw[0][3] = relu2(q0.w);
+                    fw[1][0] = relu2(q1.x); fw[1][1] = relu2(q1.y); fw[1][2] = relu2(q1.z); fw[1][3] = relu2(q1.w);
+                    // rotary rows (DW = 64: virtual heads 2g, 2g+1 are the halves of one head and rotate with
+                    // table halves 0, 1)
+                    float4 c4[2], s4[2];
+                    c4[0] = ldsf4(tab + o.tab);
+                    s4[0] = ldsf4(tab + TB / 2 + o.tab);
+                    c4[1] = VPH == 2 ? ldsf4(tab + 4096 + o.tab) : c4[0];
+                    s4[1] = VPH == 2 ? ldsf4(tab + TB / 2 + 4096 + o.tab) : s4[0];
+                    // z . phi(q) over the token's four quarters (lanes f, f ^ 1, f ^ 2, f ^ 3), then the factor
+                    // 1 / (z . phi(q) + eps)
+                    const float d0 = zdot4_x2(fw[0], za01[0], za23[0], zb01[0], zb23[0]);
+                    const float d1 = zdot4_x2(fw[1], za01[1], za23[1], zb01[1], zb23[1]);
+                    float g0, g1;
+                    if (VPH == 2) {   // one 64-dim head: the two halves' sums add
+                        float dd = d0 + d1;
+                        dd += __shfl_xor_sync(ALL, dd, 1);
+                        dd += __shfl_xor_sync(ALL, dd, 2);
+                        g0 = g1 = rcp_approx(dd + eps);
+                    } else {
+                        // lanes with odd f finish head 2g+1, even f head 2g: each first adds its partner's (lane ^ 1)
+                        // share of the head it finishes, then the other pair of quarters (lane ^ 2)
+                        const bool odd = f & 1;
+                        float keep = odd ? d1 : d0;
+                        keep += __shfl_xor_sync(ALL, odd ? d0 : d1, 1);
+                        keep += __shfl_xor_sync(ALL, keep, 2);
+                        const float mine = rcp_approx(keep + eps);
+                        const float theirs = __shfl_xor_sync(ALL, mine, 1);
+                        g0 = odd ? theirs : mine;
+                        g1 = odd ? mine : theirs;
                     }
-                    den[hh] = dd;
-                }
-                // z . phi(q) of each head over the token's four quarters (lane bits 0-1)
+                    uint32_t hi[2][4], lo[2][4];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    den[hh] += __shfl_xor_sync(ALL, den[hh], 1);
-                    den[hh] += __shfl_xor_sync(ALL, den[hh], 2);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const float4 cc = c4[hh], ss = s4[hh];
+                        rope_split4_x2(fw[hh], make_float2(cc.x, cc.y), make_float2(cc.z, cc.w),
+                                       make_float2(ss.x, ss.y), make_float2(ss.z, ss.w), make_float2(-ss.x, -ss.y),
+                                       make_float2(-ss.z, -ss.w), hh ? g1 : g0, hi[hh], lo[hh]);
+                    }
+                    // head 2g -> atom g, head 2g+1 -> atom 2+g (the operand layout the MMAs and the epilogue expect)
+                    sts128(op + o.in0, hi[0]);
+                    sts128(op + o.in1, lo[0]);
+                    sts128(op + o.out2, hi[1]);
+                    sts128(op + o.out3, lo[1]);
                 }
-                if (VPH == 2) {   // one 64-dim head: z . phi(q) over both halves
-                    const float both = den[0] + den[1];
-                    den[0] = den[1] = both;
-                }
-                // 1 / (z . phi(q) + eps): quarters with even f divide for head 2g, odd f for head 2g+1,
-                // and trade the results (lane bit 0 is bit 0 of f)
-                const float mine = 1.0f / (((o.f & 1) ? den[1] : den[0]) + eps);
-                const float theirs = __shfl_xor_sync(ALL, mine, 1);
-                const float g0 = (o.f & 1) ? theirs : mine, g1 = (o.f & 1) ? mine : theirs;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t hi[4], lo[4];
-                    rope_split4_scaled(fw[hh], c4[hh], s4[hh], hh ? g1 : g0, hi, lo);
-                    // head 2g -> atom g (over the raw chunks just read), head 2g+1 -> atom 2+g
-                    sts128(stg + (hh ? o.out2 : o.in0), hi);
-                    sts128(stg + (hh ? o.out3 : o.in1), lo);
-                }
+                // the stores above used every value this warp loaded from the raw and table slots: release both
+                // with the operand
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    bar_arrive(KREADY + 8 * st);
-                    bar_arrive(CEMPTY + 8 * ct);   // after the rows have been used: see release_after_use
+                    bar_arrive(OPREADY + 8 * grp);
+                    bar_arrive(RAWFREE + 8 * rt);
+                    bar_arrive(CEMPTY + 8 * ct);
                 }
             }
         }
     } else {
-        // ---------------- epilogue: tensor memory -> bf16 -> transposed into a TMA store box ----------------
-        // warp e: head q = e & 3 (tensor-memory lanes 32q + c), tokens [32 hf, 32 hf + 32), hf = e >> 2.
+        // ---------------- epilogue: tensor memory -> bf16 -> transposed into TMA store boxes ----------------
+        // warp q: head q of the quad (tensor-memory lanes 32q + c), the tile's 64 tokens as two halves of 32.
         // The accumulator already carries 1 / (z . phi(q) + eps): the epilogue only converts and moves.
-        const int q = w & 3, hf = w >> 2;
+        const int q = w;
         const size_t tstride = (size_t)p.H * DW;   // elements per token
         // the accumulator block of this warp's rows: its own head's (DW = 32), or column block R of head R's
         // two virtual heads (DW = 64)
         const int ocol = 64 * (VPH == 1 ? atom_of(q) : (q >> 1));
-        const uint32_t obs0 = sb + L::O_OFF + w * 2 * L::OBUF;
+        const uint32_t obs0 = sb + L::O_OFF + w * 2 * L::OBUF;       // one box per token half
         const unsigned char *obp0 = sm + L::O_OFF + w * 2 * L::OBUF;
         // stmatrix row of this lane: c group m = lane >> 3 (c in [8m, 8m + 8)), token 8j + k, k = lane & 7;
         // the box is [32 tok][32 c] bf16 with the 64-byte swizzle (16-byte chunk m of row r at m ^ ((r >> 1) & 3))
         const int smm = lane >> 3, smk = lane & 7;
-        int ob = 0;
+        const uint64_t stream_pol = policy_evict_first();
         Ring tr = {0, 0u};   // TMEM full
         bool ok = true;
         for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
@@ -1120,43 +1270,47 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 ring_next<NTM>(tr);
                 tc_after();
                 const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
-                if (lane == 0) bulk_wait_read1();   // this buffer's previous store has read it
+                if (lane == 0) bulk_wait_read0();   // the previous tile's stores have read both boxes
                 __syncwarp();
-                uint32_t v[32];
-                const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + ocol + 32 * hf;
-                tmem_ld16x256_x4x2(ta, ta + (16u << 16), v);
-                tc_before();
-                __syncwarp();
-                if (lane == 0) bar_arrive(TFREE + 8 * tb);   // the accumulator is in registers: free the slot
-                // v[16 L + 4 j + i] = D[c = 16 L + lane / 4 + 8 (i >> 1)][tok = 8 j + 2 (lane % 4) + (i & 1)]
-                const uint32_t obs = obs0 + ob * L::OBUF;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int tok = 8 * j + smk;
-                    stsm4_trans(obs + tok * 64 + ((smm ^ ((tok >> 1) & 3)) << 4),
-                                pack_bf2(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1])),
-                                pack_bf2(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])),
-                                pack_bf2(__uint_as_float(v[16 + 4 * j]), __uint_as_float(v[16 + 4 * j + 1])),
-                                pack_bf2(__uint_as_float(v[16 + 4 * j + 2]), __uint_as_float(v[16 + 4 * j + 3])));
-                }
-                if (nt == T) {
-                    fence_async_smem();
-                    __syncwarp();
-                    if (lane == 0 && head < HV) tma_store3_hint(&mo, obs, LCLA_D * head, t + 32 * hf, x.b, policy_evict_first());
-                } else {   // ragged tile: lane = token, its 64-byte row back from the box to global memory
-                    __syncwarp();
-                    const int tok = lane;
-                    if (head < HV && 32 * hf + tok < nt) {
-                        const unsigned char *row = obp0 + ob * L::OBUF + tok * 64;
-                        uint4 *g = reinterpret_cast<uint4 *>(out + ((size_t)x.b * p.N + t + 32 * hf + tok) * tstride +
-                                                             (size_t)head * LCLA_D);
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) g[m] = lds128(row + ((m ^ ((tok >> 1) & 3)) << 4));
+#pragma unroll 1
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t v[32];
+                    const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + ocol + 32 * hf;
+                    tmem_ld16x256_x4x2(ta, ta + (16u << 16), v);
+                    if (hf == 1) {   // the accumulator is in registers: free the slot
+                        tc_before();
+                        __syncwarp();
+                        if (lane == 0) bar_arrive(TFREE + 8 * tb);
                     }
-                    __syncwarp();
+                    // v[16 L + 4 j + i] = D[c = 16 L + lane / 4 + 8 (i >> 1)][tok = 8 j + 2 (lane % 4) + (i & 1)]
+                    const uint32_t obs = obs0 + hf * L::OBUF;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int tok = 8 * j + smk;
+                        stsm4_trans(obs + tok * 64 + ((smm ^ ((tok >> 1) & 3)) << 4),
+                                    pack_bf2(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1])),
+                                    pack_bf2(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])),
+                                    pack_bf2(__uint_as_float(v[16 + 4 * j]), __uint_as_float(v[16 + 4 * j + 1])),
+                                    pack_bf2(__uint_as_float(v[16 + 4 * j + 2]), __uint_as_float(v[16 + 4 * j + 3])));
+                    }
+                    if (nt == T) {
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0 && head < HV) tma_store3_hint(&mo, obs, LCLA_D * head, t + 32 * hf, x.b, stream_pol);
+                    } else {   // ragged tile: lane = token, its 64-byte row back from the box to global memory
+                        __syncwarp();
+                        const int tok = lane;
+                        if (head < HV && 32 * hf + tok < nt) {
+                            const unsigned char *row = obp0 + hf * L::OBUF + tok * 64;
+                            uint4 *gp = reinterpret_cast<uint4 *>(out + ((size_t)x.b * p.N + t + 32 * hf + tok) * tstride +
+                                                                  (size_t)head * LCLA_D);
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) gp[m] = lds128(row + ((m ^ ((tok >> 1) & 3)) << 4));
+                        }
+                        __syncwarp();
+                    }
                 }
-                if (lane == 0) bulk_commit();   // one group per buffer use keeps the read-wait accounting exact
-                ob ^= 1;
+                if (lane == 0) bulk_commit();
             }
         }
         if (lane == 0) bulk_wait_all();
