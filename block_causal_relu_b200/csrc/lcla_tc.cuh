@@ -59,6 +59,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "lcla_common.cuh"
@@ -315,6 +316,17 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uin
 {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Shared-memory matrix descriptor, 64-byte swizzle (sm_100 layout, version 1).
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
+}
+// Instruction descriptor: kind::f16 with fp16 A and B (both K-major), fp32 D.
+constexpr uint32_t idesc_f16(int M, int N)
+{
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 // Instruction descriptor: kind::f16 with bf16 A and B, fp32 D.
 constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major)
@@ -921,49 +933,94 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
 // ---------------------------------------------------------------------------
 template <int DW>
 struct LayC {
-    // raw q ring: one tile's two TMA boxes [64 tok][2 heads x 32] bf16 (16 KB) per slot, released as soon as
-    // the prologue has read it; operand ring: the tile's q~ operand, 4 atoms of [64 rows (tok)][q~hi 32 |
-    // q~lo 32] (32 KB), held until the tile's MMAs complete.  DW = 64 has table slots twice as large.
-    static constexpr int RAW = DW == 32 ? 5 : 4, RAW_BYTES = 16384;
-    static constexpr int OPS = 2, OP_BYTES = 32768;
+    // raw q ring: one tile's two TMA boxes [64 tok][2 heads x 32] bf16 (16 KB) per slot, released when the
+    // prologue has used it; operand ring: the tile's query operand, 4 atoms of [64 rows (tok)][32 fp16]
+    // (64-byte swizzle, 16 KB), held until the tile's MMAs complete.  DW = 64 has table slots twice as large.
+    static constexpr int RAW = DW == 32 ? 6 : 5, RAW_BYTES = 16384;
+    static constexpr int OPS = 2, OP_BYTES = 16384, ATOM = 4096;
     static constexpr int RAW_OFF = 0, OP_OFF = RAW * RAW_BYTES;
     static constexpr int TAB_BYTES = Width<DW>::TAB_BYTES;
-    static constexpr int NT = DW == 32 ? 4 : 3;                     // rotary-table ring slots
+    static constexpr int NT = DW == 32 ? 5 : 3;                     // rotary-table ring slots
     static constexpr int C_OFF = OP_OFF + OPS * OP_BYTES;           // rotary-table ring
-    // prefix operands [128 rows (virtual head, c)][P hi | P lo]: DW = 32, one per unit, double-buffered;
-    // DW = 64, the unit's two key halves (e < 32, e >= 32) in one buffer
+    // prefix operands [128 rows (virtual head, c)][P hi | P lo] fp16, each row scaled by a power of two: DW = 32,
+    // one per unit, double-buffered; DW = 64, the unit's two key halves (e < 32, e >= 32) in one buffer
     static constexpr int P_BYTES = 16384, NPB = DW == 32 ? 2 : 1;
     static constexpr int P_OFF = C_OFF + NT * TAB_BYTES;
-    static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 4 warps x 2 x [32 tok][32 c] bf16
+    static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 8 warps x [32 tok][32 c] bf16
     static constexpr int OBUF = 2048;
-    static constexpr int CTRL = O_OFF + 4 * 2 * OBUF;               // mbarriers, tensor-memory slot, abort flag
+    // the normaliser 1 / (z . phi(q) + eps) of each tile, [4 virtual heads][64 tok] fp32, from the prologue to the
+    // epilogue; and the inverse row scales of each prefix operand, [2][128] fp32
+    static constexpr int NG = 4, G_BYTES = 1024;
+    static constexpr int G_OFF = O_OFF + 8 * OBUF;
+    static constexpr int S_OFF = G_OFF + NG * G_BYTES;
+    static constexpr int CTRL = S_OFF + 2 * 128 * 4;                // mbarriers, tensor-memory slot, abort flag
     static constexpr int BYTES = CTRL + CTRL_BYTES + 1024;          // + worst-case 1024-byte alignment pad
     // prologue: 8 warps in two groups of 4 that take alternate tiles, so that one group's waits, fences and
     // load latencies overlap the other's arithmetic; a thread does four token rows of its group's tiles (the
     // row sets that pair_offsets gives warps 4 gw .. 4 gw + 3)
-    static constexpr int NPC = 16, NGRP = 2, GW = NPC / NGRP, RPT = NPRO / GW;
-    static constexpr int NTHREADS = 736;                            // epilogue 0-3, producer 4, MMA 5, prologue 6-21,
-                                                                    // tables 22
-    static constexpr int W_PROD = 4, W_MMA = 5, W_PRO0 = 6, W_TAB = 22, NEPI = 4;
+    static constexpr int NPC = 8, NGRP = 2, GW = NPC / NGRP, RPT = NPRO / GW;
+    static constexpr int NTHREADS = 608;                            // epilogue 0-7, producer 8, MMA 9, prologue 10-17,
+                                                                    // tables 18
+    static constexpr int W_PROD = 8, W_MMA = 9, W_PRO0 = 10, W_TAB = 18, NEPI = 8;
     static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
-    static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
+    static constexpr uint32_t IDESC = idesc_f16(128, 256);
     static constexpr int TMEM_COLS = NTM * 256;
-    static constexpr int NBARS = 2 * RAW + 2 * OPS + 2 * NT + 2 * NTM + 4;
+    static constexpr int NBARS = 2 * RAW + 2 * OPS + 2 * NT + 2 * NTM + 6 + 2 * NG;
     static_assert(NPB * Width<DW>::VPH == 2, "two prefix operands of P_BYTES");
     static_assert(BYTES <= SMEM_MAX, "pass C shared memory");
-    static_assert(8 * NBARS + 12 <= CTRL_BYTES, "pass C control block: barriers, TMEM slot, abort flag, zero word");
+    static_assert(8 * NBARS + 12 <= CTRL_BYTES, "pass C control block: barriers, TMEM slot, abort flag");
     static_assert(W_TAB - W_PRO0 == NPC && NTHREADS / 32 == W_TAB + 1, "pass C prologue warps: barrier counts use NPC");
     static_assert(GW * RPT == NPRO && OPS == NGRP, "a group's rows cover the 16 row sets; one operand slot per group");
-    static_assert(OP_OFF % 1024 == 0 && OP_BYTES % 1024 == 0, "128-byte-swizzled operand atoms need 1024-byte alignment");
+    static_assert(OP_OFF % 1024 == 0 && OP_BYTES % 1024 == 0 && P_OFF % 1024 == 0, "swizzled operands: 1 KB alignment");
     static_assert(O_OFF % 1024 == 0 && OBUF % 512 == 0, "64-byte-swizzled output boxes need 512-byte alignment");
 };
 
-// Pass C over head width DW.  At DW = 64 the quad holds two heads as four
-// virtual heads; the output of head R, half a, is sum over the key halves b of
-// P_R[32 a + c][32 b + e] q~_{R, b}[e]: one set of MMAs with the first key half
-// of P against the stage's operand, one with the second half against the
-// operand two atoms on (atoms hold virtual heads 0, 2, 1, 3, so the window from
-// atom 2 holds 1, 3), which lands both sums in column block R.
+// Chunk f (16 bytes) of row r of a [rows][64 B] operand or box with the 64-byte swizzle.
+__device__ __forceinline__ int sw64(int r, int f) { return r * 64 + ((f ^ ((r >> 1) & 3)) << 4); }
+
+// fp16 operand of one quarter (4 pairs) of a head: the ReLU features rotated in fp32, rounded once to fp16
+// (RNE).  The features are O(1) (bf16 inputs through ReLU and a rotation), inside fp16's range; the normaliser
+// is applied to the accumulator instead.  Returns four packed f16x2 words, pair j in word j.
+__device__ __forceinline__ uint4 rope4_f16(const uint32_t *fw, float2 c01, float2 c23, float2 s01, float2 s23,
+                                           float2 ns01, float2 ns23)
+{
+    const float2 a01 = make_float2(bf_low(fw[0]), bf_low(fw[1])), a23 = make_float2(bf_low(fw[2]), bf_low(fw[3]));
+    const float2 b01 = make_float2(bf_high(fw[0]), bf_high(fw[1])), b23 = make_float2(bf_high(fw[2]), bf_high(fw[3]));
+    const float2 y0_01 = __ffma2_rn(a01, c01, __fmul2_rn(b01, ns01));   // a c - b s
+    const float2 y0_23 = __ffma2_rn(a23, c23, __fmul2_rn(b23, ns23));
+    const float2 y1_01 = __ffma2_rn(b01, c01, __fmul2_rn(a01, s01));    // a s + b c
+    const float2 y1_23 = __ffma2_rn(b23, c23, __fmul2_rn(a23, s23));
+    const __half2 h0 = __floats2half2_rn(y0_01.x, y1_01.x), h1 = __floats2half2_rn(y0_01.y, y1_01.y);
+    const __half2 h2 = __floats2half2_rn(y0_23.x, y1_23.x), h3 = __floats2half2_rn(y0_23.y, y1_23.y);
+    return make_uint4(*reinterpret_cast<const uint32_t *>(&h0), *reinterpret_cast<const uint32_t *>(&h1),
+                      *reinterpret_cast<const uint32_t *>(&h2), *reinterpret_cast<const uint32_t *>(&h3));
+}
+
+// Power-of-two scale that brings a row whose largest magnitude is m below 2^14 (fp16 holds up to 65504),
+// and its inverse; zero, subnormal and non-finite maxima keep the scale 1 (NaN states stay NaN).
+__device__ __forceinline__ void row_scale(float m, float &scale, float &inv)
+{
+    const int E = (int)((__float_as_uint(m) >> 23) & 0xffu);   // biased exponent: m < 2^(E - 126)
+    if (E == 0 || E == 255) {
+        scale = inv = 1.0f;
+        return;
+    }
+    const int es = min(max(267 - E, 1), 253);                   // 2^(es - 127) = 2^(14 - (E - 126))
+    scale = __uint_as_float((uint32_t)es << 23);
+    inv = __uint_as_float((uint32_t)(254 - es) << 23);
+}
+
+// Pass C over head width DW.  The accumulator holds, per (virtual head, c)
+// row and (head, token) column, sum_e P~[c][e] q~[e] with P~ = the prefix row
+// times its power-of-two scale (fp16 hi + lo, 22 significant bits) and q~ =
+// the rotated ReLU query in fp16 (one term); the epilogue multiplies by the
+// inverse row scale and the token's 1 / (z . phi(q) + eps).  At DW = 64 the
+// quad holds two heads as four virtual heads; the output of head R, half a, is
+// sum over the key halves b of P_R[32 a + c][32 b + e] q~_{R, b}[e]: one set of
+// MMAs with the first key half of P against the tile's operand, one with the
+// second half against the operand two atoms on (atoms hold virtual heads
+// 0, 2, 1, 3, so the window from atom 2 holds 1, 3), which lands both sums in
+// column block R.
 template <int DW>
 __global__ void __launch_bounds__(LayC<DW>::NTHREADS, 1)
 pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mc,
@@ -972,21 +1029,25 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
 {
     using L = LayC<DW>;
     constexpr int R = L::RAW, O = L::OPS, NTM = L::NTM, VPH = Width<DW>::VPH, TB = L::TAB_BYTES, SZ = Width<DW>::SZ;
-    constexpr int NT = L::NT;
+    constexpr int NT = L::NT, NG = L::NG;
     const int HV = p.H * VPH;   // virtual heads
     extern __shared__ __align__(1024) unsigned char smraw[];
     const uint32_t raw = s32(smraw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     unsigned char *sm = smraw + pad;
     const uint32_t sb = raw + pad;
-    // FULL / RAWFREE: raw q slots (TMA landed / read by every prologue warp); OPREADY / OPFREE: operand slots
-    // (written by every prologue warp / the tile's MMAs complete)
+    // FULL / RAWFREE: raw q slots (TMA landed / used by the tile's prologue group); OPREADY / OPFREE: operand
+    // slots (written by the group / the tile's MMAs complete); CFULL / CEMPTY: rotary rows; TFULL / TFREE:
+    // accumulators; PFREE / PREADY: prefix operands (the unit's MMAs complete / staged by every prologue warp);
+    // SFREE: the prefix operand's inverse row scales read by every epilogue warp; GREADY / GFREE: normalisers
     const uint32_t FULL = sb + L::CTRL, RAWFREE = FULL + 8 * R, OPREADY = RAWFREE + 8 * R, OPFREE = OPREADY + 8 * O,
                    CFULL = OPFREE + 8 * O, CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
-                   PFREE = TFREE + 8 * NTM, PREADY = PFREE + 16;
+                   PFREE = TFREE + 8 * NTM, PREADY = PFREE + 16, SFREE = PREADY + 16, GREADY = SFREE + 16,
+                   GFREE = GREADY + 8 * NG;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * L::NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
-    volatile uint32_t *zero_word = tslot + 2;
+    float *gbuf = reinterpret_cast<float *>(sm + L::G_OFF);   // [NG][4 vh][64 tok]
+    float *sinv = reinterpret_cast<float *>(sm + L::S_OFF);   // [2][128 rows]
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int nunits = p.nseg * p.nquads * p.B;
@@ -1011,9 +1072,13 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         for (int i = 0; i < 2; ++i) {
             bar_init(PFREE + 8 * i, 1);
             bar_init(PREADY + 8 * i, L::NPC);
+            bar_init(SFREE + 8 * i, L::NEPI);
+        }
+        for (int i = 0; i < NG; ++i) {
+            bar_init(GREADY + 8 * i, L::GW);
+            bar_init(GFREE + 8 * i, L::NEPI);
         }
         *abort_flag = 0;
-        *zero_word = 0u;
         bar_fence_init();
     }
     if (w == L::W_MMA) {
@@ -1040,7 +1105,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         if (lane == 0) {
             Ring sr = {0, 0u}, tr = {0, 1u};   // operand ready, TMEM free
             const uint64_t pdesc0 = desc_sw128(sb + L::P_OFF, 16, 1024);
-            const uint64_t qdesc0 = desc_sw128(sb + L::OP_OFF, 16, 1024);
+            const uint64_t qdesc0 = desc_sw64(sb + L::OP_OFF, 16, 512);
             int ub = 0, issued = 0, last_tb = 0;
             uint32_t last_phase = 0;
             Ring pr = {0, 0u};   // prefix operand staged
@@ -1066,14 +1131,12 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
 #pragma unroll
                     for (int kh = 0; kh < VPH; ++kh) {   // DW = 64: key half kh of P against the operand from atom 2 kh
                         const uint64_t pk = pd + (uint64_t)((kh * L::P_BYTES) >> 4);
-                        const uint64_t bd = bd0 + (uint64_t)((kh * 2 * 8192) >> 4);
-                        // K steps of 16 elements = 32 B = 2 descriptor units; hi at +0, lo at +64 B
-                        mma_bf16(d, pk + 0, bd + 0, L::IDESC, kh);   // P hi . q~hi
+                        const uint64_t bd = bd0 + (uint64_t)((kh * 2 * L::ATOM) >> 4);
+                        // K steps of 16 elements = 32 B = 2 descriptor units; P hi at +0, P lo at +64 B
+                        mma_bf16(d, pk + 0, bd + 0, L::IDESC, kh);   // P~hi . q~
                         mma_bf16(d, pk + 2, bd + 2, L::IDESC, 1);
-                        mma_bf16(d, pk + 4, bd + 0, L::IDESC, 1);    // P lo . q~hi
+                        mma_bf16(d, pk + 4, bd + 0, L::IDESC, 1);    // P~lo . q~
                         mma_bf16(d, pk + 6, bd + 2, L::IDESC, 1);
-                        mma_bf16(d, pk + 0, bd + 4, L::IDESC, 1);    // P hi . q~lo
-                        mma_bf16(d, pk + 2, bd + 6, L::IDESC, 1);
                     }
                     mma_commit(TFULL + 8 * tr.idx);
                     mma_commit(OPFREE + 8 * sr.idx);
@@ -1089,37 +1152,40 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             if (!ok && issued > 0) bar_wait_quiet(TFULL + 8 * last_tb, last_phase);
         }
     } else if (w >= L::W_PRO0) {
-        // ---------------- prologue: prefix staging, phi, normaliser, rotary, hi/lo split ----------------
+        // ---------------- prologue: prefix staging, phi, normaliser, rotary, fp16 operand ----------------
         // Group grp of GW warps takes the tiles whose sequence number (over this CTA's units) has parity grp and
         // writes operand slot grp.  Thread: RPT token rows (row sets RPT gw .. RPT gw + RPT - 1 of pair_offsets),
         // one quarter f of the 32 dims of head pair g; all its rows share g and f (lane bits).
         const int pw = w - L::W_PRO0, pt = tid - 32 * L::W_PRO0;
         const int grp = pw / L::GW, gw = pw % L::GW;
-        PairOffs orow[L::RPT];
-#pragma unroll
-        for (int k = 0; k < L::RPT; ++k) orow[k] = pair_offsets(L::RPT * gw + k, lane);
-        const int f = orow[0].f, g = orow[0].g;
+        const int f = lane & 3, g = (lane >> 3) & 1;   // as pair_offsets gives them
         pdl_wait();   // the prefix states come from the previous kernel
-        Ring fr = {0, 0u}, cr = {0, 0u}, br = {0, 1u};   // raw full, table full, P free
-        uint32_t op_phase = 1u;                           // operand slot grp free
-        int tseq = 0;                                     // tile sequence number
+        Ring fr = {0, 0u}, cr = {0, 0u}, br = {0, 1u}, sr = {0, 1u};   // raw full, table full, P free, scales read
+        uint32_t op_phase = 1u;                                         // operand slot grp free
+        int tseq = 0;                                                   // tile sequence number
         bool ok = true;
         for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
             if (x.ntile == 0) continue;
             const int ub = br.idx;
             const size_t pbase = ((size_t)x.blk * p.B + x.b) * p.H;
-            if (!__all_sync(ALL, bar_wait(PFREE + 8 * br.idx, br.phase, abort_flag))) {
+            bool fine = bar_wait(PFREE + 8 * br.idx, br.phase, abort_flag);
+            fine = bar_wait(SFREE + 8 * sr.idx, sr.phase, abort_flag) && fine;
+            if (!__all_sync(ALL, fine)) {
                 ok = false;
                 break;
             }
             ring_next<L::NPB>(br);
-#pragma unroll
+            ring_next<L::NPB>(sr);
+#pragma unroll 1
             for (int rep = 0; rep < 512 / (32 * L::NPC); ++rep) {
-                // the quad's prefix -> A operand rows m = (virtual head, c): [P hi | P lo]; (m, quarter qq of the
-                // 32 keys of key half kh); DW = 64: row 32 (vh % 2) + c of head vh / 2, one operand per kh
+                // the quad's prefix -> A operand rows m = (virtual head, c): [P~hi | P~lo] fp16, P~ = P times the
+                // row's power-of-two scale; thread (m, quarter qq of the 32 keys of each key half kh), the row's
+                // four threads in lanes qq = 0..3; DW = 64: row 32 (vh % 2) + c of head vh / 2, one operand per kh
                 const int ptt = pt + 32 * L::NPC * rep;
                 const int m = ptt >> 2, qq = ptt & 3, vh = HQ * x.hq + (m >> 5);
+                float y[VPH][8];
+                float mx = 0.f;
 #pragma unroll
                 for (int kh = 0; kh < VPH; ++kh) {
                     float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
@@ -1129,17 +1195,30 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                         a4 = src[0];
                         b4 = src[1];
                     }
-                    const float y[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+                    y[kh][0] = a4.x; y[kh][1] = a4.y; y[kh][2] = a4.z; y[kh][3] = a4.w;
+                    y[kh][4] = b4.x; y[kh][5] = b4.y; y[kh][6] = b4.z; y[kh][7] = b4.w;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(y[kh][j]));   // NaN: fmaxf keeps the other
+                }
+                mx = fmaxf(mx, __shfl_xor_sync(ALL, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(ALL, mx, 2));
+                float scale, inv;
+                row_scale(mx, scale, inv);
+#pragma unroll
+                for (int kh = 0; kh < VPH; ++kh) {
                     uint32_t hw[4], lw[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
-                        const float2 hf = __bfloat1622float2(h2);
-                        hw[j] = bf2_bits(h2);
-                        lw[j] = pack_bf2(y[2 * j] - hf.x, y[2 * j + 1] - hf.y);
+                        const float a = y[kh][2 * j] * scale, b = y[kh][2 * j + 1] * scale;   // exact
+                        const __half2 h2 = __floats2half2_rn(a, b);
+                        const float2 hf = __half22float2(h2);
+                        const __half2 l2 = __floats2half2_rn(a - hf.x, b - hf.y);
+                        hw[j] = *reinterpret_cast<const uint32_t *>(&h2);
+                        lw[j] = *reinterpret_cast<const uint32_t *>(&l2);
                     }
                     store_quarter_hi_lo(sm + L::P_OFF + (ub + kh) * L::P_BYTES, m, qq, hw, lw);
                 }
+                if (qq == 0) sinv[ub * 128 + m] = inv;
             }
             fence_async_smem();   // the MMAs read the prefix operand
             __syncwarp();
@@ -1162,25 +1241,41 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 zb23[hh] = make_float2(b4.y, b4.w);
             }
             for (int i = 0; i < x.ntile; ++i) {
-                const int rt = fr.idx, ct = cr.idx;
-                const uint32_t rph = fr.phase, cph = cr.phase;
+                const int rt = fr.idx, ct = cr.idx, gt = tseq % NG;
+                const uint32_t rph = fr.phase, cph = cr.phase, gph = (uint32_t)(((tseq / NG) & 1) ^ 1);
                 ring_next<R>(fr);
                 ring_next<NT>(cr);
                 if (((tseq++) & 1) != grp) continue;   // the other group's tile
                 bool fine = bar_wait(FULL + 8 * rt, rph, abort_flag);
                 fine = bar_wait(CFULL + 8 * ct, cph, abort_flag) && fine;
-                fine = bar_wait(OPFREE + 8 * grp, op_phase, abort_flag) && fine;
+                fine = bar_wait(GFREE + 8 * gt, gph, abort_flag) && fine;
                 if (!__all_sync(ALL, fine)) {
                     ok = false;
                     break;
                 }
-                op_phase ^= 1u;
                 const unsigned char *rq = sm + L::RAW_OFF + rt * L::RAW_BYTES;
                 const unsigned char *tab = sm + L::C_OFF + ct * TB;
                 unsigned char *op = sm + L::OP_OFF + grp * L::OP_BYTES;
+                float *gt_buf = gbuf + gt * (L::G_BYTES / 4);
+                // rows [0, RPT / 2) are computed before the wait for the operand slot (free once the MMAs of
+                // this group's previous tile are done), so that their arithmetic overlaps those MMAs
+                uint4 hq[L::RPT / 2][2];
+                bool slot_ok = true;
 #pragma unroll
                 for (int k = 0; k < L::RPT; ++k) {
-                    const PairOffs &o = orow[k];
+                    if (k == L::RPT / 2) {
+                        slot_ok = __all_sync(ALL, bar_wait(OPFREE + 8 * grp, op_phase, abort_flag));
+                        if (!slot_ok) break;
+                        op_phase ^= 1u;
+#pragma unroll
+                        for (int k2 = 0; k2 < L::RPT / 2; ++k2) {
+                            const int r2 = pair_offsets(L::RPT * gw + k2, lane).r;
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh)   // virtual head 2g + hh -> atom atom_of(2g + hh)
+                                *reinterpret_cast<uint4 *>(op + atom_of(2 * g + hh) * L::ATOM + sw64(r2, f)) = hq[k2][hh];
+                        }
+                    }
+                    const PairOffs o = pair_offsets(L::RPT * gw + k, lane);
                     // the raw features of heads 2g, 2g+1 of this row, phi applied
                     uint32_t fw[2][4];   // [head of the pair][pair j]
                     const uint4 q0 = lds128(rq + o.in0);   // head 2g
@@ -1195,15 +1290,14 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     c4[1] = VPH == 2 ? ldsf4(tab + 4096 + o.tab) : c4[0];
                     s4[1] = VPH == 2 ? ldsf4(tab + TB / 2 + 4096 + o.tab) : s4[0];
                     // z . phi(q) over the token's four quarters (lanes f, f ^ 1, f ^ 2, f ^ 3), then the factor
-                    // 1 / (z . phi(q) + eps)
+                    // 1 / (z . phi(q) + eps) for the epilogue
                     const float d0 = zdot4_x2(fw[0], za01[0], za23[0], zb01[0], zb23[0]);
                     const float d1 = zdot4_x2(fw[1], za01[1], za23[1], zb01[1], zb23[1]);
-                    float g0, g1;
                     if (VPH == 2) {   // one 64-dim head: the two halves' sums add
                         float dd = d0 + d1;
                         dd += __shfl_xor_sync(ALL, dd, 1);
                         dd += __shfl_xor_sync(ALL, dd, 2);
-                        g0 = g1 = rcp_approx(dd + eps);
+                        if (f < 2) gt_buf[(2 * g + f) * 64 + o.r] = rcp_approx(dd + eps);
                     } else {
                         // lanes with odd f finish head 2g+1, even f head 2g: each first adds its partner's (lane ^ 1)
                         // share of the head it finishes, then the other pair of quarters (lane ^ 2)
@@ -1211,104 +1305,128 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                         float keep = odd ? d1 : d0;
                         keep += __shfl_xor_sync(ALL, odd ? d0 : d1, 1);
                         keep += __shfl_xor_sync(ALL, keep, 2);
-                        const float mine = rcp_approx(keep + eps);
-                        const float theirs = __shfl_xor_sync(ALL, mine, 1);
-                        g0 = odd ? theirs : mine;
-                        g1 = odd ? mine : theirs;
+                        if (f < 2) gt_buf[(2 * g + f) * 64 + o.r] = rcp_approx(keep + eps);
                     }
-                    uint32_t hi[2][4], lo[2][4];
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const float4 cc = c4[hh], ss = s4[hh];
-                        rope_split4_x2(fw[hh], make_float2(cc.x, cc.y), make_float2(cc.z, cc.w),
-                                       make_float2(ss.x, ss.y), make_float2(ss.z, ss.w), make_float2(-ss.x, -ss.y),
-                                       make_float2(-ss.z, -ss.w), hh ? g1 : g0, hi[hh], lo[hh]);
+                        const uint4 h = rope4_f16(fw[hh], make_float2(cc.x, cc.y), make_float2(cc.z, cc.w),
+                                              make_float2(ss.x, ss.y), make_float2(ss.z, ss.w),
+                                              make_float2(-ss.x, -ss.y), make_float2(-ss.z, -ss.w));
+                        if (k < L::RPT / 2)
+                            hq[k % (L::RPT / 2)][hh] = h;
+                        else   // virtual head 2g + hh -> atom atom_of(2g + hh): [64 tok][32 fp16], chunk f of row r
+                            *reinterpret_cast<uint4 *>(op + atom_of(2 * g + hh) * L::ATOM + sw64(o.r, f)) = h;
                     }
-                    // head 2g -> atom g, head 2g+1 -> atom 2+g (the operand layout the MMAs and the epilogue expect)
-                    sts128(op + o.in0, hi[0]);
-                    sts128(op + o.in1, lo[0]);
-                    sts128(op + o.out2, hi[1]);
-                    sts128(op + o.out3, lo[1]);
+                }
+                if (!slot_ok) {
+                    ok = false;
+                    break;
                 }
                 // the stores above used every value this warp loaded from the raw and table slots: release both
-                // with the operand
+                // with the operand and the normalisers
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
                     bar_arrive(OPREADY + 8 * grp);
+                    bar_arrive(GREADY + 8 * gt);
                     bar_arrive(RAWFREE + 8 * rt);
                     bar_arrive(CEMPTY + 8 * ct);
                 }
             }
         }
     } else {
-        // ---------------- epilogue: tensor memory -> bf16 -> transposed into TMA store boxes ----------------
-        // warp q: head q of the quad (tensor-memory lanes 32q + c), the tile's 64 tokens as two halves of 32.
-        // The accumulator already carries 1 / (z . phi(q) + eps): the epilogue only converts and moves.
-        const int q = w;
+        // ---------------- epilogue: tensor memory -> scaled -> bf16 -> transposed into a TMA store box ----------------
+        // warp e: virtual head q = e & 3 of the quad (tensor-memory lanes 32q + c), tokens [32 hf, 32 hf + 32) of
+        // the tile, hf = e >> 2.  out = accumulator x (inverse row scale of c) x (1 / (z . phi(q) + eps) of the
+        // token).
+        const int q = w & 3, hf = w >> 2;
         const size_t tstride = (size_t)p.H * DW;   // elements per token
         // the accumulator block of this warp's rows: its own head's (DW = 32), or column block R of head R's
         // two virtual heads (DW = 64)
         const int ocol = 64 * (VPH == 1 ? atom_of(q) : (q >> 1));
-        const uint32_t obs0 = sb + L::O_OFF + w * 2 * L::OBUF;       // one box per token half
-        const unsigned char *obp0 = sm + L::O_OFF + w * 2 * L::OBUF;
+        const uint32_t obs = sb + L::O_OFF + w * L::OBUF;
+        const unsigned char *obp = sm + L::O_OFF + w * L::OBUF;
         // stmatrix row of this lane: c group m = lane >> 3 (c in [8m, 8m + 8)), token 8j + k, k = lane & 7;
         // the box is [32 tok][32 c] bf16 with the 64-byte swizzle (16-byte chunk m of row r at m ^ ((r >> 1) & 3))
         const int smm = lane >> 3, smk = lane & 7;
         const uint64_t stream_pol = policy_evict_first();
-        Ring tr = {0, 0u};   // TMEM full
+        Ring tr = {0, 0u}, pr = {0, 0u}, gr = {0, 0u};   // TMEM full, prefix staged, normalisers ready
         bool ok = true;
         for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
             const Unit x = unit_at(p, u);
+            if (x.ntile == 0) continue;
             const int head = HQ * x.hq + q;
+            // this lane's accumulator rows c = lane / 4 + 8 k: their inverse scales
+            const int sb_idx = pr.idx;
+            if (!__all_sync(ALL, bar_wait(PREADY + 8 * pr.idx, pr.phase, abort_flag))) {
+                ok = false;
+                break;
+            }
+            ring_next<L::NPB>(pr);
+            float rinv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) rinv[k] = sinv[sb_idx * 128 + 32 * q + (lane >> 2) + 8 * k];
+            __syncwarp();
+            if (lane == 0) bar_arrive(SFREE + 8 * sb_idx);
             for (int i = 0; i < x.ntile; ++i) {
-                const int tb = tr.idx;
-                if (!__all_sync(ALL, bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag))) {
+                const int tb = tr.idx, gt = gr.idx;
+                bool fine = bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag);
+                fine = bar_wait(GREADY + 8 * gr.idx, gr.phase, abort_flag) && fine;
+                if (!__all_sync(ALL, fine)) {
                     ok = false;
                     break;
                 }
                 ring_next<NTM>(tr);
+                ring_next<NG>(gr);
                 tc_after();
                 const int t = x.t0 + i * T, nt = min(T, x.t1 - t);
-                if (lane == 0) bulk_wait_read0();   // the previous tile's stores have read both boxes
+                // the normalisers of this lane's token pairs (8 j + 2 (lane % 4), + 1) of the half
+                float2 gn[4];
+                const float *gq = gbuf + gt * (L::G_BYTES / 4) + q * 64 + 32 * hf + 2 * (lane & 3);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) gn[j] = *reinterpret_cast<const float2 *>(gq + 8 * j);
+                uint32_t v[32];
+                const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + ocol + 32 * hf;
+                tmem_ld16x256_x4x2(ta, ta + (16u << 16), v);
+                tc_before();
                 __syncwarp();
-#pragma unroll 1
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t v[32];
-                    const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * 256 + ocol + 32 * hf;
-                    tmem_ld16x256_x4x2(ta, ta + (16u << 16), v);
-                    if (hf == 1) {   // the accumulator is in registers: free the slot
-                        tc_before();
-                        __syncwarp();
-                        if (lane == 0) bar_arrive(TFREE + 8 * tb);
-                    }
-                    // v[16 L + 4 j + i] = D[c = 16 L + lane / 4 + 8 (i >> 1)][tok = 8 j + 2 (lane % 4) + (i & 1)]
-                    const uint32_t obs = obs0 + hf * L::OBUF;
+                if (lane == 0) {   // the accumulator and the normalisers are in registers: free both slots
+                    bar_arrive(TFREE + 8 * tb);
+                    bar_arrive(GFREE + 8 * gt);
+                    bulk_wait_read0();   // this warp's previous store has read its box
+                }
+                __syncwarp();
+                // v[16 L + 4 j + i] = D[c = 16 L + lane / 4 + 8 (i >> 1)][tok = 8 j + 2 (lane % 4) + (i & 1)];
+                // row c's inverse scale is rinv[2 L + (i >> 1)]
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int tok = 8 * j + smk;
-                        stsm4_trans(obs + tok * 64 + ((smm ^ ((tok >> 1) & 3)) << 4),
-                                    pack_bf2(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1])),
-                                    pack_bf2(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])),
-                                    pack_bf2(__uint_as_float(v[16 + 4 * j]), __uint_as_float(v[16 + 4 * j + 1])),
-                                    pack_bf2(__uint_as_float(v[16 + 4 * j + 2]), __uint_as_float(v[16 + 4 * j + 3])));
-                    }
-                    if (nt == T) {
-                        fence_async_smem();
-                        __syncwarp();
-                        if (lane == 0 && head < HV) tma_store3_hint(&mo, obs, LCLA_D * head, t + 32 * hf, x.b, stream_pol);
-                    } else {   // ragged tile: lane = token, its 64-byte row back from the box to global memory
-                        __syncwarp();
-                        const int tok = lane;
-                        if (head < HV && 32 * hf + tok < nt) {
-                            const unsigned char *row = obp0 + hf * L::OBUF + tok * 64;
-                            uint4 *gp = reinterpret_cast<uint4 *>(out + ((size_t)x.b * p.N + t + 32 * hf + tok) * tstride +
-                                                                  (size_t)head * LCLA_D);
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t pk[4];
 #pragma unroll
-                            for (int m = 0; m < 4; ++m) gp[m] = lds128(row + ((m ^ ((tok >> 1) & 3)) << 4));
-                        }
-                        __syncwarp();
+                    for (int rr = 0; rr < 4; ++rr) {   // rr = 2 L + (i >> 1)
+                        const int base = 16 * (rr >> 1) + 4 * j + 2 * (rr & 1);
+                        const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(v[base]), __uint_as_float(v[base + 1])),
+                                                     __fmul2_rn(gn[j], make_float2(rinv[rr], rinv[rr])));
+                        pk[rr] = pack_bf2(o2.x, o2.y);
                     }
+                    const int tok = 8 * j + smk;
+                    stsm4_trans(obs + tok * 64 + ((smm ^ ((tok >> 1) & 3)) << 4), pk[0], pk[1], pk[2], pk[3]);
+                }
+                if (nt == T) {
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && head < HV) tma_store3_hint(&mo, obs, LCLA_D * head, t + 32 * hf, x.b, stream_pol);
+                } else {   // ragged tile: lane = token, its 64-byte row back from the box to global memory
+                    __syncwarp();
+                    const int tok = lane;
+                    if (head < HV && 32 * hf + tok < nt) {
+                        const unsigned char *row = obp + tok * 64;
+                        uint4 *gp = reinterpret_cast<uint4 *>(out + ((size_t)x.b * p.N + t + 32 * hf + tok) * tstride +
+                                                              (size_t)head * LCLA_D);
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) gp[m] = lds128(row + ((m ^ ((tok >> 1) & 3)) << 4));
+                    }
+                    __syncwarp();
                 }
                 if (lane == 0) bulk_commit();
             }
