@@ -687,7 +687,8 @@ def time_forward(lcla, spec, inputs, out, st, ws, stream, device, K, W, ranks, c
     nseg, npref = plan["segments"], plan["prefixes"]
     sl = spec.B * spec.H * (spec.d + 1) * spec.d * 4
     bytes_a = 2 * tok_bytes + tab_bytes + nseg * sl
-    bytes_c = 2 * tok_bytes + tab_bytes + npref * sl
+    # chunk mode re-reads k and v in pass C for the in-tile term
+    bytes_c = (4 if plan["chunk_mode"] else 2) * tok_bytes + tab_bytes + npref * sl
     bytes_s = nseg * sl + npref * sl + sl
     # the grouped scan serves plans with at most 256 prefix groups (blocks, or segments in chunk mode);
     # larger plans scan in chunks with two kernels, timed together

@@ -292,6 +292,9 @@ NAMED = {
     # linear_head_dim 64 at the same model width (35 heads x 64 = 2240)
     "fwd480p_d64_bf16": Spec("fwd480p_d64_bf16", 1, 35, 21 * 30 * 52, 64, 3 * 30 * 52, "bf16", 12,
                              rope="3d", grid=(21, 30, 52)),
+    # the same latent with fp32 inputs (the CUDA-core head-dim-64 passes)
+    "fwd480p_d64_f32": Spec("fwd480p_d64_f32", 1, 35, 21 * 30 * 52, 64, 3 * 30 * 52, "f32", 13,
+                            rope="3d", grid=(21, 30, 52)),
 }
 for _i, _L in enumerate((1, 64, 1560, 4680, 65536)):
     for _dt in ("f32", "bf16"):
