@@ -279,6 +279,20 @@ bool map_table(CUtensorMap *m, const float *base, int N, int d)
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Pass C at d = 32 splits its registers between warpgroups (setmaxnreg): the
+// split adds up only if the kernel launches at exactly LayC<32>::REG_LAUNCH
+// registers a thread, so it is not launched otherwise.
+bool pass_c_launch_limit_ok()
+{
+    static const bool ok = [] {
+        cudaFuncAttributes a;
+        return cudaFuncGetAttributes(&a, lcla::tc::pass_c_tc<LCLA_D>) == cudaSuccess &&
+               a.numRegs == lcla::tc::LayC<LCLA_D>::REG_LAUNCH &&
+               a.maxThreadsPerBlock >= lcla::tc::LayC<LCLA_D>::NTHREADS;
+    }();
+    return ok;
+}
+
 // Tensor-core path: returns false (nothing enqueued) when a tensor map cannot
 // be encoded, so that the caller can run the CUDA-core kernels instead.  At
 // d = 64 the tensors are mapped as 2H virtual heads of 32 dims.
@@ -296,6 +310,10 @@ bool launch_tc(const void *q, const void *k, const void *v, const float *rc, con
         return false;
     using LA = lcla::tc::LayA<DW>;
     using LC = lcla::tc::LayC<DW>;
+    if (DW == LCLA_D && c && !pass_c_launch_limit_ok()) {   // nothing enqueued
+        *rc_out = LCLA_ERR_CUDA;
+        return true;
+    }
     float *part = reinterpret_cast<float *>(ws + p.part_off);
     float *pref = reinterpret_cast<float *>(ws + p.pref_off);
     int *status = reinterpret_cast<int *>(ws);

@@ -109,7 +109,7 @@ __device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity)
 }
 // Slow path of bar_wait: keep trying until the phase completes, the CTA's
 // abort flag is set, or LCLA_TC_WAIT_NS pass (then set the flag).
-__device__ __noinline__ bool bar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+__device__ __forceinline__ bool bar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag)
 {
     const uint64_t t0 = gtimer();
     for (;;) {
@@ -160,12 +160,25 @@ __device__ __forceinline__ void ring_next(Ring &r)
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// Per-thread register limit of the executing warpgroup (every warp of it executes the same one): dec returns
+// registers to the CTA's pool, inc takes them from it (and waits until they are there).
+template <int N> __device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N> __device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
 __device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y, int z)
 {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(x), "r"(y), "r"(z)
         : "memory");
+}
+
+// Plain bulk copy of `bytes` contiguous bytes (addresses 16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"((uint64_t)src), "r"(bytes), "r"(bar)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tma_load2(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y)
@@ -583,10 +596,11 @@ __device__ __forceinline__ void produce_boxes(const LclaPlan &p, int nunits, uin
 
 // Rotary rows: per tile, the tile's rows of the cos and sin tables into the
 // table ring (DW = 64: columns 0-15 and 16-31 of each, one box per half).
-template <int DW, int NTS>
+// after(x, i) runs once each tile's rows are issued; false gives up.
+template <int DW, int NTS, typename After>
 __device__ __forceinline__ void produce_tables(const LclaPlan &p, int nunits, uint32_t tab0, uint32_t CFULL,
                                                uint32_t CEMPTY, const CUtensorMap *mc, const CUtensorMap *ms,
-                                               volatile int *abort_flag)
+                                               volatile int *abort_flag, After &&after)
 {
     constexpr int TB = Width<DW>::TAB_BYTES, VPH = Width<DW>::VPH;
     Ring cr = {0, 1u};
@@ -609,6 +623,10 @@ __device__ __forceinline__ void produce_tables(const LclaPlan &p, int nunits, ui
             }
             ring_next<NTS>(cr);
             ++issued;
+            if (!after(x, i)) {
+                ok = false;
+                break;
+            }
         }
     }
     if (!ok)
@@ -713,7 +731,9 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
         }
     } else if (w == L::W_TAB) {
         // ---------------- producer: rotary rows of each tile ----------------
-        if (lane == 0) produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag);
+        if (lane == 0)
+            produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag,
+                                   [](const Unit &, int) { return true; });
     } else if (w == L::W_MMA) {
         // ---------------- MMA issuer: one accumulator per chunk of CHUNK tiles ----------------
         if (lane == 0) {
@@ -936,8 +956,11 @@ struct LayC {
     // raw q ring: one tile's two TMA boxes [64 tok][2 heads x 32] bf16 (16 KB) per slot, released when the
     // prologue has used it; operand ring: the tile's query operand, 4 atoms of [64 rows (tok)][32 fp16]
     // (64-byte swizzle, 16 KB), held until the tile's MMAs complete.  DW = 64 has table slots twice as large.
-    static constexpr int RAW = DW == 32 ? 6 : 5, RAW_BYTES = 16384;
-    static constexpr int OPS = 2, OP_BYTES = 16384, ATOM = 4096;
+    static constexpr int RAW = 5, RAW_BYTES = 16384;
+    // prologue: groups of 4 warps that take turns on the tiles (three at DW = 32, two at DW = 64), so that one
+    // group's waits, fences and load latencies overlap the others' arithmetic; one operand slot per group
+    static constexpr int NGRP = DW == 32 ? 3 : 2, GW = 4, NPC = GW * NGRP, RPT = NPRO / GW;
+    static constexpr int OPS = NGRP, OP_BYTES = 16384, ATOM = 4096;
     static constexpr int RAW_OFF = 0, OP_OFF = RAW * RAW_BYTES;
     static constexpr int TAB_BYTES = Width<DW>::TAB_BYTES;
     static constexpr int NT = DW == 32 ? 5 : 3;                     // rotary-table ring slots
@@ -950,27 +973,40 @@ struct LayC {
     static constexpr int OBUF = 2048;
     // the normaliser 1 / (z . phi(q) + eps) of each tile, [4 virtual heads][64 tok] fp32, from the prologue to the
     // epilogue; and the inverse row scales of each prefix operand, [2][128] fp32
-    static constexpr int NG = 4, G_BYTES = 1024;
+    static constexpr int NG = 2 * NGRP, G_BYTES = 1024;
     static constexpr int G_OFF = O_OFF + 8 * OBUF;
     static constexpr int S_OFF = G_OFF + NG * G_BYTES;
-    static constexpr int CTRL = S_OFF + 2 * 128 * 4;                // mbarriers, tensor-memory slot, abort flag
+    // DW = 32: the table producer copies each unit's prefix states ahead of time, S into the prefix operand buffer
+    // the unit will use (the prologue converts it in place: a row's raw fp32 and its fp16 hi | lo both take 128 B)
+    // and z here, [2][4 heads][32] fp32
+    static constexpr int Z_OFF = S_OFF + 2 * 128 * 4, Z_BYTES = 512;
+    static constexpr int CTRL = Z_OFF + (DW == 32 ? 2 * Z_BYTES : 0);  // mbarriers, tensor-memory slot, abort flag
     static constexpr int BYTES = CTRL + CTRL_BYTES + 1024;          // + worst-case 1024-byte alignment pad
-    // prologue: 8 warps in two groups of 4 that take alternate tiles, so that one group's waits, fences and
-    // load latencies overlap the other's arithmetic; a thread does four token rows of its group's tiles (the
-    // row sets that pair_offsets gives warps 4 gw .. 4 gw + 3)
-    static constexpr int NPC = 8, NGRP = 2, GW = NPC / NGRP, RPT = NPRO / GW;
-    static constexpr int NTHREADS = 608;                            // epilogue 0-7, producer 8, MMA 9, prologue 10-17,
-                                                                    // tables 18
-    static constexpr int W_PROD = 8, W_MMA = 9, W_PRO0 = 10, W_TAB = 18, NEPI = 8;
+    // a prologue thread does four token rows of its group's tiles (the row sets that pair_offsets gives warps
+    // 4 gw .. 4 gw + 3).  Warps: DW = 32, epilogue 0-7, prologue 8-19, producer 20, MMA 21, tables and prefix
+    // states 22, 23 idle: six warpgroups launched at 80 registers a thread, the prologue's three raise their limit
+    // to 96, the epilogue's two lower it to 72 and the last one to 40; DW = 64, epilogue 0-7, producer 8, MMA 9,
+    // prologue 10-17, tables 18, at one register limit.
+    static constexpr int NTHREADS = DW == 32 ? 768 : 608;
+    static constexpr int W_PROD = DW == 32 ? 20 : 8, W_MMA = W_PROD + 1, W_PRO0 = DW == 32 ? 8 : 10,
+                         W_TAB = DW == 32 ? 22 : 18, NEPI = 8;
+    static constexpr int REG_LAUNCH = 80, REG_PRO = 96, REG_EPI = 72, REG_LOW = 40;   // DW = 32
     static constexpr int NTM = 2;                                   // tensor-memory ring (256 columns each)
     static constexpr uint32_t IDESC = idesc_f16(128, 256);
     static constexpr int TMEM_COLS = NTM * 256;
-    static constexpr int NBARS = 2 * RAW + 2 * OPS + 2 * NT + 2 * NTM + 6 + 2 * NG;
+    static constexpr int NBARS = 2 * RAW + 2 * OPS + 2 * NT + 2 * NTM + 6 + 2 * NG + 2;
     static_assert(NPB * Width<DW>::VPH == 2, "two prefix operands of P_BYTES");
     static_assert(BYTES <= SMEM_MAX, "pass C shared memory");
     static_assert(8 * NBARS + 12 <= CTRL_BYTES, "pass C control block: barriers, TMEM slot, abort flag");
-    static_assert(W_TAB - W_PRO0 == NPC && NTHREADS / 32 == W_TAB + 1, "pass C prologue warps: barrier counts use NPC");
-    static_assert(GW * RPT == NPRO && OPS == NGRP, "a group's rows cover the 16 row sets; one operand slot per group");
+    static_assert(W_PRO0 + NPC <= W_PROD || W_PRO0 >= W_MMA + 1, "pass C prologue warps apart from the producers");
+    static_assert(DW != 32 || (NTHREADS == 768 && W_PRO0 == 8 && W_PROD == 20 && W_TAB == 22),
+                  "DW = 32: warpgroups 2-4 prologue, 5 producers (the register split assumes it)");
+    static_assert(DW != 32 || 128 * (REG_LAUNCH - REG_LOW) + 256 * (REG_LAUNCH - REG_EPI) >=
+                                  128 * NGRP * (REG_PRO - REG_LAUNCH),
+                  "the prologue warpgroups take no more registers than the others give up");
+    static_assert(DW != 64 || (W_TAB - W_PRO0 == NPC && NTHREADS / 32 == W_TAB + 1), "DW = 64 warp roles");
+    static_assert(NPB == 2 || DW != 32, "the prefix states are copied a unit ahead into the other prefix buffer");
+    static_assert(GW * RPT == NPRO, "a group's rows cover the 16 row sets");
     static_assert(OP_OFF % 1024 == 0 && OP_BYTES % 1024 == 0 && P_OFF % 1024 == 0, "swizzled operands: 1 KB alignment");
     static_assert(O_OFF % 1024 == 0 && OBUF % 512 == 0, "64-byte-swizzled output boxes need 512-byte alignment");
 };
@@ -1039,11 +1075,12 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
     // FULL / RAWFREE: raw q slots (TMA landed / used by the tile's prologue group); OPREADY / OPFREE: operand
     // slots (written by the group / the tile's MMAs complete); CFULL / CEMPTY: rotary rows; TFULL / TFREE:
     // accumulators; PFREE / PREADY: prefix operands (the unit's MMAs complete / staged by every prologue warp);
-    // SFREE: the prefix operand's inverse row scales read by every epilogue warp; GREADY / GFREE: normalisers
+    // SFREE: the prefix operand's inverse row scales read by every epilogue warp; GREADY / GFREE: normalisers;
+    // PRAW: a unit's raw prefix states landed (DW = 32)
     const uint32_t FULL = sb + L::CTRL, RAWFREE = FULL + 8 * R, OPREADY = RAWFREE + 8 * R, OPFREE = OPREADY + 8 * O,
                    CFULL = OPFREE + 8 * O, CEMPTY = CFULL + 8 * NT, TFULL = CEMPTY + 8 * NT, TFREE = TFULL + 8 * NTM,
                    PFREE = TFREE + 8 * NTM, PREADY = PFREE + 16, SFREE = PREADY + 16, GREADY = SFREE + 16,
-                   GFREE = GREADY + 8 * NG;
+                   GFREE = GREADY + 8 * NG, PRAW = GFREE + 8 * NG;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + L::CTRL + 8 * L::NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     float *gbuf = reinterpret_cast<float *>(sm + L::G_OFF);   // [NG][4 vh][64 tok]
@@ -1073,6 +1110,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             bar_init(PFREE + 8 * i, 1);
             bar_init(PREADY + 8 * i, L::NPC);
             bar_init(SFREE + 8 * i, L::NEPI);
+            bar_init(PRAW + 8 * i, 1);
         }
         for (int i = 0; i < NG; ++i) {
             bar_init(GREADY + 8 * i, L::GW);
@@ -1090,17 +1128,54 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
     tc_after();
     const uint32_t tmem = *tslot;
 
-    if (w == L::W_PROD) {
+    auto run_producer = [&]() {
         // ---------------- producer (q and the tables are inputs: no wait on earlier kernels) ----------------
         if (lane == 0) {
             const CUtensorMap *const maps[1] = {&mq};
             const int offs[1] = {0};
             produce_boxes<R, L::RAW_BYTES, 1, 2>(p, nunits, sb + L::RAW_OFF, FULL, RAWFREE, maps, offs, abort_flag);
         }
-    } else if (w == L::W_TAB) {
-        // ---------------- producer: rotary rows of each tile ----------------
-        if (lane == 0) produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag);
-    } else if (w == L::W_MMA) {
+    };
+    auto run_tables = [&]() {
+        // ---------------- producer: rotary rows of each tile; DW = 32, also each unit's prefix states ----------------
+        if (lane == 0) {
+            if (DW == 32) {
+                // the copy of unit k's states waits for its buffer (the MMAs of unit k - 2 done): it goes out with
+                // unit k's first table rows, a few tiles before the prologue reaches the unit, and for the first
+                // unit once the table ring is full (the states come from the previous kernel)
+                Ring br = {0, 1u};
+                int k = 0, copies = 0;
+                auto prefix_copy = [&](const Unit &x, int i) -> bool {
+                    if (i != (k == 0 ? min(NT, x.ntile) - 1 : 0)) return true;
+                    if (k++ == 0) pdl_wait();
+                    if (!bar_wait(PFREE + 8 * br.idx, br.phase, abort_flag)) return false;
+                    // the quad's heads inside H: per head S (rows c, 128 B each) and z; the prologue reads heads past
+                    // H as zeros
+                    const int nh = min(HQ, HV - HQ * x.hq);
+                    const uint32_t fb = PRAW + 8 * br.idx;
+                    const float *src = pref + (((size_t)x.blk * p.B + x.b) * p.H + HQ * x.hq) * SZ;
+                    bar_expect_tx(fb, (uint32_t)(nh * SZ * 4));
+                    for (int j = 0; j < nh; ++j) {
+                        bulk_load(sb + L::P_OFF + br.idx * L::P_BYTES + j * (DW * DW * 4), src + (size_t)j * SZ,
+                                  DW * DW * 4, fb);
+                        bulk_load(sb + L::Z_OFF + br.idx * L::Z_BYTES + j * (DW * 4), src + (size_t)j * SZ + DW * DW,
+                                  DW * 4, fb);
+                    }
+                    ring_next<L::NPB>(br);
+                    ++copies;
+                    return true;
+                };
+                produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag, prefix_copy);
+                // let the copies issued land before the CTA releases its memory (at once unless a role gave up)
+                for (int j = copies > L::NPB ? copies - L::NPB : 0; j < copies; ++j)
+                    bar_wait_quiet(PRAW + 8 * (j % L::NPB), (uint32_t)((j / L::NPB) & 1));
+            } else {
+                produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag,
+                                       [](const Unit &, int) { return true; });
+            }
+        }
+    };
+    auto run_mma = [&]() {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             Ring sr = {0, 0u}, tr = {0, 1u};   // operand ready, TMEM free
@@ -1151,16 +1226,18 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             }
             if (!ok && issued > 0) bar_wait_quiet(TFULL + 8 * last_tb, last_phase);
         }
-    } else if (w >= L::W_PRO0) {
+    };
+    auto run_prologue = [&]() {
         // ---------------- prologue: prefix staging, phi, normaliser, rotary, fp16 operand ----------------
-        // Group grp of GW warps takes the tiles whose sequence number (over this CTA's units) has parity grp and
-        // writes operand slot grp.  Thread: RPT token rows (row sets RPT gw .. RPT gw + RPT - 1 of pair_offsets),
-        // one quarter f of the 32 dims of head pair g; all its rows share g and f (lane bits).
+        // Group grp of GW warps takes the tiles whose sequence number (over this CTA's units) is grp modulo NGRP
+        // and writes operand slot grp.  Thread: RPT token rows (row sets RPT gw .. RPT gw + RPT - 1 of
+        // pair_offsets), one quarter f of the 32 dims of head pair g; all its rows share g and f (lane bits).
         const int pw = w - L::W_PRO0, pt = tid - 32 * L::W_PRO0;
         const int grp = pw / L::GW, gw = pw % L::GW;
         const int f = lane & 3, g = (lane >> 3) & 1;   // as pair_offsets gives them
         pdl_wait();   // the prefix states come from the previous kernel
-        Ring fr = {0, 0u}, cr = {0, 0u}, br = {0, 1u}, sr = {0, 1u};   // raw full, table full, P free, scales read
+        // raw full, table full, prefix buffer free (DW = 64) or its raw states landed (DW = 32), scales read
+        Ring fr = {0, 0u}, cr = {0, 0u}, br = {0, DW == 32 ? 0u : 1u}, sr = {0, 1u};
         uint32_t op_phase = 1u;                                         // operand slot grp free
         int tseq = 0;                                                   // tile sequence number
         bool ok = true;
@@ -1169,7 +1246,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             if (x.ntile == 0) continue;
             const int ub = br.idx;
             const size_t pbase = ((size_t)x.blk * p.B + x.b) * p.H;
-            bool fine = bar_wait(PFREE + 8 * br.idx, br.phase, abort_flag);
+            bool fine = bar_wait((DW == 32 ? PRAW : PFREE) + 8 * br.idx, br.phase, abort_flag);
             fine = bar_wait(SFREE + 8 * sr.idx, sr.phase, abort_flag) && fine;
             if (!__all_sync(ALL, fine)) {
                 ok = false;
@@ -1178,11 +1255,12 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             ring_next<L::NPB>(br);
             ring_next<L::NPB>(sr);
 #pragma unroll 1
-            for (int rep = 0; rep < 512 / (32 * L::NPC); ++rep) {
+            for (int rep = 0; 32 * L::NPC * rep < 512; ++rep) {
                 // the quad's prefix -> A operand rows m = (virtual head, c): [P~hi | P~lo] fp16, P~ = P times the
                 // row's power-of-two scale; thread (m, quarter qq of the 32 keys of each key half kh), the row's
                 // four threads in lanes qq = 0..3; DW = 64: row 32 (vh % 2) + c of head vh / 2, one operand per kh
                 const int ptt = pt + 32 * L::NPC * rep;
+                if (ptt >= 512) break;   // whole warps
                 const int m = ptt >> 2, qq = ptt & 3, vh = HQ * x.hq + (m >> 5);
                 float y[VPH][8];
                 float mx = 0.f;
@@ -1190,10 +1268,17 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 for (int kh = 0; kh < VPH; ++kh) {
                     float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
                     if (vh < HV) {
-                        const float4 *src = reinterpret_cast<const float4 *>(
-                            pref + (pbase + vh / VPH) * SZ + (size_t)(32 * (vh % VPH) + (m & 31)) * DW + 32 * kh + 8 * qq);
-                        a4 = src[0];
-                        b4 = src[1];
+                        if (DW == 32) {   // the raw row in place: head m / 32, row c = m % 32, 128 B
+                            const unsigned char *rowp = sm + L::P_OFF + ub * L::P_BYTES + m * 128 + qq * 32;
+                            a4 = ldsf4(rowp);
+                            b4 = ldsf4(rowp + 16);
+                        } else {
+                            const float4 *src = reinterpret_cast<const float4 *>(
+                                pref + (pbase + vh / VPH) * SZ + (size_t)(32 * (vh % VPH) + (m & 31)) * DW + 32 * kh +
+                                8 * qq);
+                            a4 = src[0];
+                            b4 = src[1];
+                        }
                     }
                     y[kh][0] = a4.x; y[kh][1] = a4.y; y[kh][2] = a4.z; y[kh][3] = a4.w;
                     y[kh][4] = b4.x; y[kh][5] = b4.y; y[kh][6] = b4.z; y[kh][7] = b4.w;
@@ -1202,6 +1287,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 }
                 mx = fmaxf(mx, __shfl_xor_sync(ALL, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(ALL, mx, 2));
+                if (DW == 32) __syncwarp();   // the row's four lanes have read it before any of them overwrites it
                 float scale, inv;
                 row_scale(mx, scale, inv);
 #pragma unroll
@@ -1220,32 +1306,39 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 }
                 if (qq == 0) sinv[ub * 128 + m] = inv;
             }
-            fence_async_smem();   // the MMAs read the prefix operand
-            __syncwarp();
-            if (lane == 0) bar_arrive(PREADY + 8 * ub);
-            // z[8f, 8f+8) of virtual heads 2g, 2g+1, as (even, odd) element vectors over pairs 0-1 and 2-3
+            // z[8f, 8f+8) of virtual heads 2g, 2g+1, as (even, odd) element vectors over pairs 0-1 and 2-3; read
+            // before the arrival on PREADY (DW = 32: the unit's MMAs completing frees the buffer for the next copy)
             float2 za01[2], za23[2], zb01[2], zb23[2];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int vh = HQ * x.hq + 2 * g + hh;
                 float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
                 if (vh < HV) {
-                    const float4 *src = reinterpret_cast<const float4 *>(pref + (pbase + vh / VPH) * SZ + DW * DW +
-                                                                         32 * (vh % VPH) + 8 * f);
-                    a4 = src[0];
-                    b4 = src[1];
+                    if (DW == 32) {
+                        const unsigned char *zp = sm + L::Z_OFF + ub * L::Z_BYTES + (2 * g + hh) * 128 + 32 * f;
+                        a4 = ldsf4(zp);
+                        b4 = ldsf4(zp + 16);
+                    } else {
+                        const float4 *src = reinterpret_cast<const float4 *>(pref + (pbase + vh / VPH) * SZ + DW * DW +
+                                                                             32 * (vh % VPH) + 8 * f);
+                        a4 = src[0];
+                        b4 = src[1];
+                    }
                 }
                 za01[hh] = make_float2(a4.x, a4.z);
                 zb01[hh] = make_float2(a4.y, a4.w);
                 za23[hh] = make_float2(b4.x, b4.z);
                 zb23[hh] = make_float2(b4.y, b4.w);
             }
+            fence_async_smem();   // the MMAs read the prefix operand
+            __syncwarp();
+            if (lane == 0) bar_arrive(PREADY + 8 * ub);
             for (int i = 0; i < x.ntile; ++i) {
                 const int rt = fr.idx, ct = cr.idx, gt = tseq % NG;
                 const uint32_t rph = fr.phase, cph = cr.phase, gph = (uint32_t)(((tseq / NG) & 1) ^ 1);
                 ring_next<R>(fr);
                 ring_next<NT>(cr);
-                if (((tseq++) & 1) != grp) continue;   // the other group's tile
+                if ((tseq++) % L::NGRP != grp) continue;   // another group's tile
                 bool fine = bar_wait(FULL + 8 * rt, rph, abort_flag);
                 fine = bar_wait(CFULL + 8 * ct, cph, abort_flag) && fine;
                 fine = bar_wait(GFREE + 8 * gt, gph, abort_flag) && fine;
@@ -1335,7 +1428,8 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 }
             }
         }
-    } else {
+    };
+    auto run_epilogue = [&]() {
         // ---------------- epilogue: tensor memory -> scaled -> bf16 -> transposed into a TMA store box ----------------
         // warp e: virtual head q = e & 3 of the quad (tensor-memory lanes 32q + c), tokens [32 hf, 32 hf + 32) of
         // the tile, hf = e >> 2.  out = accumulator x (inverse row scale of c) x (1 / (z . phi(q) + eps) of the
@@ -1432,6 +1526,37 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             }
         }
         if (lane == 0) bulk_wait_all();
+    };
+    // DW = 32: each warpgroup first sets its register limit (the host checks that the kernel launches at
+    // REG_LAUNCH): the last one (producer, MMA, tables, one idle warp) lowers it, the epilogue's two lower it a
+    // little, the prologue's three raise it by what the others gave up
+    if (DW == 32) {
+        if (w >= L::W_PROD) {
+            setmaxnreg_dec<L::REG_LOW>();
+            if (w == L::W_PROD)
+                run_producer();
+            else if (w == L::W_MMA)
+                run_mma();
+            else if (w == L::W_TAB)
+                run_tables();
+        } else if (w >= L::W_PRO0) {
+            setmaxnreg_inc<L::REG_PRO>();
+            run_prologue();
+        } else {
+            setmaxnreg_dec<L::REG_EPI>();
+            run_epilogue();
+        }
+    } else {
+        if (w == L::W_PROD)
+            run_producer();
+        else if (w == L::W_TAB)
+            run_tables();
+        else if (w == L::W_MMA)
+            run_mma();
+        else if (w >= L::W_PRO0)
+            run_prologue();
+        else
+            run_epilogue();
     }
 
     tc_before();
