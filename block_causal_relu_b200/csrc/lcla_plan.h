@@ -59,10 +59,10 @@ struct LclaSeg {
 
 LCLA_HD int lcla_min_i(int a, int b) { return a < b ? a : b; }
 
-// Token range of segment s.  N <= 2^30 (the API rejects larger N), so block
-// starts and token counts fit in 32 bits; the tile split nt * j / nsb is taken
-// in 64 bits and its result, at most nt, is multiplied by the tile length only
-// where that stays within the block length.
+// Token range of segment s.  All arithmetic fits in 32 bits: N <= 2^30 (the
+// API rejects larger N), so block starts, token counts and j * per stay below
+// 2^30 before the final multiply by the tile length, which is bounded by the
+// block length.
 LCLA_HD LclaSeg lcla_segment(const LclaPlan &p, int s)
 {
     LclaSeg g;
@@ -78,10 +78,10 @@ LCLA_HD LclaSeg lcla_segment(const LclaPlan &p, int s)
             b0 = g.blk * p.L;
             bl = lcla_min_i(p.L, p.N - b0);
         }
-        // the block's nt tiles split as evenly as whole tiles allow: segment j ends at tile nt (j + 1) / nsb
-        const long long nt = (bl + p.T - 1) / p.T;
-        g.t0 = b0 + lcla_min_i((int)(nt * j / p.nsb) * p.T, bl);
-        g.t1 = b0 + lcla_min_i((int)(nt * (j + 1) / p.nsb) * p.T, bl);
+        const int nt = (bl + p.T - 1) / p.T;               // tiles in this block
+        const int per = (nt + p.nsb - 1) / p.nsb;          // tiles per segment
+        g.t0 = b0 + lcla_min_i(lcla_min_i(j * per, nt) * p.T, bl);
+        g.t1 = b0 + lcla_min_i(lcla_min_i((j + 1) * per, nt) * p.T, bl);
     } else {
         const int span = p.tps * p.T;
         g.t0 = s < p.nseg ? lcla_min_i(s * span, p.N) : p.N;   // (nseg - 1) * span < N + T

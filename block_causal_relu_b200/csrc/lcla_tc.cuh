@@ -109,7 +109,7 @@ __device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity)
 }
 // Slow path of bar_wait: keep trying until the phase completes, the CTA's
 // abort flag is set, or LCLA_TC_WAIT_NS pass (then set the flag).
-__device__ __forceinline__ bool bar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+__device__ __forceinline__ bool bar_wait_slow_body(uint32_t bar, uint32_t parity, volatile int *abort_flag)
 {
     const uint64_t t0 = gtimer();
     for (;;) {
@@ -121,17 +121,26 @@ __device__ __forceinline__ bool bar_wait_slow(uint32_t bar, uint32_t parity, vol
         }
     }
 }
+// Out of line, so that the rare slow path does not grow every wait site.
+__device__ __noinline__ bool bar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    return bar_wait_slow_body(bar, parity, abort_flag);
+}
 // Bounded wait for the phase with the given parity to complete; gives up when
-// the CTA's abort flag is set.  Sets the flag itself on timeout.
+// the CTA's abort flag is set.  Sets the flag itself on timeout.  INL: the slow
+// path inline, for code that runs under a setmaxnreg limit (no calls there).
+template <bool INL = false>
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
 {
+    if (INL) return bar_try(bar, parity) || bar_wait_slow_body(bar, parity, abort_flag);
     return bar_try(bar, parity) || bar_wait_slow(bar, parity, abort_flag);
 }
 // Bounded wait that ignores the abort flag (used to let in-flight work land).
+template <bool INL = false>
 __device__ __forceinline__ void bar_wait_quiet(uint32_t bar, uint32_t parity)
 {
     volatile int never = 0;
-    bar_wait(bar, parity, &never);
+    bar_wait<INL>(bar, parity, &never);
 }
 __device__ __forceinline__ void bar_arrive(uint32_t bar)
 {
@@ -562,7 +571,7 @@ struct Width {
 // Input boxes: per tile, TMA loads of the quad's boxes into the stage ring
 // (NBOX boxes of [64 token][4 / NBOX heads] per tensor map, heads past H read
 // as zeros).  On abort, waits (bounded) for the loads already issued.
-template <int S, int STAGE, int NMAP, int NBOX>
+template <int S, int STAGE, int NMAP, int NBOX, bool INL = false>
 __device__ __forceinline__ void produce_boxes(const LclaPlan &p, int nunits, uint32_t sb, uint32_t FULL, uint32_t EMPTY,
                                               const CUtensorMap *const (&maps)[NMAP], const int (&offs)[NMAP],
                                               volatile int *abort_flag)
@@ -576,7 +585,7 @@ __device__ __forceinline__ void produce_boxes(const LclaPlan &p, int nunits, uin
         const int x0 = HQ * LCLA_D * x.hq;
         for (int i = 0; i < x.ntile; ++i) {
             const int t = x.t0 + i * T;
-            if (!bar_wait(EMPTY + 8 * er.idx, er.phase, abort_flag)) {
+            if (!bar_wait<INL>(EMPTY + 8 * er.idx, er.phase, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -594,13 +603,13 @@ __device__ __forceinline__ void produce_boxes(const LclaPlan &p, int nunits, uin
     }
     if (!ok)   // let the copies already issued land before the CTA releases its memory
         for (int j = issued > S ? issued - S : 0; j < issued; ++j)
-            bar_wait_quiet(FULL + 8 * (j % S), (uint32_t)((j / S) & 1));
+            bar_wait_quiet<INL>(FULL + 8 * (j % S), (uint32_t)((j / S) & 1));
 }
 
 // Rotary rows: per tile, the tile's rows of the cos and sin tables into the
 // table ring (DW = 64: columns 0-15 and 16-31 of each, one box per half).
 // after(x, i) runs once each tile's rows are issued; false gives up.
-template <int DW, int NTS, typename After>
+template <int DW, int NTS, bool INL, typename After>
 __device__ __forceinline__ void produce_tables(const LclaPlan &p, int nunits, uint32_t tab0, uint32_t CFULL,
                                                uint32_t CEMPTY, const CUtensorMap *mc, const CUtensorMap *ms,
                                                volatile int *abort_flag, After &&after)
@@ -613,7 +622,7 @@ __device__ __forceinline__ void produce_tables(const LclaPlan &p, int nunits, ui
         const Unit x = unit_at(p, u);
         for (int i = 0; i < x.ntile; ++i) {
             const int t = x.t0 + i * T;
-            if (!bar_wait(CEMPTY + 8 * cr.idx, cr.phase, abort_flag)) {
+            if (!bar_wait<INL>(CEMPTY + 8 * cr.idx, cr.phase, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -634,7 +643,7 @@ __device__ __forceinline__ void produce_tables(const LclaPlan &p, int nunits, ui
     }
     if (!ok)
         for (int j = issued > NTS ? issued - NTS : 0; j < issued; ++j)
-            bar_wait_quiet(CFULL + 8 * (j % NTS), (uint32_t)((j / NTS) & 1));
+            bar_wait_quiet<INL>(CFULL + 8 * (j % NTS), (uint32_t)((j / NTS) & 1));
 }
 
 // ---------------------------------------------------------------------------
@@ -735,8 +744,8 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
     } else if (w == L::W_TAB) {
         // ---------------- producer: rotary rows of each tile ----------------
         if (lane == 0)
-            produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag,
-                                   [](const Unit &, int) { return true; });
+            produce_tables<DW, NT, false>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag,
+                                          [](const Unit &, int) { return true; });
     } else if (w == L::W_MMA) {
         // ---------------- MMA issuer: one accumulator per chunk of CHUNK tiles ----------------
         if (lane == 0) {
@@ -1067,6 +1076,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
           const float *__restrict__ pref, const float eps, __nv_bfloat16 *__restrict__ out, int *__restrict__ status)
 {
     using L = LayC<DW>;
+    constexpr bool INL = DW == 32;   // the register split: no calls in the role code
     constexpr int R = L::RAW, O = L::OPS, NTM = L::NTM, VPH = Width<DW>::VPH, TB = L::TAB_BYTES, SZ = Width<DW>::SZ;
     constexpr int NT = L::NT, NG = L::NG;
     const int HV = p.H * VPH;   // virtual heads
@@ -1136,7 +1146,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         if (lane == 0) {
             const CUtensorMap *const maps[1] = {&mq};
             const int offs[1] = {0};
-            produce_boxes<R, L::RAW_BYTES, 1, 2>(p, nunits, sb + L::RAW_OFF, FULL, RAWFREE, maps, offs, abort_flag);
+            produce_boxes<R, L::RAW_BYTES, 1, 2, INL>(p, nunits, sb + L::RAW_OFF, FULL, RAWFREE, maps, offs, abort_flag);
         }
     };
     auto run_tables = [&]() {
@@ -1151,7 +1161,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 auto prefix_copy = [&](const Unit &x, int i) -> bool {
                     if (i != (k == 0 ? min(NT, x.ntile) - 1 : 0)) return true;
                     if (k++ == 0) pdl_wait();
-                    if (!bar_wait(PFREE + 8 * br.idx, br.phase, abort_flag)) return false;
+                    if (!bar_wait<INL>(PFREE + 8 * br.idx, br.phase, abort_flag)) return false;
                     // the quad's heads inside H: per head S (rows c, 128 B each) and z; the prologue reads heads past
                     // H as zeros
                     const int nh = min(HQ, HV - HQ * x.hq);
@@ -1168,12 +1178,12 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     ++copies;
                     return true;
                 };
-                produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag, prefix_copy);
+                produce_tables<DW, NT, INL>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag, prefix_copy);
                 // let the copies issued land before the CTA releases its memory (at once unless a role gave up)
                 for (int j = copies > L::NPB ? copies - L::NPB : 0; j < copies; ++j)
-                    bar_wait_quiet(PRAW + 8 * (j % L::NPB), (uint32_t)((j / L::NPB) & 1));
+                    bar_wait_quiet<INL>(PRAW + 8 * (j % L::NPB), (uint32_t)((j / L::NPB) & 1));
             } else {
-                produce_tables<DW, NT>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag,
+                produce_tables<DW, NT, INL>(p, nunits, sb + L::C_OFF, CFULL, CEMPTY, &mc, &ms, abort_flag,
                                        [](const Unit &, int) { return true; });
             }
         }
@@ -1191,15 +1201,15 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const Unit x = unit_at(p, u);
                 if (x.ntile == 0) continue;
-                if (!bar_wait(PREADY + 8 * pr.idx, pr.phase, abort_flag)) {
+                if (!bar_wait<INL>(PREADY + 8 * pr.idx, pr.phase, abort_flag)) {
                     ok = false;
                     break;
                 }
                 ring_next<L::NPB>(pr);
                 const uint64_t pd = pdesc0 + (uint64_t)((ub * L::P_BYTES) >> 4);
                 for (int i = 0; i < x.ntile; ++i) {
-                    if (!bar_wait(OPREADY + 8 * sr.idx, sr.phase, abort_flag) ||
-                        !bar_wait(TFREE + 8 * tr.idx, tr.phase, abort_flag)) {
+                    if (!bar_wait<INL>(OPREADY + 8 * sr.idx, sr.phase, abort_flag) ||
+                        !bar_wait<INL>(TFREE + 8 * tr.idx, tr.phase, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -1227,7 +1237,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 }
                 ub = (ub + 1) % L::NPB;
             }
-            if (!ok && issued > 0) bar_wait_quiet(TFULL + 8 * last_tb, last_phase);
+            if (!ok && issued > 0) bar_wait_quiet<INL>(TFULL + 8 * last_tb, last_phase);
         }
     };
     auto run_prologue = [&]() {
@@ -1249,8 +1259,8 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             if (x.ntile == 0) continue;
             const int ub = br.idx;
             const size_t pbase = ((size_t)x.blk * p.B + x.b) * p.H;
-            bool fine = bar_wait((DW == 32 ? PRAW : PFREE) + 8 * br.idx, br.phase, abort_flag);
-            fine = bar_wait(SFREE + 8 * sr.idx, sr.phase, abort_flag) && fine;
+            bool fine = bar_wait<INL>((DW == 32 ? PRAW : PFREE) + 8 * br.idx, br.phase, abort_flag);
+            fine = bar_wait<INL>(SFREE + 8 * sr.idx, sr.phase, abort_flag) && fine;
             if (!__all_sync(ALL, fine)) {
                 ok = false;
                 break;
@@ -1342,9 +1352,9 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                 ring_next<R>(fr);
                 ring_next<NT>(cr);
                 if ((tseq++) % L::NGRP != grp) continue;   // another group's tile
-                bool fine = bar_wait(FULL + 8 * rt, rph, abort_flag);
-                fine = bar_wait(CFULL + 8 * ct, cph, abort_flag) && fine;
-                fine = bar_wait(GFREE + 8 * gt, gph, abort_flag) && fine;
+                bool fine = bar_wait<INL>(FULL + 8 * rt, rph, abort_flag);
+                fine = bar_wait<INL>(CFULL + 8 * ct, cph, abort_flag) && fine;
+                fine = bar_wait<INL>(GFREE + 8 * gt, gph, abort_flag) && fine;
                 if (!__all_sync(ALL, fine)) {
                     ok = false;
                     break;
@@ -1360,7 +1370,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
 #pragma unroll
                 for (int k = 0; k < L::RPT; ++k) {
                     if (k == L::RPT / 2) {
-                        slot_ok = __all_sync(ALL, bar_wait(OPFREE + 8 * grp, op_phase, abort_flag));
+                        slot_ok = __all_sync(ALL, bar_wait<INL>(OPFREE + 8 * grp, op_phase, abort_flag));
                         if (!slot_ok) break;
                         op_phase ^= 1u;
 #pragma unroll
@@ -1456,7 +1466,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             const int head = HQ * x.hq + q;
             // this lane's accumulator rows c = lane / 4 + 8 k: their inverse scales
             const int sb_idx = pr.idx;
-            if (!__all_sync(ALL, bar_wait(PREADY + 8 * pr.idx, pr.phase, abort_flag))) {
+            if (!__all_sync(ALL, bar_wait<INL>(PREADY + 8 * pr.idx, pr.phase, abort_flag))) {
                 ok = false;
                 break;
             }
@@ -1468,8 +1478,8 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
             if (lane == 0) bar_arrive(SFREE + 8 * sb_idx);
             for (int i = 0; i < x.ntile; ++i) {
                 const int tb = tr.idx, gt = gr.idx;
-                bool fine = bar_wait(TFULL + 8 * tr.idx, tr.phase, abort_flag);
-                fine = bar_wait(GREADY + 8 * gr.idx, gr.phase, abort_flag) && fine;
+                bool fine = bar_wait<INL>(TFULL + 8 * tr.idx, tr.phase, abort_flag);
+                fine = bar_wait<INL>(GREADY + 8 * gr.idx, gr.phase, abort_flag) && fine;
                 if (!__all_sync(ALL, fine)) {
                     ok = false;
                     break;
