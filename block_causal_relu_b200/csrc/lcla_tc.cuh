@@ -979,7 +979,9 @@ struct LayC {
     static constexpr int C_OFF = OP_OFF + OPS * OP_BYTES;           // rotary-table ring
     // prefix operands [128 rows (virtual head, c)][P hi | P lo] fp16, each row scaled by a power of two: DW = 32,
     // one per unit, double-buffered; DW = 64, the unit's two key halves (e < 32, e >= 32) in one buffer
-    static constexpr int P_BYTES = 16384, NPB = DW == 32 ? 2 : 1;
+    // DW = 64: two key halves (e < 32, e >= 32) per unit, each [128 rows][P~] as one fp16 term (64-byte swizzle,
+    // 8 KB); both widths double-buffered
+    static constexpr int P_BYTES = 16384, NPB = 2, PH_BYTES = 8192, VPH_C = Width<DW>::VPH;
     static constexpr int P_OFF = C_OFF + NT * TAB_BYTES;
     static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 8 warps x [32 tok][32 c] bf16
     static constexpr int OBUF = 2048;
@@ -1007,7 +1009,7 @@ struct LayC {
     static constexpr uint32_t IDESC = idesc_f16(128, 256);
     static constexpr int TMEM_COLS = NTM * 256;
     static constexpr int NBARS = 2 * RAW + 2 * OPS + 2 * NT + 2 * NTM + 6 + 2 * NG + 2;
-    static_assert(NPB * Width<DW>::VPH == 2, "two prefix operands of P_BYTES");
+    static_assert(NPB == 2 && VPH_C * PH_BYTES <= P_BYTES, "two prefix buffers of P_BYTES");
     static_assert(BYTES <= SMEM_MAX, "pass C shared memory");
     static_assert(8 * NBARS + 12 <= CTRL_BYTES, "pass C control block: barriers, TMEM slot, abort flag");
     static_assert(W_PRO0 + NPC <= W_PROD || W_PRO0 >= W_MMA + 1, "pass C prologue warps apart from the producers");
@@ -1192,7 +1194,7 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             Ring sr = {0, 0u}, tr = {0, 1u};   // operand ready, TMEM free
-            const uint64_t pdesc0 = desc_sw128(sb + L::P_OFF, 16, 1024);
+            const uint64_t pdesc0 = DW == 32 ? desc_sw128(sb + L::P_OFF, 16, 1024) : desc_sw64(sb + L::P_OFF, 16, 512);
             const uint64_t qdesc0 = desc_sw64(sb + L::OP_OFF, 16, 512);
             int ub = 0, issued = 0, last_tb = 0;
             uint32_t last_phase = 0;
@@ -1216,15 +1218,20 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     tc_after();
                     const uint32_t d = tmem + tr.idx * 256;
                     const uint64_t bd0 = qdesc0 + (uint64_t)((sr.idx * L::OP_BYTES) >> 4);
-#pragma unroll
-                    for (int kh = 0; kh < VPH; ++kh) {   // DW = 64: key half kh of P against the operand from atom 2 kh
-                        const uint64_t pk = pd + (uint64_t)((kh * L::P_BYTES) >> 4);
-                        const uint64_t bd = bd0 + (uint64_t)((kh * 2 * L::ATOM) >> 4);
+                    if (DW == 32) {
                         // K steps of 16 elements = 32 B = 2 descriptor units; P hi at +0, P lo at +64 B
-                        mma_bf16(d, pk + 0, bd + 0, L::IDESC, kh);   // P~hi . q~
-                        mma_bf16(d, pk + 2, bd + 2, L::IDESC, 1);
-                        mma_bf16(d, pk + 4, bd + 0, L::IDESC, 1);    // P~lo . q~
-                        mma_bf16(d, pk + 6, bd + 2, L::IDESC, 1);
+                        mma_bf16(d, pd + 0, bd0 + 0, L::IDESC, 0);   // P~hi . q~
+                        mma_bf16(d, pd + 2, bd0 + 2, L::IDESC, 1);
+                        mma_bf16(d, pd + 4, bd0 + 0, L::IDESC, 1);   // P~lo . q~
+                        mma_bf16(d, pd + 6, bd0 + 2, L::IDESC, 1);
+                    } else {
+#pragma unroll
+                        for (int kh = 0; kh < VPH; ++kh) {   // key half kh of P against the operand from atom 2 kh
+                            const uint64_t pk = pd + (uint64_t)((kh * L::PH_BYTES) >> 4);
+                            const uint64_t bd = bd0 + (uint64_t)((kh * 2 * L::ATOM) >> 4);
+                            mma_bf16(d, pk + 0, bd + 0, L::IDESC, kh);
+                            mma_bf16(d, pk + 2, bd + 2, L::IDESC, 1);
+                        }
                     }
                     mma_commit(TFULL + 8 * tr.idx);
                     mma_commit(OPFREE + 8 * sr.idx);
@@ -1310,12 +1317,18 @@ pass_c_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtens
                     for (int j = 0; j < 4; ++j) {
                         const float a = y[kh][2 * j] * scale, b = y[kh][2 * j + 1] * scale;   // exact
                         const __half2 h2 = __floats2half2_rn(a, b);
-                        const float2 hf = __half22float2(h2);
-                        const __half2 l2 = __floats2half2_rn(a - hf.x, b - hf.y);
                         hw[j] = *reinterpret_cast<const uint32_t *>(&h2);
-                        lw[j] = *reinterpret_cast<const uint32_t *>(&l2);
+                        if (DW == 32) {
+                            const float2 hf = __half22float2(h2);
+                            const __half2 l2 = __floats2half2_rn(a - hf.x, b - hf.y);
+                            lw[j] = *reinterpret_cast<const uint32_t *>(&l2);
+                        }
                     }
-                    store_quarter_hi_lo(sm + L::P_OFF + (ub + kh) * L::P_BYTES, m, qq, hw, lw);
+                    if (DW == 32)
+                        store_quarter_hi_lo(sm + L::P_OFF + ub * L::P_BYTES, m, qq, hw, lw);
+                    else   // DW = 64: one fp16 term, key half kh: [128 rows][32 fp16], 64-byte swizzle
+                        *reinterpret_cast<uint4 *>(sm + L::P_OFF + ub * L::P_BYTES + kh * L::PH_BYTES + sw64(m, qq)) =
+                            make_uint4(hw[0], hw[1], hw[2], hw[3]);
                 }
                 if (qq == 0) sinv[ub * 128 + m] = inv;
             }
