@@ -12,23 +12,21 @@
 // (segment, head quad, batch entry) -- four heads of 32 -- and a tile is 64
 // tokens of those four heads.  Both kernels are persistent (one CTA per SM,
 // units c, c + gridDim.x, ..., quad fastest) and warp-specialised:
-//   producer warp   TMA loads of each tile's q or k, v boxes into a ring of
-//                   stages and of its rotary rows into a smaller table ring;
+//   box producer    TMA loads of each tile's q, or k and v, boxes into a ring;
+//   table producer  the tile's rotary rows into their own ring (pass C at
+//                   d = 32: also each unit's prefix states, a unit ahead);
 //   MMA warp        one thread issues tcgen05.mma and tcgen05.commit;
-//   prologue warps  ReLU, rotary (pass C: and the normaliser), bf16 hi + lo
-//                   split of q or k, written in
-//                   place over the stage's raw input as the MMA operand
-//                   (pass A: 8 warps, a thread doing one token quarter of all
-//                   four heads; pass C: 16 warps, one token quarter of a head
-//                   pair -- pass C's register budget is shared with its 8
-//                   epilogue warps);
+//   prologue warps  ReLU and rotary of k or q into the MMA operand (pass A:
+//                   16 warps on each tile, bf16 hi + lo written in place over
+//                   the stage's raw k; pass C: groups of 4 warps taking turns
+//                   on the tiles -- three groups at d = 32, whose registers
+//                   come from a setmaxnreg split -- one fp16 term into the
+//                   group's own operand slot, and the normaliser);
 //   drain/epilogue  tensor memory -> registers: warp w reads tensor memory
 //                   lanes 32(w & 3)..+31, which belong to head w & 3 of the
 //                   quad (pass A: 4 drain warps; pass C: 8 epilogue warps,
 //                   two per head, one per half of the tile's tokens).
-// Roles talk only through mbarriers.  A stage holds one tile from its TMA
-// load until the tile's MMAs complete; the table slot is released as soon as
-// the prologue has read it.
+// Roles talk only through mbarriers.
 //
 // Pass A.  A = V^T of the quad exactly as TMA lands it (MN-major, rows
 // (head, c)), B = the rotated keys split into bf16 hi + lo (k~ = hi + lo to
@@ -36,18 +34,22 @@
 //     D[(h', c)][(h, part, e)] = sum_tok v[tok][h', c] part(k~)[tok][h, e].
 // Warp q adds the diagonal block h = h' of every tile (hi + lo) into fp32
 // registers; the unrotated key sum z comes from the prologue's registers.
+// A stage holds one tile from its TMA load until the tile's MMAs complete.
 //
-// Pass C.  A = the block's prefix state P of the quad split into hi + lo,
-// rows (h', c), K-major [P hi | P lo]; B = the rotated queries, already
-// divided by their normaliser z . phi(q) + eps (fp32, before the split), in
-// hi + lo, rows (head, token), K-major [q~hi | q~lo]:
-//     D[(h', c)][(h, tok)] = Phi.q~hi + Plo.q~hi + Phi.q~lo   (6 MMAs of K = 16),
-// so the diagonal block h = h' is the output itself.  Epilogue warp q reads it
-// in the 16x256b fragment (two c rows x two tokens per thread), packs token
-// pairs to bf16 and writes the [32 tok][32 c] box transposed with stmatrix
-// into a 64-byte-swizzled buffer, stored by one TMA store; two epilogue warps
-// share a head, one per 32 tokens (ragged tiles: the valid rows are copied
-// out of the same buffer with plain stores).
+// Pass C.  A = the block's prefix state of the quad, each row c scaled by a
+// power of two (P~), K-major: fp16 [P~hi | P~lo] at d = 32, one fp16 term per
+// key half at d = 64; B = the rotated ReLU queries q~ as one fp16 term, rows
+// (head, token), K-major:
+//     D[(h', c)][(h, tok)] = P~ . q~   (4 MMAs of K = 16 per tile),
+// so the diagonal block h = h' is the output times the row's scale and the
+// token's normaliser z . phi(q) + eps.  The raw q slot is freed once its
+// prologue group has read it, the operand slot when the tile's MMAs complete.
+// Epilogue warp q reads the accumulator in the 16x256b fragment (two c rows x
+// two tokens per thread), multiplies by the inverse row scale and 1 / (z .
+// phi(q) + eps), packs token pairs to bf16 and writes the [32 tok][32 c] box
+// transposed with stmatrix into a 64-byte-swizzled buffer, stored by one TMA
+// store (ragged tiles: the valid rows are copied out of the same buffer with
+// plain stores).
 //
 // Every mbarrier wait is bounded (LCLA_TC_WAIT_NS of globaltimer) and gives
 // up when another role has set the CTA's abort flag; each warp makes the
@@ -977,10 +979,9 @@ struct LayC {
     static constexpr int TAB_BYTES = Width<DW>::TAB_BYTES;
     static constexpr int NT = DW == 32 ? 5 : 3;                     // rotary-table ring slots
     static constexpr int C_OFF = OP_OFF + OPS * OP_BYTES;           // rotary-table ring
-    // prefix operands [128 rows (virtual head, c)][P hi | P lo] fp16, each row scaled by a power of two: DW = 32,
-    // one per unit, double-buffered; DW = 64, the unit's two key halves (e < 32, e >= 32) in one buffer
-    // DW = 64: two key halves (e < 32, e >= 32) per unit, each [128 rows][P~] as one fp16 term (64-byte swizzle,
-    // 8 KB); both widths double-buffered
+    // prefix operands, each row scaled by a power of two (P~), one buffer per unit, double-buffered: DW = 32,
+    // [128 rows (head, c)][P~hi | P~lo] fp16 (128-byte swizzle, 16 KB); DW = 64, the unit's two key halves
+    // (e < 32, e >= 32), each [128 rows (virtual head, c)][P~] as one fp16 term (64-byte swizzle, 8 KB)
     static constexpr int P_BYTES = 16384, NPB = 2, PH_BYTES = 8192, VPH_C = Width<DW>::VPH;
     static constexpr int P_OFF = C_OFF + NT * TAB_BYTES;
     static constexpr int O_OFF = P_OFF + 2 * P_BYTES;               // output staging: 8 warps x [32 tok][32 c] bf16
