@@ -176,14 +176,6 @@ __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.a
 template <int N> __device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 template <int N> __device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
-__device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y, int z)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
-        ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(x), "r"(y), "r"(z)
-        : "memory");
-}
-
 // Plain bulk copy of `bytes` contiguous bytes (addresses 16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
 {
@@ -387,66 +379,10 @@ __device__ __forceinline__ void rope_split4(const uint32_t *fw, const float4 &c4
         lo[p] = pack_bf2(y0 - hf.x, y1 - hf.y);
     }
 }
-// rope_split4 of the features times a per-row factor g (applied in fp32, before the split).
-__device__ __forceinline__ void rope_split4_scaled(const uint32_t *fw, const float4 &c4, const float4 &s4, float g,
-                                                   uint32_t *hi, uint32_t *lo)
-{
-    const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const float a = bf_lo(fw[p]) * g, b = bf_hi(fw[p]) * g;
-        const float y0 = a * cv[p] - b * sv[p];
-        const float y1 = a * sv[p] + b * cv[p];
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
-        const float2 hf = __bfloat1622float2(h2);
-        hi[p] = bf2_bits(h2);
-        lo[p] = pack_bf2(y0 - hf.x, y1 - hf.y);
-    }
-}
-// Arrive on an mbarrier only once `dep` is known.  A warp that releases a
-// shared buffer for a TMA refill passes a value computed from its loads out of
-// that buffer (lane 0's, which returns with the whole warp's instruction) and
-// `zero`, a register holding 0 that the compiler cannot see through: the
-// barrier address then depends on the loaded data, so the arrive cannot issue
-// before the loads have returned (see release_after_use).
-__device__ __forceinline__ void bar_arrive_dep(uint32_t bar, uint32_t dep, uint32_t zero)
-{
-    bar_arrive(bar + (dep & zero));
-}
-
 // Packed bf16 -> fp32: the element in the low half, and the one in the high half.
 __device__ __forceinline__ float bf_low(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_high(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Rotate, scale and split one quarter (4 pairs) of a head on the paired fp32
-// pipes (fma/mul .f32x2, two lanes per instruction).  fw[j]: packed bf16
-// features of pair j (element 2j low, 2j+1 high); (c, s) of pairs 0-1 and
-// 2-3; g: the factor applied after the rotation.  hi[j], lo[j]: packed bf16
-// hi + lo of the rotated pair j, hi = RNE(y), lo = RNE(y - hi).
-__device__ __forceinline__ void rope_split4_x2(const uint32_t *fw, float2 c01, float2 c23, float2 s01, float2 s23,
-                                               float2 ns01, float2 ns23, float g, uint32_t *hi, uint32_t *lo)
-{
-    const float2 a01 = make_float2(bf_low(fw[0]), bf_low(fw[1])), a23 = make_float2(bf_low(fw[2]), bf_low(fw[3]));
-    const float2 b01 = make_float2(bf_high(fw[0]), bf_high(fw[1])), b23 = make_float2(bf_high(fw[2]), bf_high(fw[3]));
-    const float2 g2 = make_float2(g, g), m1 = make_float2(-1.f, -1.f);
-    // y0 = a c - b s, y1 = a s + b c, then times g
-    const float2 y0_01 = __fmul2_rn(__ffma2_rn(a01, c01, __fmul2_rn(b01, ns01)), g2);
-    const float2 y0_23 = __fmul2_rn(__ffma2_rn(a23, c23, __fmul2_rn(b23, ns23)), g2);
-    const float2 y1_01 = __fmul2_rn(__ffma2_rn(b01, c01, __fmul2_rn(a01, s01)), g2);
-    const float2 y1_23 = __fmul2_rn(__ffma2_rn(b23, c23, __fmul2_rn(a23, s23)), g2);
-    const uint32_t h0 = pack_bf2(y0_01.x, y1_01.x), h1 = pack_bf2(y0_01.y, y1_01.y);
-    const uint32_t h2 = pack_bf2(y0_23.x, y1_23.x), h3 = pack_bf2(y0_23.y, y1_23.y);
-    // y - hi, exact in fp32
-    const float2 l0_01 = __ffma2_rn(make_float2(bf_low(h0), bf_low(h1)), m1, y0_01);
-    const float2 l1_01 = __ffma2_rn(make_float2(bf_high(h0), bf_high(h1)), m1, y1_01);
-    const float2 l0_23 = __ffma2_rn(make_float2(bf_low(h2), bf_low(h3)), m1, y0_23);
-    const float2 l1_23 = __ffma2_rn(make_float2(bf_high(h2), bf_high(h3)), m1, y1_23);
-    hi[0] = h0; hi[1] = h1; hi[2] = h2; hi[3] = h3;
-    lo[0] = pack_bf2(l0_01.x, l1_01.x);
-    lo[1] = pack_bf2(l0_01.y, l1_01.y);
-    lo[2] = pack_bf2(l0_23.x, l1_23.x);
-    lo[3] = pack_bf2(l0_23.y, l1_23.y);
-}
 
 // 1 / x from the hardware approximation (relative error of a few ulp; the
 // products it scales carry bf16 operands, far coarser).
