@@ -237,46 +237,107 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
+// Encoded tensor maps of recent calls, keyed by what the map encodes (kind, base address, shape): a streaming
+// caller that reuses its buffers skips the host-side encode.  A map holds an address and a shape only, so a hit
+// is exact even when a buffer was freed and another allocated at the same address.
+class MapCache {
+  public:
+    bool get(int kind, const void *base, int a, int b, int c, CUtensorMap *m)
+    {
+        std::lock_guard<std::mutex> lock(mu_);
+        for (Entry &e : e_)
+            if (e.used && e.kind == kind && e.base == base && e.a == a && e.b == b && e.c == c) {
+                *m = e.map;
+                e.tick = ++tick_;
+                return true;
+            }
+        return false;
+    }
+    void put(int kind, const void *base, int a, int b, int c, const CUtensorMap &m)
+    {
+        std::lock_guard<std::mutex> lock(mu_);
+        Entry *v = &e_[0];
+        for (Entry &e : e_) {
+            if (!e.used) {
+                v = &e;
+                break;
+            }
+            if (e.tick < v->tick) v = &e;   // least recently used
+        }
+        *v = Entry{true, kind, base, a, b, c, ++tick_, m};
+    }
+
+  private:
+    struct Entry {
+        bool used;
+        int kind;
+        const void *base;
+        int a, b, c;
+        unsigned long long tick;
+        CUtensorMap map;
+    };
+    std::mutex mu_;
+    Entry e_[64] = {};
+    unsigned long long tick_ = 0;
+};
+MapCache &map_cache()
+{
+    static MapCache c;
+    return c;
+}
+
 // [B, N, H*d] bf16 viewed as a 3-D tensor; box = 2 heads x 64 tokens, 128-byte swizzle.
 bool map_tokens(CUtensorMap *m, const void *base, int B, int N, int H)
 {
+    if (map_cache().get(0, base, B, N, H, m)) return true;
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)H * LCLA_D, (cuuint64_t)N, (cuuint64_t)B};
     cuuint64_t strides[2] = {(cuuint64_t)H * LCLA_D * 2, (cuuint64_t)N * H * LCLA_D * 2};
     cuuint32_t box[3] = {2 * LCLA_D, LCLA_TC_T, 1};   // 128 B of a token row: 2 heads
     cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    map_cache().put(0, base, B, N, H, *m);
+    return true;
 }
 
 // [B, N, H*d] bf16 output blocks of one head x 32 tokens, 64-byte swizzle (TMA stores).
 bool map_out_blocks(CUtensorMap *m, const void *base, int B, int N, int H)
 {
+    if (map_cache().get(1, base, B, N, H, m)) return true;
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)H * LCLA_D, (cuuint64_t)N, (cuuint64_t)B};
     cuuint64_t strides[2] = {(cuuint64_t)H * LCLA_D * 2, (cuuint64_t)N * H * LCLA_D * 2};
     cuuint32_t box[3] = {LCLA_D, LCLA_TC_T / 2, 1};
     cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    map_cache().put(1, base, B, N, H, *m);
+    return true;
 }
 
 // [N, d/2] fp32 rotary table; box = 16 columns of one tile of tokens, 64-byte swizzle (d = 64: two boxes).
 bool map_table(CUtensorMap *m, const float *base, int N, int d)
 {
+    if (map_cache().get(2, base, N, d, 0, m)) return true;
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)d / 2, (cuuint64_t)N};
     cuuint64_t strides[1] = {(cuuint64_t)(d / 2) * 4};
     cuuint32_t box[2] = {LCLA_D / 2, LCLA_TC_T};
     cuuint32_t es[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    map_cache().put(2, base, N, d, 0, *m);
+    return true;
 }
 
 // Pass C at d = 32 splits its registers between warpgroups (setmaxnreg): the
@@ -320,8 +381,7 @@ bool launch_tc(const void *q, const void *k, const void *v, const float *rc, con
     const long long units = (long long)p.nseg * p.nquads * p.B;
     const dim3 grid((unsigned)(units < LCLA_TC_CTAS ? units : LCLA_TC_CTAS));
     if (a) {
-        set_smem(lcla::tc::pass_a_tc<DW>, LA::BYTES);
-        cudaMemsetAsync(status, 0, sizeof(int), st);
+        set_smem(lcla::tc::pass_a_tc<DW>, LA::BYTES);   // pass A zeroes the status word itself
         if (ev) cudaEventRecord(ev[0], st);
         lcla::tc::pass_a_tc<DW><<<grid, LA::NTHREADS, LA::BYTES, st>>>(mk, mv, mc, ms, p, part, status);
         if (ev) cudaEventRecord(ev[1], st);

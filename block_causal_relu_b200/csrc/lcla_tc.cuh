@@ -643,6 +643,9 @@ pass_a_tc(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtens
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int nunits = p.nseg * p.nquads * p.B;
 
+    // the call's status word starts at 0: pass A is the call's first kernel (launched after everything before it
+    // in the stream), and a bounded wait of this call can only give up a second after this store
+    if (blockIdx.x == 0 && tid == 0) *status = 0;
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
             bar_init(FULL + 8 * i, 1);

@@ -341,7 +341,9 @@ LCLA_API int lcla_forward_noalloc(const void *q, const void *k, const void *v,
 /*
  * Device status of a call.  The first 4 bytes of the workspace of
  * lcla_forward, lcla_forward_blocks, lcla_step and the shard calls hold an int
- * that the call zeroes first (lcla_shard_end keeps lcla_shard_begin's) and
+ * that the call zeroes first -- on the tensor-core path its first kernel does,
+ * before any of its waits can give up (lcla_shard_end keeps
+ * lcla_shard_begin's) -- and
  * that its tensor-core kernels OR bits into when one of their bounded waits
  * (1 s) gives up: bit 0 pass A, bit 1 pass C.  A CTA that gives up lets its
  * copies and MMAs in flight land, frees its tensor memory, writes NaN partial
