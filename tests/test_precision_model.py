@@ -14,6 +14,9 @@ keeps the worst output excess (beyond the output's own half-ulp, against the
 largest output of its row: the GPU tests' metric) below half the 2e-3 bar on
 robustness-style inputs -- Laplace q and k with negative rows, v of scale 2 --
 and that the one-term prefix at head dim 64 stays within the same margin.
+A second model restates pass A's key operand (bf16 hi + lo of the rotated key,
+fp32 accumulation per 64-token tile) and checks the carried state against
+its 1e-5 bar, with and without the lo term.
 It models the operand roundings, not the tensor core's accumulation order."""
 import numpy as np
 import pytest
@@ -103,3 +106,40 @@ def test_model_detects_a_coarser_query_operand():
     finally:
         f16 = saved
     assert coarse > 3 * fine, (fine, coarse)
+
+
+def model_pass_a_state(inp, hilo):
+    """Pass A's products for the whole sequence as one block: S[c][e] = sum_t v[t][c] k~[t][e] with v as
+    stored (bf16, exact), k~ = the rotated ReLU key in fp32 split into bf16 hi (+ lo), products exact and
+    accumulated in fp32 over tiles of 64 tokens (the tensor core's fp32 accumulator, one tile at a time)."""
+    k = inp.as_f32("k")[0].astype(np.float64)                  # [N, H, d]
+    v = inp.as_f32("v")[0].astype(np.float64)
+    c = inp.rope_cos.astype(np.float64)[:, None, :]
+    s = inp.rope_sin.astype(np.float64)[:, None, :]
+    fk = np.maximum(k, 0.0)
+    a, b = fk[..., 0::2], fk[..., 1::2]
+    kr = np.empty_like(fk)
+    kr[..., 0::2] = f32(a * c - b * s)
+    kr[..., 1::2] = f32(a * s + b * c)
+    hi = bf16(kr)
+    parts = [hi, bf16(kr - hi)] if hilo else [hi]
+    N, H, d = k.shape
+    S = np.zeros((H, d, d))
+    for t0 in range(0, N, 64):
+        tile = sum(np.einsum("thc,the->hce", v[t0:t0 + 64], p[t0:t0 + 64]) for p in parts)
+        S = f32(S + tile)
+    return S
+
+
+def test_pass_a_needs_the_hi_lo_key_split_for_the_state_bar():
+    # the carried state must hold 1e-5 (max |dS| / max |S|): with the bf16 hi + lo key operand the model stays
+    # well inside it, with the hi term alone it does not
+    spec = Spec("precision_model_state", 1, 4, 8192, 32, 8192, "bf16", 91,
+                qk_dist="laplace_negrows", v_sigma=2.0, rope="1d")
+    inp = make_inputs(spec)
+    _, st, _ = oracle.recurrence(inp.q, inp.k, inp.v, inp.rope_cos, inp.rope_sin, spec.block_len, spec.eps,
+                                 want_out=False)
+    S_ref = st[0, :, :32, :]
+    err = lambda S: float(np.max(np.abs(S - S_ref)) / np.max(np.abs(S_ref)))
+    assert err(model_pass_a_state(inp, True)) < 5e-6
+    assert err(model_pass_a_state(inp, False)) > 1e-5
